@@ -1,0 +1,438 @@
+#!/usr/bin/env python3
+"""Benchmark of the LLM.int8() mixed-precision decomposition matmul on B200.
+
+One step = one call of the whole forward path (outlier scan + row quantize +
+gather, int8 tcgen05 GEMM with the dequantize + fp16 outlier epilogue) on the
+6.7B-style FFN up-projection prefill: X fp16 [2048, 4096] with 6 outlier
+columns, W [4096, 16384] pre-quantized column-wise (weight conversion is
+offline, timed separately).  Metric: effective TOPS = 2*M*N*K / time.
+
+Arms:
+  (default)          this library, inputs resident in HBM; ``e2e`` adds the
+                     host->device copy of X and device->host copy of Y per step.
+  --impl reference   the CPU oracle (plain C, OpenMP) on a bounded row sample.
+Multi-GPU (torchrun): independent replicas, one per GPU (the path has no
+exchange step); value = all ranks' operations / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "effective TOPS (2MNK/s) of LLM.int8 mixed matmul; % of INT8/HBM roofline"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_PER_BF16 = 2.0  # nominal dense ratio, 4.5 POPS int8 / 2.25 PFLOP/s bf16
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=30)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="ffn_6p7b_prefill")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ peaks
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def algorithmic_bytes(M, N, K, n_o):
+    """X read + Wq read + fp16 outlier rows of W + scales + Y write."""
+    return 2 * M * K + N * K + 2 * n_o * N + 4 * (M + N) + 2 * M * N
+
+
+# ------------------------------------------------------------------ clocks
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML (read only)."""
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self.ok = True
+        except Exception as e:  # noqa: BLE001 - clocks are reported as unavailable
+            self.err = repr(e)
+        self.t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = int(self._reasons(self.h))
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self.ok:
+            self.t.join(timeout=2)
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = f"{len(win)} NVML samples inside the timed region"
+        if len(win) < 3:  # short region: widen to the samples taken under load around it
+            win = [s for s in self.samples if t0 - 1.0 <= s[0] <= t1 + 0.2]
+            note += f"; widened to {len(win)} samples within 1 s before it"
+        reasons = set()
+        for _, _, r in win:
+            for bit, name in REASON_BITS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median([s[1] for s in win]) if win else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "note": note}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, torch):
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+        else:
+            torch.cuda.set_device(0)
+
+    def barrier(self, torch):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, torch, v: float) -> float:
+        if not self.pg:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def oracle_sample(X, W, tau, rows, weight):
+    """Run the oracle's a1-a7 on the first `rows` rows; returns seconds."""
+    import oracle
+    Xs = X[:rows]
+    t0 = time.perf_counter()
+    oracle.mixed_matmul(Xs, W, tau, weight=weight)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl_, X, W, budget_s):
+    import oracle
+    weight = oracle.quantize_weight(W)  # offline conversion, not timed
+    t1 = oracle_sample(X, W, wl_.tau, 1, weight)
+    rows = int(max(1, min(wl_.M, budget_s / max(t1, 1e-6))))
+    t = oracle_sample(X, W, wl_.tau, rows, weight)
+    tops = 2.0 * rows * wl_.N * wl_.K / t / 1e12
+    return {"value": tops, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"oracle a1-a7 on the first {rows} of {wl_.M} rows of X ({t:.2f} s); all steps are "
+                      f"linear in the rows, so TOPS = 2*rows*N*K/t"}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, wl_, dist):
+    if dist.rank != 0:
+        return 0
+    import numpy as np  # noqa: F401
+
+    import oracle
+    import workloads as wl
+    X, W = wl.make_inputs(wl_)
+    weight = oracle.quantize_weight(W)
+    t1 = oracle_sample(X, W, wl_.tau, 1, weight)
+    per_step = min(0.5, 150.0 / max(1, args.steps + args.warmup))
+    rows = int(max(1, min(wl_.M, per_step / max(t1, 1e-6))))
+    for _ in range(args.warmup):
+        oracle_sample(X, W, wl_.tau, rows, weight)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample(X, W, wl_.tau, rows, weight)
+    el = time.perf_counter() - t0
+    tops = 2.0 * rows * wl_.N * wl_.K * args.steps / el / 1e12
+    sample = (f"each step: oracle a1-a7 on the first {rows} of {wl_.M} rows (all steps are linear in the rows; "
+              f"weights converted once, untimed)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": config_of(wl_, None),
+        "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(wl_, n_o, extra=None):
+    c = {"workload": wl_.name, "M": wl_.M, "N": wl_.N, "K": wl_.K, "tau": wl_.tau,
+         "outlier_columns_planted": int(wl_.n_planted if wl_.planted is None else len(wl_.planted)),
+         "outlier_columns_detected": n_o, "global_batch": wl_.M, "parallelism": "replicas"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------ our arm
+def source_digest(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(wl_name):
+    """DRAM bytes per GEMM launch from a committed ncu summary, only if it was
+    taken on the kernel source as it is now."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "gemm_i8_traffic.json")) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    src = os.path.join(ROOT, "int8_quantized_matmul_colwise_b200", "csrc", "gemm_i8.cu")
+    ent = d.get(wl_name)
+    if not ent or ent.get("gemm_source_sha256_16") != source_digest(src):
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def run_ours(args, wl_, dist):
+    import numpy as np
+    import torch
+
+    import int8_quantized_matmul_colwise_b200 as L
+    import workloads as wl
+
+    dist.init(torch)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+
+    X_np, W_np = wl.make_inputs(wl_)
+    M, N, K = wl_.M, wl_.N, wl_.K
+    cap = K
+    W = torch.from_numpy(W_np).to(dev)
+    X0 = torch.from_numpy(X_np).to(dev)
+
+    # offline weight conversion (reported, not part of the metric)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    Wq0, cs0 = L.quantize_weight_colwise(W)
+    e1.record()
+    torch.cuda.synchronize()
+    wq_ms = e0.elapsed_time(e1)
+
+    ws_bytes = L.llmint8_workspace_size(M, N, K, cap)
+    per_set = 2 * M * K + Wq0.numel() + 2 * M * N + M * L.round_up(K, 16)
+    n_sets = max(2, min(64, math.ceil(3 * L2_BYTES / per_set)))
+    sets = []
+    for i in range(n_sets):
+        sets.append({
+            "X": X0.clone(), "Wq": Wq0.clone(), "cs": cs0.clone(),
+            "Y": torch.empty((M, N), dtype=torch.float16, device=dev),
+            "ws": L.empty_workspace(M, N, K, cap, device=dev),
+        })
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        s = sets[i % n_sets]
+        L.llmint8_mixed_matmul(s["X"], s["Wq"], s["cs"], W, wl_.tau, cap, s["Y"], s["ws"], stream)
+
+    clocks = ClockSampler(torch.cuda.current_device()).start()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    st, flags = L.llmint8_check_status(sets[0]["ws"])
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {st} flags={flags}")
+    views = L.workspace_views(sets[0]["ws"], M, N, K, cap)
+    n_o = int(views["n_outlier"].item())
+
+    # ---- timed region: exactly K steps, inputs resident in HBM
+    dist.barrier(torch)
+    torch.cuda.synchronize()
+    ev_a, ev_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_host0 = time.perf_counter()
+    ev_a.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev_b.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
+    dist.barrier(torch)
+    el_ms = dist.max(torch, ev_a.elapsed_time(ev_b))
+    clk = clocks.summary(t_host0, t_host1)
+
+    ops = 2.0 * M * N * K
+    value = dist.world * ops * args.steps / (el_ms / 1e3) / 1e12
+    ms_per_step = el_ms / args.steps
+
+    # ---- per-kernel durations (same inputs, split entry points, events on the launching stream)
+    acts = []
+    for s in sets:
+        acts.append({
+            "Xq": torch.empty((M, L.round_up(K, 16)), dtype=torch.int8, device=dev),
+            "row_scale": torch.empty(M, dtype=torch.float32, device=dev),
+            "outlier_idx": torch.empty(cap, dtype=torch.int32, device=dev),
+            "n_outlier": torch.empty(1, dtype=torch.int32, device=dev),
+            "Xo": torch.empty((M, cap), dtype=torch.float16, device=dev),
+        })
+    n_k = max(10, min(args.steps, 200))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(n_k)]
+    for rep in range(2):  # first pass warms up
+        for i in range(n_k):
+            s, a = sets[i % n_sets], acts[i % n_sets]
+            if rep:
+                evs[i][0].record(stream)
+            L.llmint8_quantize_act_rowwise_outliers(s["X"], wl_.tau, a["Xq"], a["row_scale"], a["outlier_idx"],
+                                                    a["n_outlier"], a["Xo"], s["ws"], stream)
+            if rep:
+                evs[i][1].record(stream)
+            L.llmint8_mixed_gemm(a["Xq"], a["row_scale"], a["outlier_idx"], a["n_outlier"], a["Xo"], s["Wq"],
+                                 s["cs"], W, K, s["Y"], s["ws"], stream)
+            if rep:
+                evs[i][2].record(stream)
+        torch.cuda.synchronize()
+    t_quant = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) * 1e3  # us
+    t_gemm = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) * 1e3
+    t_gemm = dist.max(torch, t_gemm)
+    gemm_tops = ops / (t_gemm * 1e-6) / 1e12
+
+    traffic = recorded_traffic(wl_.name)
+    roofline = {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TFLOP/s",
+                "frac": gemm_tops / int8_peak, "traffic": traffic,
+                "kernel": "gemm_i8_kernel (tcgen05 kind::i8 + dequant/outlier epilogue)",
+                "peak_note": f"int8 dense = {INT8_PER_BF16:g} x bf16 burst {peaks['bf16_tflops']:.1f} TFLOP/s "
+                             f"({peaks['source']}); algorithmic ops per launch = 2MNK = {ops:.4g}"}
+    byts = algorithmic_bytes(M, N, K, n_o)
+    t_roof = max(ops / (int8_peak * 1e12), byts / (peaks["hbm_gbs"] * 1e9))
+    path = {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step * 1e-3),
+            "algorithmic_bytes": byts, "int8_peak_tops": int8_peak, "hbm_gbs": peaks["hbm_gbs"],
+            "scan_quantize_us": t_quant, "gemm_us": t_gemm,
+            "scan_quantize_gbs": (2 * M * K + M * K) / (t_quant * 1e-6) / 1e9}
+
+    # ---- end to end through the public API with host buffers
+    Xh = torch.from_numpy(X_np).pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.float16).pin_memory()
+    n_e = max(5, min(args.steps, 50))
+
+    def e2e_step(i):
+        s = sets[i % n_sets]
+        s["X"].copy_(Xh, non_blocking=True)
+        L.llmint8_mixed_matmul(s["X"], s["Wq"], s["cs"], W, wl_.tau, cap, s["Y"], s["ws"], stream)
+        Yh.copy_(s["Y"], non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    ev_a.record(stream)
+    for i in range(n_e):
+        e2e_step(i)
+    ev_b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dist.max(torch, ev_a.elapsed_time(ev_b)) / n_e
+    e2e = {"value": dist.world * ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+           "h2d_bytes_per_step": Xh.numel() * 2, "d2h_bytes_per_step": Yh.numel() * 2,
+           "ms_per_step": e2e_ms, "steps": n_e}
+    clocks.stop()
+
+    st, flags = L.llmint8_check_status(sets[0]["ws"])
+    if st != 0:
+        raise RuntimeError(f"device status after the run: {st} flags={flags}")
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl_, X_np, W_np, args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": dist.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": config_of(wl_, n_o, {
+            "l2": f"{n_sets} rotating input sets (X, Wq, Y, workspace) of {per_set / 2**20:.0f} MiB each "
+                  f"> 3x L2; consecutive steps touch different buffers",
+            "weight_quant_ms_offline": wq_ms, "workspace_bytes": ws_bytes,
+            "launch": "llmint8_mixed_matmul: 3 kernels chained with programmatic dependent launch"}),
+        "roofline": roofline, "path_roofline": path, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": 3 * args.steps, "clocks": clk,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+def main():
+    args = parse_args()
+    import workloads as wl
+    wl_ = wl.get(args.workload)
+    dist = Dist()
+    if args.impl == "reference":
+        return run_reference(args, wl_, dist)
+    return run_ours(args, wl_, dist)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

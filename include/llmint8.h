@@ -1,0 +1,196 @@
+/*
+ * llmint8.h -- C ABI of the B200 (sm_100a) LLM.int8() mixed-precision
+ * decomposition matmul  Y[M,N] = X[M,K] . W[K,N].
+ *
+ * The method (page titles and sections it is taken from):
+ *  - "LLM.int8(): 8-bit Matrix Multiplication for Transformers at Scale",
+ *    arXiv abstract: weights are loaded, converted to int8 and used at once;
+ *    vector-wise quantization with one normalization constant per inner
+ *    product; the emergent outlier feature dimensions go to a 16-bit matmul
+ *    while more than 99.9 % of the values are multiplied in 8-bit.
+ *  - "Compress your LLMs", bullets "Vector-wise quantization" and
+ *    "Mixed-precision decomposition": one scaling constant per row of the
+ *    input X and one per column of the weight W; outlier dimensions (~0.1 %)
+ *    in 16-bit, the rest in 8-bit.
+ *  - "8-bit Matrix Multiplication for Large Language Models", Summary &
+ *    Methodology Analysis: the int8 product is dequantized by the outer
+ *    product of the row and column constants and added to the outlier product
+ *    in 16-bit floating point.
+ *  - "What is 8-bit LLM quantization?", How does INT8 quantization work?:
+ *    q = round(value / step), value ~ q * step.
+ *
+ * Definitions used by every entry point (tau = threshold):
+ *   O      = ascending { k : |X[i,k]| >= tau for some row i of this call }
+ *   rs[i]  = max over k not in O of |X[i,k]|           (row absmax, fp32)
+ *   Xq[i,k]= k in O or rs[i]==0 ? 0 : rha(127 * X[i,k] / rs[i])
+ *   cs[j]  = max over all k of |W[k,j]|                 (column absmax, fp32)
+ *   Wq[j,k]= cs[j]==0 ? 0 : rha(127 * W[k,j] / cs[j])
+ *   acc    = Xq . Wq^T (exact, int32; needs K <= 133143)
+ *   Y[i,j] = fp16_RNE( acc[i,j] * rs[i] * cs[j] / 127^2
+ *                      + sum over k in O of X[i,k] * W[k,j] )
+ * rha = round half away from zero; every code is exact (no approximate
+ * division), so Xq, Wq, rs, cs, O and acc are unique.  The outlier product is
+ * accumulated in fp32 and Y is rounded once to fp16.
+ *
+ * Conventions.  Every pointer argument except host-only ones is a DEVICE
+ * pointer on the current CUDA device; the library allocates no memory and
+ * keeps no per-call state.  `stream` is a cudaStream_t (NULL = legacy default
+ * stream); every call only enqueues work on it and returns without waiting.
+ * Leading dimensions are in ELEMENTS.  Arguments are validated on the host
+ * before anything is launched; on an error nothing is launched.  Conditions
+ * only the device can see (outlier overflow, a bounded wait that gave up) set
+ * bits of a status word held in the workspace; llmint8_check_status() reads
+ * and clears it.  Calls that share a workspace must be ordered on one stream.
+ */
+#ifndef LLMINT8_H
+#define LLMINT8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum llmint8_status {
+    LLMINT8_OK = 0,
+    LLMINT8_ERR_INVALID_ARG = 1,      /* bad size, null or misaligned pointer, bad ld, NaN tau */
+    LLMINT8_ERR_UNSUPPORTED = 2,      /* current device is not sm_100 (B200) */
+    LLMINT8_ERR_WORKSPACE = 3,        /* workspace null, too small or not 256-byte aligned */
+    LLMINT8_ERR_CUDA = 4,             /* a CUDA runtime or driver call failed */
+    LLMINT8_ERR_OUTLIER_OVERFLOW = 5, /* device: n_o > outlier_cap (Y is NaN-filled) */
+    LLMINT8_ERR_TIMEOUT = 6           /* device: a bounded wait inside a kernel gave up */
+} llmint8_status;
+
+/* Bits of the device status word (see llmint8_check_status). */
+#define LLMINT8_STATUS_OUTLIER_OVERFLOW 0x1u
+#define LLMINT8_STATUS_TIMEOUT 0x2u
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* llmint8_status_string(llmint8_status s);
+
+/* Size in bytes of the workspace one call of llmint8_mixed_matmul or
+ * llmint8_quantize_act_rowwise_outliers needs for these sizes.  The workspace
+ * is caller-owned device memory, 256-byte aligned, zero-filled once before its
+ * first use (llmint8_workspace_init or any memset); the library leaves the
+ * parts that must start at zero back at zero.  It holds the status word, the
+ * column maxima, the outlier set, the row scales, Xq and the gathered outlier
+ * columns of X.  Returns 0 for invalid sizes. */
+size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K, int64_t outlier_cap);
+
+/* Zero-fill `ws` (cudaMemsetAsync on `stream`). */
+llmint8_status llmint8_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Byte offsets of the intermediates inside a workspace sized by
+ * llmint8_workspace_size (for inspection by tests and tools). */
+typedef struct llmint8_ws_layout {
+    size_t status;      /* uint32 status word */
+    size_t n_outlier;   /* int32 n_o (true count, may exceed outlier_cap) */
+    size_t outlier_idx; /* int32 [outlier_cap], ascending O */
+    size_t row_scale;   /* fp32 [M] */
+    size_t xq;          /* int8 [M, ldq], ldq = round_up(K, 16) */
+    size_t xo;          /* fp16 [M, ldo], ldo = round_up(max(outlier_cap,1), 8): X[:, O] */
+    int64_t ldq;
+    int64_t ldo;
+    size_t total;
+} llmint8_ws_layout;
+llmint8_status llmint8_workspace_layout(int64_t M, int64_t N, int64_t K, int64_t outlier_cap,
+                                        llmint8_ws_layout* out /* host */);
+
+/* Step a0, offline: column-wise int8 quantization of the weight ("Compress
+ * your LLMs", Vector-wise quantization: one constant per column of W; arXiv
+ * abstract: a 16-bit checkpoint is converted to int8 at load time).
+ *   W         fp16 [K, N], row stride ldw >= N (row-major, as stored in a
+ *             checkpoint).  Read only.
+ *   Wq        int8 [N, ldk] written: Wq[j*ldk + k] = code of W[k,j] (the
+ *             transpose, K contiguous, the layout the int8 tensor-core GEMM
+ *             reads); ldk >= K, ldk % 16 == 0, Wq 16-byte aligned; entries
+ *             k in [K, ldk) are written 0.
+ *   col_scale fp32 [N] written: cs[j] (the absmax, exact fp16 value).
+ * Errors: INVALID_ARG for K < 1, N < 1, ldw < N, bad ldk or alignment, null
+ * pointers; UNSUPPORTED off sm_100; CUDA on a launch failure. */
+llmint8_status llmint8_quantize_weight_colwise(const void* W, int64_t K, int64_t N, int64_t ldw,
+                                               int8_t* Wq, int64_t ldk, float* col_scale,
+                                               void* stream);
+
+/* Steps a1-a4 on the activation: outlier-column scan, row absmax over the
+ * non-outlier columns, row-wise int8 quantization and gather of the outlier
+ * columns ("Compress your LLMs", both bullets; arXiv abstract).
+ *   X           fp16 [M, K], row stride ldx >= K.  Read only.
+ *   tau         threshold, >= 0 or +inf (NaN rejected).  |x| >= tau marks x's
+ *               column an outlier over all M rows of this call.
+ *   Xq          int8 [M, ldq] written; ldq >= K, ldq % 16 == 0, 16-byte
+ *               aligned; outlier columns and columns [K, ldq) are 0.
+ *   row_scale   fp32 [M] written.
+ *   outlier_idx int32 [outlier_cap] written: the first min(n_o, cap) entries
+ *               of O, ascending.
+ *   n_outlier   int32 [1] written: n_o (may exceed outlier_cap; then the
+ *               status word gets LLMINT8_STATUS_OUTLIER_OVERFLOW).
+ *   Xo          optional fp16 [M, ldo] (NULL to skip): Xo[i,t] = X[i,O[t]]
+ *               for t < min(n_o, cap); ldo >= outlier_cap.
+ *   ws          workspace (see llmint8_workspace_size).
+ * All outputs are device-side; nothing is copied to the host. */
+llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, int64_t K, int64_t ldx,
+                                                     float tau, int8_t* Xq, int64_t ldq, float* row_scale,
+                                                     int32_t* outlier_idx, int64_t outlier_cap,
+                                                     int32_t* n_outlier, void* Xo, int64_t ldo, void* ws,
+                                                     size_t ws_bytes, void* stream);
+
+/* The whole forward path a1-a7: Y = X . W by the mixed-precision
+ * decomposition ("8-bit Matrix Multiplication for Large Language Models",
+ * Summary & Methodology Analysis; arXiv abstract).
+ *   X          fp16 [M, K], row stride ldx >= K.
+ *   Wq, ldk    int8 [N, ldk] and
+ *   col_scale  fp32 [N] from llmint8_quantize_weight_colwise.
+ *   W, ldw     fp16 [K, N] row-major, row stride ldw >= N: only the rows in O
+ *              are read (the 16-bit outlier product).
+ *   tau        threshold (>= 0 or +inf).
+ *   outlier_cap  bound on n_o the workspace is sized for; outlier_cap = K is
+ *              always enough.  If n_o > outlier_cap, Y is filled with NaN and
+ *              LLMINT8_STATUS_OUTLIER_OVERFLOW is set.
+ *   Y, ldy     fp16 [M, N] written, row stride ldy >= N.
+ *   ws         workspace of at least llmint8_workspace_size(M, N, K, cap).
+ * Runs three kernels on `stream` (scan/max, quantize/gather, int8 tcgen05
+ * GEMM with the dequantize + outlier epilogue); no host synchronisation. */
+llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
+                                    int64_t ldk, const float* col_scale, const void* W, int64_t ldw,
+                                    int64_t N, float tau, int64_t outlier_cap, void* Y, int64_t ldy,
+                                    void* ws, size_t ws_bytes, void* stream);
+
+/* Steps a5-a7 alone, on an activation already quantized by
+ * llmint8_quantize_act_rowwise_outliers (so that one quantized X can feed
+ * several weights, e.g. projections that share their input):
+ *   Y = fp16( (Xq . Wq^T) * rs (x) cs / 127^2 + Xo . W[O, :] ).
+ *   Xq, ldq          int8 [M, ldq] (ldq % 16 == 0, 16-byte aligned)
+ *   row_scale        fp32 [M]
+ *   outlier_idx      int32 [outlier_cap], n_outlier int32 [1] (device)
+ *   Xo, ldo          fp16 [M, ldo], ldo >= outlier_cap
+ *   Wq, ldk, col_scale, W, ldw, Y, ldy  as for llmint8_mixed_matmul
+ *   ws               at least 256 bytes (status word).
+ * If n_outlier > outlier_cap, Y is NaN-filled (the status bit was set by the
+ * quantize call).  One kernel launch (the tcgen05 GEMM). */
+llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* row_scale,
+                                  const int32_t* outlier_idx, const int32_t* n_outlier, int64_t outlier_cap,
+                                  const void* Xo, int64_t ldo, const int8_t* Wq, int64_t ldk,
+                                  const float* col_scale, const void* W, int64_t ldw, int64_t M, int64_t N,
+                                  int64_t K, void* Y, int64_t ldy, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read the status word of `ws`, clear it, and return
+ * LLMINT8_OK, LLMINT8_ERR_OUTLIER_OVERFLOW or LLMINT8_ERR_TIMEOUT (timeout
+ * wins).  `flags_out` (host, may be NULL) receives the raw bits. */
+llmint8_status llmint8_check_status(void* ws, void* stream, uint32_t* flags_out);
+
+/* Test hook for step a5 alone: C[i,j] = sum_k Xq[i,k] * Wq[j,k] as int32,
+ * computed by the same tcgen05 kernel as llmint8_mixed_matmul (the epilogue
+ * stores the raw accumulator instead of dequantizing).
+ *   Xq int8 [M, ldq], Wq int8 [N, ldk] (ld % 16 == 0, 16-byte aligned),
+ *   C int32 [M, ldc] written, ldc >= N.  `ws` supplies the status word. */
+llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const int8_t* Wq, int64_t ldk,
+                                           int64_t M, int64_t N, int64_t K, int32_t* C, int64_t ldc,
+                                           void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLMINT8_H */

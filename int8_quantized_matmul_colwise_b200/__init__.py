@@ -1,0 +1,124 @@
+"""LLM.int8() mixed-precision decomposition matmul for NVIDIA B200 (sm_100a).
+
+Y = X . W with the outlier feature dimensions of X (any |x| >= tau) multiplied
+in 16-bit and everything else in int8 with one absmax scale per row of X and
+per column of W ("LLM.int8(): 8-bit Matrix Multiplication for Transformers at
+Scale", arXiv abstract; "Compress your LLMs", Vector-wise quantization and
+Mixed-precision decomposition).
+
+The work runs in hand-written CUDA kernels behind the C ABI of
+``include/llmint8.h`` (``libllmint8.so``, built in-tree); this package only
+marshals torch tensors to it (``capi``) and offers allocating conveniences.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional, Tuple
+
+from . import capi
+from .capi import (LLMInt8Error, empty_workspace, llmint8_check_status, llmint8_debug_int8_gemm_i32,
+                   llmint8_mixed_gemm, llmint8_mixed_matmul, llmint8_quantize_act_rowwise_outliers, llmint8_quantize_weight_colwise,
+                   llmint8_status_string, llmint8_workspace_init, llmint8_workspace_layout,
+                   llmint8_workspace_size, round_up, workspace_views)
+
+__all__ = [
+    "capi", "LLMInt8Error", "quantize_weight_colwise", "quantize_act_rowwise_outliers", "mixed_matmul",
+    "check_status", "debug_int8_gemm_i32", "empty_workspace", "workspace_views", "Int8Weight",
+    "llmint8_quantize_weight_colwise", "llmint8_quantize_act_rowwise_outliers", "llmint8_mixed_matmul",
+    "llmint8_mixed_gemm", "mixed_gemm",
+    "llmint8_check_status", "llmint8_debug_int8_gemm_i32", "llmint8_status_string", "llmint8_workspace_size",
+    "llmint8_workspace_init", "llmint8_workspace_layout",
+]
+
+
+def quantize_weight_colwise(W, stream=None):
+    """W fp16 [K, N] -> (Wq int8 [N, round_up(K,16)], col_scale fp32 [N])."""
+    import torch
+    K, N = W.shape
+    Wq = torch.empty((N, round_up(K, 16)), dtype=torch.int8, device=W.device)
+    cs = torch.empty(N, dtype=torch.float32, device=W.device)
+    llmint8_quantize_weight_colwise(W, Wq, cs, stream)
+    return Wq, cs
+
+
+def quantize_act_rowwise_outliers(X, tau: float = 6.0, outlier_cap: Optional[int] = None, ws=None,
+                                  stream=None) -> Dict[str, object]:
+    """Steps a1-a4 on X fp16 [M, K]; returns device tensors Xq, row_scale,
+    outlier_idx (first min(n_o, cap) valid), n_outlier [1] and Xo."""
+    import torch
+    M, K = X.shape
+    cap = K if outlier_cap is None else outlier_cap
+    dev = X.device
+    out = {
+        "Xq": torch.empty((M, round_up(K, 16)), dtype=torch.int8, device=dev),
+        "row_scale": torch.empty(M, dtype=torch.float32, device=dev),
+        "outlier_idx": torch.empty(cap, dtype=torch.int32, device=dev),
+        "n_outlier": torch.empty(1, dtype=torch.int32, device=dev),
+        "Xo": torch.empty((M, cap), dtype=torch.float16, device=dev),
+    }
+    if ws is None:
+        ws = empty_workspace(M, 1, K, cap, device=dev)
+    llmint8_quantize_act_rowwise_outliers(X, tau, out["Xq"], out["row_scale"], out["outlier_idx"],
+                                          out["n_outlier"], out["Xo"], ws, stream)
+    out["ws"] = ws
+    return out
+
+
+def mixed_matmul(X, Wq, col_scale, W, tau: float = 6.0, outlier_cap: Optional[int] = None, Y=None, ws=None,
+                 stream=None):
+    """Y = X . W by the LLM.int8() decomposition (fp16 [M, N])."""
+    import torch
+    M, K = X.shape
+    N = Wq.size(0)
+    cap = K if outlier_cap is None else outlier_cap
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    if ws is None:
+        ws = empty_workspace(M, N, K, cap, device=X.device)
+    llmint8_mixed_matmul(X, Wq, col_scale, W, tau, cap, Y, ws, stream)
+    return Y
+
+
+def mixed_gemm(act: Dict[str, object], Wq, col_scale, W, Y=None, ws=None, stream=None):
+    """Steps a5-a7 on the output of quantize_act_rowwise_outliers."""
+    import torch
+    Xq = act["Xq"]
+    M, N = Xq.size(0), Wq.size(0)
+    K = W.size(0)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=Xq.device)
+    if ws is None:
+        ws = act["ws"]
+    llmint8_mixed_gemm(Xq, act["row_scale"], act["outlier_idx"], act["n_outlier"], act["Xo"], Wq, col_scale, W,
+                       K, Y, ws, stream)
+    return Y
+
+
+def check_status(ws, stream=None) -> int:
+    """Raise if the device reported an outlier overflow or a timeout."""
+    st, _ = llmint8_check_status(ws, stream)
+    if st != capi.OK:
+        raise LLMInt8Error(st, "device status")
+    return st
+
+
+def debug_int8_gemm_i32(Xq, Wq, K: int, stream=None):
+    """int32 [M, N] = Xq[:, :K] . Wq[:, :K]^T through the tcgen05 kernel."""
+    import torch
+    M, N = Xq.size(0), Wq.size(0)
+    C = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
+    ws = torch.zeros(256, dtype=torch.uint8, device=Xq.device)
+    llmint8_debug_int8_gemm_i32(Xq, Wq, K, C, ws, stream)
+    return C
+
+
+class Int8Weight:
+    """A weight converted once at load time: int8 codes, column scales and
+    the fp16 matrix whose outlier rows the 16-bit product reads."""
+
+    def __init__(self, W, stream=None):
+        self.W = W
+        self.K, self.N = W.shape
+        self.Wq, self.col_scale = quantize_weight_colwise(W, stream)
+
+    def matmul(self, X, tau: float = 6.0, outlier_cap: Optional[int] = None, Y=None, ws=None, stream=None):
+        return mixed_matmul(X, self.Wq, self.col_scale, self.W, tau, outlier_cap, Y, ws, stream)

@@ -1,0 +1,337 @@
+// capi.cu -- the extern "C" boundary declared in include/llmint8.h:
+// argument validation, workspace layout, TMA tensor-map encoding and kernel
+// launches.  No memory is allocated here; every buffer is the caller's.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.cuh"
+#include "llmint8.h"
+
+using namespace llmint8;
+
+namespace {
+
+constexpr int64_t kMaxK = 133143;  // 127^2 * K < 2^31: the int32 accumulator cannot overflow
+constexpr int kMaxDevices = 64;
+
+int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+bool aligned(const void* p, size_t a) { return reinterpret_cast<uintptr_t>(p) % a == 0; }
+
+// ------------------------------------------------------------------ devices
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+  int num_sms = 0;
+};
+std::mutex g_dev_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+llmint8_status current_device(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LLMINT8_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return LLMINT8_ERR_CUDA;
+    d.supported = (major == 10 && minor == 0);  // sm_100: the code is built for sm_100a only
+    d.num_sms = sms;
+    d.probed = true;
+  }
+  if (!d.supported) return LLMINT8_ERR_UNSUPPORTED;
+  if (num_sms) *num_sms = d.num_sms;
+  return LLMINT8_OK;
+}
+
+// ------------------------------------------------------------------ TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// int8 matrix [rows, cols] with row stride ld (bytes), read in boxes of
+// box_rows x 128 bytes with the 128-byte swizzle; out-of-range reads are 0.
+bool encode_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                        uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemmBK), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ workspace
+// [0, 256)        header: status u32 @0, scan counter u32 @4, n_o i32 @8
+// colmax          u32 [K]
+// bitmask         u32 [ceil(K/32)]
+// outlier_idx     i32 [cap]
+// row_scale       f32 [M]
+// xq              i8  [M, ldq]
+// xo              f16 [M, ldo]
+bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t* colmax, size_t* bitmask) {
+  if (M < 1 || K < 1 || K > kMaxK || cap < 0 || cap > K) return false;
+  size_t off = 256;
+  *colmax = off;
+  off = align_up(off + 4 * size_t(K), 256);
+  *bitmask = off;
+  off = align_up(off + 4 * size_t((K + 31) / 32), 256);
+  L->status = 0;
+  L->n_outlier = 8;
+  L->outlier_idx = off;
+  off = align_up(off + 4 * size_t(cap > 0 ? cap : 1), 256);
+  L->row_scale = off;
+  off = align_up(off + 4 * size_t(M), 1024);
+  L->ldq = round_up(K, 16);
+  L->xq = off;
+  off = align_up(off + size_t(M) * size_t(L->ldq), 256);
+  L->ldo = round_up(cap > 0 ? cap : 1, 8);
+  L->xo = off;
+  off = align_up(off + 2 * size_t(M) * size_t(L->ldo), 256);
+  L->total = off;
+  return true;
+}
+
+ActWs act_ws(void* ws, size_t colmax_off, size_t bitmask_off) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  ActWs a;
+  a.status = reinterpret_cast<uint32_t*>(b);
+  a.counter = reinterpret_cast<uint32_t*>(b + 4);
+  a.colmax = reinterpret_cast<uint32_t*>(b + colmax_off);
+  a.bitmask = reinterpret_cast<uint32_t*>(b + bitmask_off);
+  return a;
+}
+
+llmint8_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA; }
+
+bool valid_tau(float tau) { return !std::isnan(tau) && tau >= 0.0f; }
+
+}  // namespace
+
+extern "C" {
+
+const char* llmint8_status_string(llmint8_status s) {
+  switch (s) {
+    case LLMINT8_OK: return "LLMINT8_OK";
+    case LLMINT8_ERR_INVALID_ARG: return "LLMINT8_ERR_INVALID_ARG";
+    case LLMINT8_ERR_UNSUPPORTED: return "LLMINT8_ERR_UNSUPPORTED";
+    case LLMINT8_ERR_WORKSPACE: return "LLMINT8_ERR_WORKSPACE";
+    case LLMINT8_ERR_CUDA: return "LLMINT8_ERR_CUDA";
+    case LLMINT8_ERR_OUTLIER_OVERFLOW: return "LLMINT8_ERR_OUTLIER_OVERFLOW";
+    case LLMINT8_ERR_TIMEOUT: return "LLMINT8_ERR_TIMEOUT";
+  }
+  return "LLMINT8_UNKNOWN_STATUS";
+}
+
+llmint8_status llmint8_workspace_layout(int64_t M, int64_t N, int64_t K, int64_t outlier_cap,
+                                        llmint8_ws_layout* out) {
+  if (!out || N < 1) return LLMINT8_ERR_INVALID_ARG;
+  size_t c, b;
+  if (!make_layout(M, K, outlier_cap, out, &c, &b)) return LLMINT8_ERR_INVALID_ARG;
+  return LLMINT8_OK;
+}
+
+size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K, int64_t outlier_cap) {
+  llmint8_ws_layout L;
+  if (llmint8_workspace_layout(M, N, K, outlier_cap, &L) != LLMINT8_OK) return 0;
+  return L.total;
+}
+
+llmint8_status llmint8_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < 256 || !aligned(ws, 256)) return LLMINT8_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+llmint8_status llmint8_quantize_weight_colwise(const void* W, int64_t K, int64_t N, int64_t ldw, int8_t* Wq,
+                                               int64_t ldk, float* col_scale, void* stream) {
+  if (!W || !Wq || !col_scale) return LLMINT8_ERR_INVALID_ARG;
+  if (K < 1 || N < 1 || K > kMaxK || N > (int64_t(1) << 31) - 1 || ldw < N) return LLMINT8_ERR_INVALID_ARG;
+  if (ldk < K || ldk % 16 != 0 || !aligned(Wq, 16) || !aligned(W, 2) || !aligned(col_scale, 4))
+    return LLMINT8_ERR_INVALID_ARG;
+  llmint8_status st = current_device(nullptr);
+  if (st != LLMINT8_OK) return st;
+  return cuda_status(
+      launch_quantize_weight_colwise(W, K, N, ldw, Wq, ldk, col_scale, static_cast<cudaStream_t>(stream)));
+}
+
+llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, int64_t K, int64_t ldx,
+                                                     float tau, int8_t* Xq, int64_t ldq, float* row_scale,
+                                                     int32_t* outlier_idx, int64_t outlier_cap,
+                                                     int32_t* n_outlier, void* Xo, int64_t ldo, void* ws,
+                                                     size_t ws_bytes, void* stream) {
+  if (!X || !Xq || !row_scale || !outlier_idx || !n_outlier) return LLMINT8_ERR_INVALID_ARG;
+  if (M < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || ldx < K || !valid_tau(tau))
+    return LLMINT8_ERR_INVALID_ARG;
+  if (outlier_cap < 1 || outlier_cap > K) return LLMINT8_ERR_INVALID_ARG;
+  if (ldq < K || ldq % 16 != 0 || !aligned(Xq, 16) || !aligned(X, 2)) return LLMINT8_ERR_INVALID_ARG;
+  if (Xo && (ldo < outlier_cap || !aligned(Xo, 2))) return LLMINT8_ERR_INVALID_ARG;
+  llmint8_ws_layout L;
+  size_t colmax, bitmask;
+  if (!make_layout(M, K, outlier_cap, &L, &colmax, &bitmask)) return LLMINT8_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return LLMINT8_ERR_WORKSPACE;
+  llmint8_status st = current_device(nullptr);
+  if (st != LLMINT8_OK) return st;
+  return cuda_status(launch_quantize_act(X, M, K, ldx, tau, Xq, ldq, row_scale, outlier_idx, outlier_cap,
+                                         n_outlier, Xo, ldo, act_ws(ws, colmax, bitmask),
+                                         static_cast<cudaStream_t>(stream), true));
+}
+
+llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
+                                    int64_t ldk, const float* col_scale, const void* W, int64_t ldw, int64_t N,
+                                    float tau, int64_t outlier_cap, void* Y, int64_t ldy, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  if (!X || !Wq || !col_scale || !W || !Y) return LLMINT8_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1)
+    return LLMINT8_ERR_INVALID_ARG;
+  if (ldx < K || ldw < N || ldy < N || ldk < K || ldk % 16 != 0 || !valid_tau(tau))
+    return LLMINT8_ERR_INVALID_ARG;
+  if (outlier_cap < 1 || outlier_cap > K) return LLMINT8_ERR_INVALID_ARG;
+  if (!aligned(Wq, 16) || !aligned(X, 2) || !aligned(W, 2) || !aligned(Y, 2) || !aligned(col_scale, 4))
+    return LLMINT8_ERR_INVALID_ARG;
+  llmint8_ws_layout L;
+  size_t colmax_off, bitmask_off;
+  if (!make_layout(M, K, outlier_cap, &L, &colmax_off, &bitmask_off)) return LLMINT8_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return LLMINT8_ERR_WORKSPACE;
+  int num_sms = 0;
+  llmint8_status st = current_device(&num_sms);
+  if (st != LLMINT8_OK) return st;
+
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  int8_t* xq = reinterpret_cast<int8_t*>(b + L.xq);
+  float* rs = reinterpret_cast<float*>(b + L.row_scale);
+  int32_t* O = reinterpret_cast<int32_t*>(b + L.outlier_idx);
+  int32_t* n_o = reinterpret_cast<int32_t*>(b + L.n_outlier);
+  void* xo = b + L.xo;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  CUtensorMap tmA, tmB;
+  if (!encode_operand_map(&tmA, xq, M, K, L.ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, kGemmBN))
+    return LLMINT8_ERR_CUDA;
+
+  cudaError_t e = launch_quantize_act(X, M, K, ldx, tau, xq, L.ldq, rs, O, outlier_cap, n_o, xo, L.ldo,
+                                      act_ws(ws, colmax_off, bitmask_off), s, true);
+  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+
+  GemmArgs a = {};
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.rs = rs;
+  a.cs = col_scale;
+  a.Xo = xo;
+  a.ldo = L.ldo;
+  a.O = O;
+  a.n_o = n_o;
+  a.cap = static_cast<int>(outlier_cap);
+  a.W = W;
+  a.ldw = ldw;
+  a.Y = Y;
+  a.ldy = ldy;
+  a.C = nullptr;
+  a.ldc = 0;
+  a.status = reinterpret_cast<uint32_t*>(b + L.status);
+  return cuda_status(launch_gemm_i8(tmA, tmB, a, false, num_sms, s, true));
+}
+
+llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* row_scale,
+                                  const int32_t* outlier_idx, const int32_t* n_outlier, int64_t outlier_cap,
+                                  const void* Xo, int64_t ldo, const int8_t* Wq, int64_t ldk,
+                                  const float* col_scale, const void* W, int64_t ldw, int64_t M, int64_t N,
+                                  int64_t K, void* Y, int64_t ldy, void* ws, size_t ws_bytes, void* stream) {
+  if (!Xq || !row_scale || !outlier_idx || !n_outlier || !Xo || !Wq || !col_scale || !W || !Y)
+    return LLMINT8_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1)
+    return LLMINT8_ERR_INVALID_ARG;
+  if (outlier_cap < 1 || outlier_cap > K || ldo < outlier_cap) return LLMINT8_ERR_INVALID_ARG;
+  if (ldq < K || ldk < K || ldq % 16 != 0 || ldk % 16 != 0 || ldw < N || ldy < N) return LLMINT8_ERR_INVALID_ARG;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Xo, 2) || !aligned(W, 2) || !aligned(Y, 2) ||
+      !aligned(row_scale, 4) || !aligned(col_scale, 4))
+    return LLMINT8_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < 256) return LLMINT8_ERR_WORKSPACE;
+  int num_sms = 0;
+  llmint8_status st = current_device(&num_sms);
+  if (st != LLMINT8_OK) return st;
+  CUtensorMap tmA, tmB;
+  if (!encode_operand_map(&tmA, Xq, M, K, ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, kGemmBN))
+    return LLMINT8_ERR_CUDA;
+  GemmArgs a = {};
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.rs = row_scale;
+  a.cs = col_scale;
+  a.Xo = Xo;
+  a.ldo = ldo;
+  a.O = outlier_idx;
+  a.n_o = n_outlier;
+  a.cap = static_cast<int>(outlier_cap);
+  a.W = W;
+  a.ldw = ldw;
+  a.Y = Y;
+  a.ldy = ldy;
+  a.status = static_cast<uint32_t*>(ws);
+  return cuda_status(launch_gemm_i8(tmA, tmB, a, false, num_sms, static_cast<cudaStream_t>(stream), true));
+}
+
+llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const int8_t* Wq, int64_t ldk,
+                                           int64_t M, int64_t N, int64_t K, int32_t* C, int64_t ldc, void* ws,
+                                           size_t ws_bytes, void* stream) {
+  if (!Xq || !Wq || !C) return LLMINT8_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1)
+    return LLMINT8_ERR_INVALID_ARG;
+  if (ldq < K || ldk < K || ldq % 16 != 0 || ldk % 16 != 0 || ldc < N) return LLMINT8_ERR_INVALID_ARG;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(C, 4)) return LLMINT8_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < 256) return LLMINT8_ERR_WORKSPACE;
+  int num_sms = 0;
+  llmint8_status st = current_device(&num_sms);
+  if (st != LLMINT8_OK) return st;
+  CUtensorMap tmA, tmB;
+  if (!encode_operand_map(&tmA, Xq, M, K, ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, kGemmBN))
+    return LLMINT8_ERR_CUDA;
+  GemmArgs a = {};
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.C = C;
+  a.ldc = ldc;
+  a.status = static_cast<uint32_t*>(ws);
+  return cuda_status(launch_gemm_i8(tmA, tmB, a, true, num_sms, static_cast<cudaStream_t>(stream), false));
+}
+
+llmint8_status llmint8_check_status(void* ws, void* stream, uint32_t* flags_out) {
+  if (!ws || !aligned(ws, 256)) return LLMINT8_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LLMINT8_ERR_CUDA;
+  uint32_t flags = 0;
+  if (cudaMemcpy(&flags, ws, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess) return LLMINT8_ERR_CUDA;
+  if (flags != 0 && cudaMemset(ws, 0, sizeof(flags)) != cudaSuccess) return LLMINT8_ERR_CUDA;
+  if (flags_out) *flags_out = flags;
+  if (flags & LLMINT8_STATUS_TIMEOUT) return LLMINT8_ERR_TIMEOUT;
+  if (flags & LLMINT8_STATUS_OUTLIER_OVERFLOW) return LLMINT8_ERR_OUTLIER_OVERFLOW;
+  return LLMINT8_OK;
+}
+
+}  // extern "C"

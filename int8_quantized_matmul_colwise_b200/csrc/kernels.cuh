@@ -1,0 +1,55 @@
+// kernels.cuh -- launch interfaces between the C ABI (capi.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace llmint8 {
+
+// Scratch the activation kernels keep in the caller's workspace.
+struct ActWs {
+  uint32_t* colmax;   // [K] fp16 bit patterns of the column maxima; zero between calls
+  uint32_t* counter;  // CTA completion counter of the scan kernel; zero between calls
+  uint32_t* bitmask;  // [ceil(K/32)] outlier flags of this call
+  uint32_t* status;   // status word
+};
+
+cudaError_t launch_quantize_weight_colwise(const void* W, int64_t K, int64_t N, int64_t ldw, int8_t* Wq,
+                                           int64_t ldk, float* col_scale, cudaStream_t stream);
+
+cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx, float tau, int8_t* Xq,
+                                int64_t ldq, float* rs, int32_t* O, int64_t cap, int32_t* n_out, void* Xo,
+                                int64_t ldo, ActWs ws, cudaStream_t stream, bool pdl);
+
+// Everything the GEMM epilogue needs besides the two tensor maps.
+struct GemmArgs {
+  int M, N, K;
+  const float* rs;    // [M] row scales
+  const float* cs;    // [N] column scales
+  const void* Xo;     // fp16 [M, ldo] gathered outlier columns of X
+  int64_t ldo;
+  const int32_t* O;   // [cap] outlier columns (rows of W)
+  const int32_t* n_o; // device count
+  int cap;
+  const void* W;      // fp16 [K, ldw]
+  int64_t ldw;
+  void* Y;            // fp16 [M, ldy]
+  int64_t ldy;
+  int32_t* C;         // int32 [M, ldc] (raw accumulator output mode)
+  int64_t ldc;
+  uint32_t* status;
+};
+
+// tmA: Xq [M rows, K cols] int8, tmB: Wq [N rows, K cols] int8, both encoded
+// by encode_operand_map().  raw_i32 selects the accumulator-dump epilogue.
+cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, bool raw_i32,
+                           int num_sms, cudaStream_t stream, bool pdl);
+
+// Tile sizes of the GEMM (rows of Xq / rows of Wq per tile, K bytes per stage).
+constexpr int kGemmBM = 128;
+constexpr int kGemmBN = 256;
+constexpr int kGemmBK = 128;
+
+}  // namespace llmint8

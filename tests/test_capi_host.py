@@ -1,0 +1,101 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function the header declares, sizes workspaces, names statuses, and
+rejects invalid arguments before touching the device."""
+import ctypes
+
+import pytest
+
+from int8_quantized_matmul_colwise_b200 import _build, capi
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build_library()
+    return capi.lib()
+
+
+def test_every_declared_function_is_exported(lib):
+    names = capi.header_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(capi.SIGNATURES), set(names) ^ set(capi.SIGNATURES)
+
+
+def test_status_strings(lib):
+    for code, name in capi.STATUS_NAMES.items():
+        assert capi.llmint8_status_string(code) == name
+    assert capi.llmint8_status_string(99) == "LLMINT8_UNKNOWN_STATUS"
+
+
+def test_workspace_layout_and_size(lib):
+    M, N, K, cap = 2048, 16384, 4096, 4096
+    L = capi.llmint8_workspace_layout(M, N, K, cap)
+    assert L.ldq == 4096 and L.ldo == 4096
+    assert L.total == capi.llmint8_workspace_size(M, N, K, cap)
+    regions = sorted([(L.outlier_idx, 4 * cap), (L.row_scale, 4 * M), (L.xq, M * L.ldq), (L.xo, 2 * M * L.ldo)])
+    for (a, na), (b, _) in zip(regions, regions[1:]):
+        assert a + na <= b
+    assert L.xq % 256 == 0 and L.xo % 256 == 0 and L.outlier_idx % 256 == 0
+    assert regions[-1][0] + regions[-1][1] <= L.total
+    L2 = capi.llmint8_workspace_layout(3, 33, 24, 1)
+    assert L2.ldq == 32 and L2.ldo == 8
+
+
+@pytest.mark.parametrize("M,N,K,cap", [(0, 1, 1, 1), (1, 0, 1, 1), (1, 1, 0, 1), (1, 1, 133144, 1),
+                                       (1, 1, 8, 9), (1, 1, 8, -1)])
+def test_workspace_size_rejects_bad_sizes(lib, M, N, K, cap):
+    assert capi.llmint8_workspace_size(M, N, K, cap) == 0
+
+
+def _mm(lib, **kw):
+    a = dict(X=0x1000, M=4, K=32, ldx=32, Wq=0x2000, ldk=32, cs=0x3000, W=0x4000, ldw=16, N=16, tau=6.0,
+             cap=32, Y=0x5000, ldy=16, ws=0x10000, ws_bytes=1 << 20, stream=None)
+    a.update(kw)
+    return lib.llmint8_mixed_matmul(a["X"], a["M"], a["K"], a["ldx"], a["Wq"], a["ldk"], a["cs"], a["W"],
+                                    a["ldw"], a["N"], a["tau"], a["cap"], a["Y"], a["ldy"], a["ws"],
+                                    a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(X=None), capi.ERR_INVALID_ARG),
+    (dict(M=0), capi.ERR_INVALID_ARG),
+    (dict(K=133144, ldx=133144, ldk=133152, cap=1), capi.ERR_INVALID_ARG),
+    (dict(ldx=31), capi.ERR_INVALID_ARG),
+    (dict(ldk=24), capi.ERR_INVALID_ARG),
+    (dict(ldk=40), capi.ERR_INVALID_ARG),        # not a multiple of 16
+    (dict(Wq=0x2008), capi.ERR_INVALID_ARG),     # not 16-byte aligned
+    (dict(ldy=8), capi.ERR_INVALID_ARG),
+    (dict(tau=float("nan")), capi.ERR_INVALID_ARG),
+    (dict(tau=-1.0), capi.ERR_INVALID_ARG),
+    (dict(cap=0), capi.ERR_INVALID_ARG),
+    (dict(cap=33), capi.ERR_INVALID_ARG),
+    (dict(ws=None), capi.ERR_WORKSPACE),
+    (dict(ws=0x10010), capi.ERR_WORKSPACE),      # not 256-byte aligned
+    (dict(ws_bytes=1024), capi.ERR_WORKSPACE),
+])
+def test_mixed_matmul_rejects_invalid_arguments_on_the_host(lib, kw, expect):
+    # these fail validation before any CUDA call, so no device is needed
+    assert _mm(lib, **kw) == expect
+
+
+def test_weight_quant_rejects_invalid_arguments(lib):
+    f = lib.llmint8_quantize_weight_colwise
+    assert f(None, 4, 4, 4, 0x2000, 16, 0x3000, None) == capi.ERR_INVALID_ARG
+    assert f(0x1000, 4, 4, 3, 0x2000, 16, 0x3000, None) == capi.ERR_INVALID_ARG   # ldw < N
+    assert f(0x1000, 4, 4, 4, 0x2000, 8, 0x3000, None) == capi.ERR_INVALID_ARG    # ldk % 16
+    assert f(0x1000, 20, 4, 4, 0x2000, 16, 0x3000, None) == capi.ERR_INVALID_ARG   # ldk < K
+
+
+def test_debug_gemm_rejects_invalid_arguments(lib):
+    f = lib.llmint8_debug_int8_gemm_i32
+    assert f(0x1000, 16, 0x2000, 16, 1, 1, 17, 0x3000, 1, 0x10000, 256, None) == capi.ERR_INVALID_ARG
+    assert f(0x1000, 16, 0x2000, 16, 1, 1, 16, 0x3000, 1, 0x10000, 128, None) == capi.ERR_WORKSPACE
+
+
+def test_binding_refuses_host_tensors():
+    torch = pytest.importorskip("torch")
+    import int8_quantized_matmul_colwise_b200 as L
+    W = torch.zeros(8, 8, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        L.llmint8_quantize_weight_colwise(W, torch.zeros(8, 16, dtype=torch.int8), torch.zeros(8))

@@ -1,0 +1,298 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Bit-exact: Wq, col scales, outlier set and count, row scales, Xq, the gathered
+outlier columns and the int32 accumulator.  Y (fp16) within
+|Y_gpu - Y_oracle| <= 1e-3 |Y_oracle| + 1e-3 max|Y_oracle|.
+Small and ragged shapes are compared element by element; the full-size
+workloads are compared on every intermediate and on the accumulator and Y of
+64 seeded rows plus the first and last row, in the launch configuration the
+benchmark times.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as wl
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+RTOL = 1e-3
+ATOL_REL_MAX = 1e-3
+
+
+@pytest.fixture(scope="module")
+def L():
+    from int8_quantized_matmul_colwise_b200 import _build
+    _build.build_library()
+    import int8_quantized_matmul_colwise_b200 as lib
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return lib
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    return t.detach().cpu().numpy()
+
+
+def y_close(y_gpu: np.ndarray, y_ref: np.ndarray):
+    g = y_gpu.astype(np.float64)
+    r = y_ref.astype(np.float64)
+    bound = RTOL * np.abs(r) + ATOL_REL_MAX * np.abs(r).max()
+    bad = ~(np.abs(g - r) <= bound)
+    assert not bad.any(), (f"{bad.sum()} of {bad.size} outside tolerance; worst |d|="
+                           f"{np.abs(g - r)[bad].max()} at {np.argwhere(bad)[0]}")
+
+
+def assert_status_ok(L, ws):
+    st, flags = L.llmint8_check_status(ws)
+    assert st == 0 and flags == 0, (st, flags)
+
+
+# ------------------------------------------------------------------ a0: weights
+
+WEIGHT_SHAPES = [(256, 256), (1000, 1000), (4100, 4095), (520, 257), (24, 33), (1, 5), (4096, 4096)]
+
+
+@pytest.mark.parametrize("K,N", WEIGHT_SHAPES)
+def test_weight_quantization_bit_exact(L, K, N):
+    rng = np.random.default_rng(K * 7 + N)
+    W = (rng.standard_normal((K, N), dtype=np.float32) * 0.02).astype(np.float16)
+    W[rng.integers(0, K), :] = 0  # a zero row
+    W[:, rng.integers(0, N)] = 0  # a zero column: scale 0, codes 0
+    Wq, cs = L.quantize_weight_colwise(dev(W))
+    torch.cuda.synchronize()
+    Wq_ref, cs_ref = oracle.quantize_weight(W)
+    assert np.array_equal(host(cs), cs_ref)
+    g = host(Wq)
+    assert np.array_equal(g[:, :K], Wq_ref.T)
+    assert not g[:, K:].any()
+
+
+def test_weight_quantization_full_size_ffn(L):
+    w = wl.get("ffn_6p7b_prefill")
+    W = wl.make_w(w)
+    Wq, cs = L.quantize_weight_colwise(dev(W))
+    Wq_ref, cs_ref = oracle.quantize_weight(W)
+    assert np.array_equal(host(cs), cs_ref)
+    assert np.array_equal(host(Wq)[:, :w.K], Wq_ref.T)
+
+
+# ------------------------------------------------------------------ a1-a4: activations
+
+ACT_WORKLOADS = ["tiny", "decode_m1", "decode_m8", "decode_m32", "ffn_6p7b_prefill", "sweep8k_o1",
+                 "ragged_1000x1000x1000", "ragged_2047x4095x4100", "ragged_129x257x520", "ragged_1x1001x1000",
+                 "ragged_3x33x24"]
+
+
+def check_act(L, X, tau, cap=None):
+    M, K = X.shape
+    out = L.quantize_act_rowwise_outliers(dev(X), tau, cap)
+    O, rs, Xq = oracle.quantize_activation(X, tau)
+    n = int(host(out["n_outlier"])[0])
+    assert n == O.size
+    cap_ = K if cap is None else cap
+    k = min(n, cap_)
+    assert np.array_equal(host(out["outlier_idx"])[:k], O[:k])
+    assert np.array_equal(host(out["row_scale"]), rs)
+    g = host(out["Xq"])
+    assert np.array_equal(g[:, :K], Xq)
+    assert not g[:, K:].any()
+    Xo_ref, _ = oracle.gather_outliers(X, O[:k])
+    assert np.array_equal(host(out["Xo"])[:, :k].view(np.uint16), Xo_ref.view(np.uint16))
+    return out
+
+
+@pytest.mark.parametrize("name", ACT_WORKLOADS)
+def test_activation_quantization_bit_exact(L, name):
+    w = wl.get(name)
+    X = wl.make_x(w)
+    out = check_act(L, X, w.tau)
+    assert_status_ok(L, out["ws"])
+    planted = set(wl.planted_columns(w).tolist())
+    if w.M >= 8:
+        got = set(host(out["outlier_idx"])[:int(host(out["n_outlier"])[0])].tolist())
+        assert planted <= got
+
+
+@pytest.mark.parametrize("tau", [np.inf, 0.0, 2.5])
+def test_activation_thresholds(L, tau):
+    X = wl.make_x(wl.get("ragged_129x257x520"))
+    check_act(L, X, tau)
+
+
+SCALES = [65504.0, 127.0, 12.703125, 6.0, 1.984375, 1.0, float(np.float16(0.1)), 2.0 ** -14, 2.0 ** -24, 1000.5]
+
+
+@pytest.mark.parametrize("s", SCALES)
+def test_exact_quantizer_every_fp16_value(L, s):
+    """Rows [s, x_1, ...] with every finite fp16 |x| <= s: the division-free
+    kernel quantizer equals the oracle's correctly rounded one."""
+    h = np.arange(65536, dtype=np.uint32).astype(np.uint16).view(np.float16)
+    xs = h[np.isfinite(h) & (np.abs(h.astype(np.float64)) <= s)]
+    per = 4095
+    rows = -(-xs.size // per)
+    body = np.zeros(rows * per, np.float16)
+    body[:xs.size] = xs
+    X = np.concatenate([np.full((rows, 1), s, np.float16), body.reshape(rows, per)], axis=1)
+    check_act(L, X, np.inf)
+
+
+def test_activation_strided_rows(L):
+    X = wl.make_x(wl.get("tiny"))
+    wide = np.zeros((X.shape[0], X.shape[1] + 40), np.float16)
+    wide[:, 8:8 + X.shape[1]] = X
+    t = dev(wide)[:, 8:8 + X.shape[1]]
+    out = L.quantize_act_rowwise_outliers(t, 6.0)
+    O, rs, Xq = oracle.quantize_activation(X, 6.0)
+    assert np.array_equal(host(out["Xq"])[:, :X.shape[1]], Xq)
+    assert np.array_equal(host(out["row_scale"]), rs)
+
+
+# ------------------------------------------------------------------ a5: int8 GEMM (raw accumulator)
+
+GEMM_SHAPES = [(128, 256, 128), (1, 1, 1), (5, 7, 3), (3, 33, 24), (129, 257, 520), (1, 1001, 1000),
+               (1000, 1000, 1000), (300, 600, 4096), (2047, 4095, 4100), (256, 512, 8192)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_int8_gemm_accumulator_bit_exact(L, M, N, K):
+    rng = np.random.default_rng(M + 3 * N + 7 * K)
+    Xq = rng.integers(-127, 128, (M, K), dtype=np.int8)
+    Wq = rng.integers(-127, 128, (N, K), dtype=np.int8)
+    ldq = L.round_up(K, 16)
+    Xp = np.zeros((M, ldq), np.int8)
+    Xp[:, :K] = Xq
+    Wp = np.zeros((N, ldq), np.int8)
+    Wp[:, :K] = Wq
+    C = host(L.debug_int8_gemm_i32(dev(Xp), dev(Wp), K))
+    rows = None if M * N * K <= 2e9 else wl.sample_rows(M)
+    ref = oracle.int8_matmul(Xq, np.ascontiguousarray(Wq.T), rows)
+    got = C.astype(np.int64) if rows is None else C[rows].astype(np.int64)
+    assert np.array_equal(got, ref)
+
+
+def test_int8_gemm_extreme_codes(L):
+    """All +-127 codes at the largest K of the workloads: the int32 sum
+    reaches 127^2 * K without overflow."""
+    M, N, K = 130, 260, 12288
+    Xq = np.full((M, K), 127, np.int8)
+    Xq[1::2] = -127
+    Wq = np.full((N, K), 127, np.int8)
+    C = host(L.debug_int8_gemm_i32(dev(Xq), dev(Wq), K))
+    assert np.all(C[0::2] == 127 * 127 * K) and np.all(C[1::2] == -127 * 127 * K)
+
+
+# ------------------------------------------------------------------ a0-a7: the whole path
+
+def run_path(L, X, W, tau, cap=None, rows=None):
+    M, K = X.shape
+    N = W.shape[1]
+    cap = K if cap is None else cap
+    Wd = dev(W)
+    Wq, cs = L.quantize_weight_colwise(Wd)
+    ws = L.empty_workspace(M, N, K, cap)
+    Y = L.mixed_matmul(dev(X), Wq, cs, Wd, tau, cap, ws=ws)
+    st, flags = L.llmint8_check_status(ws)
+    views = L.workspace_views(ws, M, N, K, cap)
+    return Y, ws, views, (Wq, cs), (st, flags)
+
+
+def check_path(L, X, W, tau, rows=None, cap=None):
+    M, K = X.shape
+    N = W.shape[1]
+    Y, ws, v, (Wq, cs), (st, flags) = run_path(L, X, W, tau, cap)
+    assert st == 0 and flags == 0, (st, flags)
+    Wq_ref, cs_ref = oracle.quantize_weight(W)
+    r = oracle.mixed_matmul(X, W, tau, rows=rows, weight=(Wq_ref, cs_ref))
+    n = int(host(v["n_outlier"])[0])
+    assert n == r["O"].size
+    assert np.array_equal(host(v["outlier_idx"])[:n], r["O"])
+    assert np.array_equal(host(v["row_scale"]), r["rs"])
+    assert np.array_equal(host(v["xq"])[:, :K], r["Xq"])
+    assert np.array_equal(host(cs), cs_ref)
+    Yg = host(Y)
+    Yg = Yg if rows is None else Yg[rows]
+    y_close(Yg, r["Y"])
+    return Yg, r
+
+
+SMALL_PATH = ["tiny", "decode_m1", "decode_m8", "decode_m32", "ragged_1000x1000x1000", "ragged_129x257x520",
+              "ragged_1x1001x1000", "ragged_3x33x24", "ragged_2047x4095x4100"]
+
+
+@pytest.mark.parametrize("name", SMALL_PATH)
+def test_mixed_matmul_small_and_ragged(L, name):
+    w = wl.get(name)
+    X, W = wl.make_inputs(w)
+    rows = wl.sample_rows(w.M) if w.M * w.N * w.K > 4e9 else None
+    check_path(L, X, W, w.tau, rows=rows)
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_129x257x520", "ragged_3x33x24"])
+def test_mixed_matmul_tau_inf_and_zero(L, name):
+    w = wl.get(name)
+    X, W = wl.make_inputs(w)
+    check_path(L, X, W, np.inf)
+    Yg, r = check_path(L, X, W, 0.0)
+    assert r["O"].size == w.K  # every column is an outlier: the fp16 matmul
+
+
+def test_mixed_matmul_accumulator_matches_oracle(L):
+    """The int32 accumulator of the whole path equals the oracle's, through
+    the raw-accumulator epilogue on the workspace's own Xq and the GPU Wq."""
+    w = wl.get("ragged_1000x1000x1000")
+    X, W = wl.make_inputs(w)
+    Y, ws, v, (Wq, cs), _ = run_path(L, X, W, w.tau)
+    C = host(L.debug_int8_gemm_i32(v["xq"], Wq, w.K))
+    r = oracle.mixed_matmul(X, W, w.tau)
+    assert np.array_equal(C.astype(np.int64), r["acc"])
+
+
+def test_outlier_overflow_sets_status_and_nan(L):
+    w = wl.get("tiny")
+    X, W = wl.make_inputs(w)
+    Y, ws, v, _, (st, flags) = run_path(L, X, W, w.tau, cap=1)
+    assert st == 5 and flags & 1
+    assert int(host(v["n_outlier"])[0]) == 2
+    assert np.isnan(host(Y).astype(np.float32)).all()
+    # the status word is cleared by reading it
+    assert L.llmint8_check_status(ws) == (0, 0)
+
+
+def test_repeat_calls_are_deterministic_and_reuse_workspace(L):
+    w = wl.get("ragged_129x257x520")
+    X, W = wl.make_inputs(w)
+    Wd = dev(W)
+    Wq, cs = L.quantize_weight_colwise(Wd)
+    ws = L.empty_workspace(w.M, w.N, w.K, w.K)
+    Xd = dev(X)
+    a = host(L.mixed_matmul(Xd, Wq, cs, Wd, w.tau, ws=ws)).view(np.uint16)
+    b = host(L.mixed_matmul(Xd, Wq, cs, Wd, w.tau, ws=ws)).view(np.uint16)
+    # a different X through the same workspace, then the first again
+    L.mixed_matmul(dev(wl.make_x(wl.get("ragged_129x257x520"))[::-1].copy()), Wq, cs, Wd, 3.0, ws=ws)
+    c = host(L.mixed_matmul(Xd, Wq, cs, Wd, w.tau, ws=ws)).view(np.uint16)
+    assert np.array_equal(a, b) and np.array_equal(a, c)
+    assert_status_ok(L, ws)
+
+
+# ------------------------------------------------------------------ full-size workloads (sampled rows)
+
+@pytest.mark.parametrize("name", ["ffn_6p7b_prefill", "sweep8k_o0", "sweep8k_o0p1", "sweep8k_o1"])
+def test_mixed_matmul_full_size(L, name):
+    w = wl.get(name)
+    X, W = wl.make_inputs(w)
+    rows = wl.sample_rows(w.M)
+    check_path(L, X, W, w.tau, rows=rows)
+    if name.startswith("sweep"):
+        check_path(L, X, W, np.inf, rows=rows)
+
+
+def test_mixed_matmul_full_size_175b(L):
+    w = wl.get("hidden_175b")
+    X, W = wl.make_inputs(w)
+    rows = wl.sample_rows(w.M, n=16)
+    check_path(L, X, W, w.tau, rows=rows)
