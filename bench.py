@@ -179,11 +179,22 @@ def oracle_sample(X, W, tau, rows, weight):
     return time.perf_counter() - t0
 
 
+def calibrate_rows(X, W, tau, weight, budget_s, M):
+    """Rows of the oracle sample that take about budget_s on this host (the
+    oracle parallelises over rows, so calibrate with one row per thread)."""
+    import oracle
+    nt = max(1, oracle.num_threads())
+    rows0 = min(M, nt)
+    t0 = oracle_sample(X, W, tau, rows0, weight)
+    per_row = max(t0, 1e-6) / rows0
+    rows = int(budget_s / per_row) // nt * nt
+    return int(max(rows0, min(M, rows)))
+
+
 def cpu_baseline(wl_, X, W, budget_s):
     import oracle
     weight = oracle.quantize_weight(W)  # offline conversion, not timed
-    t1 = oracle_sample(X, W, wl_.tau, 1, weight)
-    rows = int(max(1, min(wl_.M, budget_s / max(t1, 1e-6))))
+    rows = calibrate_rows(X, W, wl_.tau, weight, budget_s, wl_.M)
     t = oracle_sample(X, W, wl_.tau, rows, weight)
     tops = 2.0 * rows * wl_.N * wl_.K / t / 1e12
     return {"value": tops, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
@@ -201,9 +212,8 @@ def run_reference(args, wl_, dist):
     import workloads as wl
     X, W = wl.make_inputs(wl_)
     weight = oracle.quantize_weight(W)
-    t1 = oracle_sample(X, W, wl_.tau, 1, weight)
     per_step = min(0.5, 150.0 / max(1, args.steps + args.warmup))
-    rows = int(max(1, min(wl_.M, per_step / max(t1, 1e-6))))
+    rows = calibrate_rows(X, W, wl_.tau, weight, per_step, wl_.M)
     for _ in range(args.warmup):
         oracle_sample(X, W, wl_.tau, rows, weight)
     t0 = time.perf_counter()

@@ -228,7 +228,7 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   CUtensorMap tmA, tmB;
-  if (!encode_operand_map(&tmA, xq, M, K, L.ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, kGemmBN))
+  if (!encode_operand_map(&tmA, xq, M, K, L.ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, gemm_b_box_rows(static_cast<int>(M))))
     return LLMINT8_ERR_CUDA;
 
   cudaError_t e = launch_quantize_act(X, M, K, ldx, tau, xq, L.ldq, rs, O, outlier_cap, n_o, xo, L.ldo,
@@ -275,7 +275,7 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
   llmint8_status st = current_device(&num_sms);
   if (st != LLMINT8_OK) return st;
   CUtensorMap tmA, tmB;
-  if (!encode_operand_map(&tmA, Xq, M, K, ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, kGemmBN))
+  if (!encode_operand_map(&tmA, Xq, M, K, ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, gemm_b_box_rows(static_cast<int>(M))))
     return LLMINT8_ERR_CUDA;
   GemmArgs a = {};
   a.M = static_cast<int>(M);
@@ -309,7 +309,7 @@ llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const 
   llmint8_status st = current_device(&num_sms);
   if (st != LLMINT8_OK) return st;
   CUtensorMap tmA, tmB;
-  if (!encode_operand_map(&tmA, Xq, M, K, ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, kGemmBN))
+  if (!encode_operand_map(&tmA, Xq, M, K, ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, gemm_b_box_rows(static_cast<int>(M))))
     return LLMINT8_ERR_CUDA;
   GemmArgs a = {};
   a.M = static_cast<int>(M);

@@ -10,19 +10,31 @@
 // Mixed-precision decomposition: 16-bit matmul for the ~0.1 % outlier
 // dimensions, 8-bit for the other 99.9 %.
 //
-// Structure (one persistent CTA per SM, 192 threads):
-//   warp 0      TMA producer: Xq tile [128 x 128 B] + Wq tile [256 x 128 B]
-//               per stage into a 4-stage shared-memory ring (128-byte swizzle);
-//   warp 1      allocates 512 TMEM columns and issues tcgen05.mma kind::i8
-//               (M=128, N=256, K=32) from one thread; accumulators are double
-//               buffered (2 x 256 int32 columns) so the epilogue of tile i
-//               overlaps the main loop of tile i+1;
-//   warps 2-5   epilogue: tcgen05.ld of 32 columns at a time, dequantize with
-//               rs[i] * cs[j] / 127^2, add sum_t Xo[i,t] * W[O[t], j] (fp16
-//               operands, fp32 accumulation; W rows staged through shared
-//               memory), round once to fp16 and store.
-// Every mbarrier wait is bounded; a wait that gives up sets the status
-// word's timeout bit, raises a CTA abort flag and the CTA drains and exits.
+// Two tile shapes share one code path (kPair):
+//   single CTA   128 x 256 tile per CTA, MMA M=128 N=256 K=32, 4-stage ring of
+//                48 KB (Xq 128 x 128 B, Wq 256 x 128 B);
+//   CTA pair     256 x 256 tile per 2-CTA cluster (tcgen05 cta_group::2): each
+//                CTA loads 128 rows of Xq and 128 rows of Wq per stage (6-stage
+//                ring of 32 KB), the leader issues M=256 N=256 K=32 MMAs that
+//                read both CTAs' shared memory, and each CTA holds its 128 x 256
+//                half of the accumulator in its own TMEM.  Per-SM operand
+//                traffic per MAC is two thirds of the single-CTA tile's.
+// Roles (320 threads per CTA, one persistent CTA per SM):
+//   warp 0      TMA producer (128-byte swizzle, zero fill past the edges);
+//   warp 1      TMEM allocation (512 columns = 2 accumulators of 256 int32
+//               columns, so the epilogue of tile i overlaps the main loop of
+//               tile i+1) and, in the single CTA or the pair leader, the MMA
+//               issuer (one thread);
+//   warps 2-9   epilogue, two warps per TMEM lane quarter, 16 rows each:
+//               tcgen05.ld in the mma.m16n8 fragment layout, dequantize with
+//               rs[i] * cs[j] / 127^2, add the 16-bit outlier product
+//               sum_t Xo[i,t] * W[O[t], j] with warp-level tensor-core MMAs
+//               (fp16 operands, fp32 accumulation) straight into that
+//               fragment, round once to fp16 and store.  The tile's W rows,
+//               column scales, row scales and Xo fragments are fetched before
+//               the accumulator wait.
+// Every mbarrier wait is bounded; a wait that gives up sets the status word's
+// timeout bit, raises a CTA abort flag and the CTA drains and exits.
 #include <cuda_fp16.h>
 
 #include "kernels.cuh"
@@ -32,33 +44,44 @@ namespace llmint8 {
 
 namespace {
 
-constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK;
-constexpr int kStages = 4;
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
-constexpr uint32_t kBytesA = BM * BK;
-constexpr uint32_t kBytesB = BN * BK;
+constexpr int BM = kGemmBM;   // accumulator rows per CTA (TMEM lanes)
+constexpr int BN = kGemmBN;   // accumulator columns per CTA
+constexpr int BK = kGemmBK;   // K bytes per stage
+constexpr int kEpiWarps = 8;     // two per TMEM lane quarter, 16 rows each
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kAccCols = BN;
 constexpr uint32_t kTmemCols = 2 * kAccCols;
-constexpr int kOutT = 32;      // outlier rows of W staged per step
-constexpr int kChunk = 32;     // accumulator columns per tcgen05.ld
+constexpr int kChunk = 32;     // accumulator columns per tcgen05.ld (raw int32 epilogue)
+constexpr int kSG = 32;        // outlier rows of W staged per pass over a tile (two k16 MMA steps)
+constexpr int kWoStride = BN + 8;  // halves per staged row: 528 bytes, conflict-free ldmatrix
 
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffB = kOffA + kStages * kBytesA;
-constexpr uint32_t kOffWo = kOffB + kStages * kBytesB;
-constexpr uint32_t kOffBars = kOffWo + kOutT * kChunk * 2;
-constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;  // full, empty, tmem full, tmem empty, drain
-constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
-constexpr uint32_t kSmemUsed = kOffMisc + 16;
-constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack for 1024-byte alignment
-
-static_assert(kBytesA % 1024 == 0 && kBytesB % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+template <bool kPair>
+struct Geo {
+  static constexpr int kTileM = kPair ? 2 * BM : BM;      // rows of Y per tile
+  static constexpr int kRowsB = kPair ? BN / 2 : BN;      // rows of Wq loaded per CTA per stage
+  static constexpr int kStages = kPair ? 6 : 4;
+  static constexpr uint32_t kBytesA = BM * BK;
+  static constexpr uint32_t kBytesB = kRowsB * BK;
+  static constexpr uint32_t kOffA = 0;
+  static constexpr uint32_t kOffB = kOffA + kStages * kBytesA;
+  static constexpr uint32_t kOffWo = kOffB + kStages * kBytesB;     // fp16 [kSG][kWoStride]
+  static constexpr uint32_t kOffCs = kOffWo + kSG * kWoStride * 2;  // fp32 [BN]
+  static constexpr uint32_t kOffBars = kOffCs + BN * 4;
+  static constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;  // full, empty, tmem full/empty, drain
+  static constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
+  static constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+  // Arrivals that free a TMEM accumulator: one per epilogue warp of each CTA.
+  static constexpr uint32_t kTmemEmptyArrivals = kPair ? 2 * kEpiWarps : kEpiWarps;
+  static_assert(kBytesA % 1024 == 0 && kBytesB % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
 
 struct Shared {
   uint8_t* a;
   uint8_t* b;
-  __half* wo;
+  __half* wo;  // outlier rows of W over the tile's columns
+  float* cs;  // column scales of the tile
   uint64_t* full;
   uint64_t* empty;
   uint64_t* tfull;
@@ -68,20 +91,23 @@ struct Shared {
   volatile int* abort;
 };
 
+template <bool kPair>
 __device__ __forceinline__ Shared carve(uint8_t* raw) {
+  using G = Geo<kPair>;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   Shared s;
-  s.a = base + kOffA;
-  s.b = base + kOffB;
-  s.wo = reinterpret_cast<__half*>(base + kOffWo);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kOffBars);
+  s.a = base + G::kOffA;
+  s.b = base + G::kOffB;
+  s.wo = reinterpret_cast<__half*>(base + G::kOffWo);
+  s.cs = reinterpret_cast<float*>(base + G::kOffCs);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + G::kOffBars);
   s.full = bars;
-  s.empty = bars + kStages;
-  s.tfull = bars + 2 * kStages;
-  s.tempty = bars + 2 * kStages + 2;
-  s.drain = bars + 2 * kStages + 4;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
-  s.abort = reinterpret_cast<volatile int*>(base + kOffMisc + 4);
+  s.empty = bars + G::kStages;
+  s.tfull = bars + 2 * G::kStages;
+  s.tempty = bars + 2 * G::kStages + 2;
+  s.drain = bars + 2 * G::kStages + 4;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(base + G::kOffMisc);
+  s.abort = reinterpret_cast<volatile int*>(base + G::kOffMisc + 4);
   return s;
 }
 
@@ -105,50 +131,70 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, ui
   }
 }
 
+// Tiles are ordered with the M index fastest, so that the tiles in flight at
+// one time share their Wq columns and all of Xq stays in L2.
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int& mb, int& nb) {
   mb = tile % num_m;
   nb = tile / num_m;
 }
 
-__device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const Shared& s, int num_m,
-                             int num_tiles, int num_k, uint32_t* status) {
+struct Sched {
+  int first, stride, num_tiles, num_m, num_k;
+};
+
+template <bool kPair>
+__device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const Shared& s, const Sched& sc,
+                             uint32_t rank, uint32_t* status) {
+  using G = Geo<kPair>;
   const uint64_t hint = policy_evict_last();
   uint32_t stage = 0, phase = 0;
-  uint32_t issued = 0;            // bit s: stage s has had a load issued
-  uint32_t issued_phase = 0;      // bit s: the phase of that load
+  uint32_t issued = 0;        // bit s: stage s has had a load issued
+  uint32_t issued_phase = 0;  // bit s: the phase of that load
   bool ok = true;
-  for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+  for (int tile = sc.first; tile < sc.num_tiles && ok; tile += sc.stride) {
     int mb, nb;
-    tile_coords(tile, num_m, mb, nb);
-    for (int kb = 0; kb < num_k; ++kb) {
+    tile_coords(tile, sc.num_m, mb, nb);
+    const int ya = mb * G::kTileM + (kPair ? static_cast<int>(rank) * BM : 0);
+    const int yb = nb * BN + (kPair ? static_cast<int>(rank) * G::kRowsB : 0);
+    for (int kb = 0; kb < sc.num_k; ++kb) {
       if (!wait_or_abort(&s.empty[stage], phase ^ 1u, status, s.abort)) {
         ok = false;
         break;
       }
-      mbar_arrive_expect_tx(&s.full[stage], kBytesA + kBytesB);
-      tma_load_2d(s.a + stage * kBytesA, tmA, &s.full[stage], kb * BK, mb * BM, hint);
-      tma_load_2d(s.b + stage * kBytesB, tmB, &s.full[stage], kb * BK, nb * BN, hint);
+      if constexpr (kPair) {
+        // both CTAs' bytes are counted on the leader's full barrier
+        if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * (G::kBytesA + G::kBytesB));
+        const uint32_t bar = mapa_shared(smem_u32(&s.full[stage]), 0);
+        tma_load_2d_pair(s.a + stage * G::kBytesA, tmA, bar, kb * BK, ya, hint);
+        tma_load_2d_pair(s.b + stage * G::kBytesB, tmB, bar, kb * BK, yb, hint);
+      } else {
+        mbar_arrive_expect_tx(&s.full[stage], G::kBytesA + G::kBytesB);
+        tma_load_2d(s.a + stage * G::kBytesA, tmA, &s.full[stage], kb * BK, ya, hint);
+        tma_load_2d(s.b + stage * G::kBytesB, tmB, &s.full[stage], kb * BK, yb, hint);
+      }
       issued |= 1u << stage;
       issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-      if (++stage == kStages) {
+      if (++stage == G::kStages) {
         stage = 0;
         phase ^= 1u;
       }
     }
   }
-  if (!ok) {
+  if (!ok && (!kPair || rank == 0)) {
     // Let the copies already in flight land before the CTA exits.
-    for (int st = 0; st < kStages; ++st)
+    for (int st = 0; st < G::kStages; ++st)
       if (issued & (1u << st)) mbar_wait(&s.full[st], (issued_phase >> st) & 1u, nullptr);
   }
 }
 
-__device__ void run_mma(const Shared& s, uint32_t tmem_base, int num_tiles, int num_k, uint32_t* status) {
-  constexpr uint32_t idesc = idesc_i8(BM, BN);
+template <bool kPair>
+__device__ void run_mma(const Shared& s, uint32_t tmem_base, const Sched& sc, uint32_t* status) {
+  using G = Geo<kPair>;
+  constexpr uint32_t idesc = idesc_i8(G::kTileM, BN);
   uint32_t stage = 0, phase = 0, it = 0;
   bool ok = true;
   bool any = false;
-  for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+  for (int tile = sc.first; tile < sc.num_tiles && ok; tile += sc.stride, ++it) {
     const uint32_t b = it & 1u;
     const uint32_t use = (it >> 1) & 1u;
     if (!wait_or_abort(&s.tempty[b], use ^ 1u, status, s.abort)) {
@@ -157,74 +203,197 @@ __device__ void run_mma(const Shared& s, uint32_t tmem_base, int num_tiles, int 
     }
     tc_fence_after();
     const uint32_t d = tmem_base + b * kAccCols;
-    for (int kb = 0; kb < num_k; ++kb) {
+    for (int kb = 0; kb < sc.num_k; ++kb) {
       if (!wait_or_abort(&s.full[stage], phase, status, s.abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint64_t da = smem_desc_k_sw128(smem_u32(s.a + stage * kBytesA));
-      const uint64_t db = smem_desc_k_sw128(smem_u32(s.b + stage * kBytesB));
+      const uint64_t da = smem_desc_k_sw128(smem_u32(s.a + stage * G::kBytesA));
+      const uint64_t db = smem_desc_k_sw128(smem_u32(s.b + stage * G::kBytesB));
 #pragma unroll
       for (int kk = 0; kk < BK / 32; ++kk) {
         // +32 bytes along K inside the 128-byte swizzle atom = +2 in the
         // descriptor's 16-byte address units.
-        mma_i8(d, da + 2u * kk, db + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+        if constexpr (kPair)
+          mma_i8_pair(d, da + 2u * kk, db + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+        else
+          mma_i8(d, da + 2u * kk, db + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
       }
       any = true;
-      mma_commit(&s.empty[stage]);
-      if (++stage == kStages) {
+      if constexpr (kPair)
+        mma_commit_pair(&s.empty[stage], 0x3);
+      else
+        mma_commit(&s.empty[stage]);
+      if (++stage == G::kStages) {
         stage = 0;
         phase ^= 1u;
       }
     }
-    if (ok) mma_commit(&s.tfull[b]);
+    if (ok) {
+      if constexpr (kPair)
+        mma_commit_pair(&s.tfull[b], 0x3);
+      else
+        mma_commit(&s.tfull[b]);
+    }
   }
   if (!ok && any) {
     // Make sure no MMA is still writing TMEM before it is freed.
-    mma_commit(s.drain);
+    if constexpr (kPair)
+      mma_commit_pair(s.drain, 0x1);
+    else
+      mma_commit(s.drain);
     mbar_wait(s.drain, 0, nullptr);
   }
 }
 
-template <bool kRaw>
-__device__ void run_epilogue(const GemmArgs& p, const Shared& s, uint32_t tmem_base, int num_m, int num_tiles,
-                             uint32_t warp, uint32_t lane) {
-  const uint32_t q = warp & 3u;  // TMEM lane quarter this warp may access
-  const int et = static_cast<int>(threadIdx.x) - 64;  // 0..127
+// Column scales of the tile into shared memory.
+__device__ __forceinline__ void stage_scales(const GemmArgs& p, const Shared& s, int nb, int et, bool cs_vec) {
+  const int n0 = nb * BN;
+  if (et < BN / 4) {
+    const int c = n0 + 4 * et;
+    float4 v;
+    if (cs_vec && c + 4 <= p.N) {
+      v = __ldg(reinterpret_cast<const float4*>(p.cs + c));
+    } else {
+      v.x = c < p.N ? __ldg(p.cs + c) : 0.0f;
+      v.y = c + 1 < p.N ? __ldg(p.cs + c + 1) : 0.0f;
+      v.z = c + 2 < p.N ? __ldg(p.cs + c + 2) : 0.0f;
+      v.w = c + 3 < p.N ? __ldg(p.cs + c + 3) : 0.0f;
+    }
+    *reinterpret_cast<float4*>(s.cs + 4 * et) = v;
+  }
+}
+
+// Outlier rows O[t0 .. t0+tn) of W over the tile's BN columns into shared
+// memory (fp16, rows kWoStride apart); rows up to the next multiple of 16 are
+// zero so that a partly used k16 step adds exact zeros.
+__device__ __forceinline__ void stage_outlier_rows(const GemmArgs& p, const Shared& s, int nb, int t0, int tn,
+                                                   int et, bool w_vec) {
+  const __half* W = static_cast<const __half*>(p.W);
+  const int n0 = nb * BN;
+  const int rows = (tn + 15) & ~15;
+  const int pieces = rows * (BN / 8);  // 8 columns each
+  for (int pc = et; pc < pieces; pc += kEpiThreads) {
+    const int t = pc / (BN / 8);
+    const int cc = 8 * (pc % (BN / 8));
+    const int c = n0 + cc;
+    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    if (t < tn) {
+      const __half* wr = W + static_cast<int64_t>(__ldg(p.O + t0 + t)) * p.ldw + c;
+      if (w_vec && c + 8 <= p.N) {
+        u = __ldg(reinterpret_cast<const uint4*>(wr));
+      } else {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t lo = (c + 2 * e < p.N) ? __half_as_ushort(wr[2 * e]) : 0u;
+          const uint32_t hi = (c + 2 * e + 1 < p.N) ? __half_as_ushort(wr[2 * e + 1]) : 0u;
+          w[e] = lo | (hi << 16);
+        }
+        u = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    *reinterpret_cast<uint4*>(s.wo + t * kWoStride + cc) = u;
+  }
+}
+
+// Exact int32 -> fp32 for |a| < 2^22 by the exponent-bias trick (two full-rate
+// operations instead of one conversion-pipe instruction); falls back to the
+// conversion instruction otherwise.  Both give the exact value whenever it is
+// representable; the int32 accumulator needs |a| <= 127^2 K.
+__device__ __forceinline__ float i2f_exact(int32_t a) {
+  if (static_cast<uint32_t>(a) + (1u << 22) < (1u << 23))
+    return __fsub_rn(__int_as_float(0x4B400000 + a), 12582912.0f);
+  return static_cast<float>(a);
+}
+
+// A fragment (16 rows x 16 outliers, fp16) of mma.m16n8k16 for rows r0..r0+15
+// and outliers k0..k0+15 of the gathered Xo; outliers at or past `kend` and
+// rows past M read as zero.
+__device__ __forceinline__ void load_xo_fragment(const GemmArgs& p, int r0, int k0, int kend, uint32_t lane,
+                                                 uint32_t (&a)[4]) {
+  const __half* Xo = static_cast<const __half*>(p.Xo);
+  const int g = static_cast<int>(lane >> 2), t4 = static_cast<int>(lane & 3);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + g + ((i & 1) ? 8 : 0);
+    const int k = k0 + 2 * t4 + ((i & 2) ? 8 : 0);
+    uint32_t lo = 0u, hi = 0u;
+    if (r < p.M) {
+      const __half* x = Xo + static_cast<int64_t>(r) * p.ldo;
+      if (k < kend) lo = __half_as_ushort(x[k]);
+      if (k + 1 < kend) hi = __half_as_ushort(x[k + 1]);
+    }
+    a[i] = lo | (hi << 16);
+  }
+}
+
+template <bool kRaw, bool kPair>
+__device__ void run_epilogue(const GemmArgs& p, const Shared& s, uint32_t tmem_base, const Sched& sc,
+                             uint32_t rank, uint32_t warp, uint32_t lane) {
+  using G = Geo<kPair>;
+  const uint32_t q = warp & 3u;             // TMEM lane quarter this warp may access
+  const int ab = static_cast<int>(warp - 2) >> 2;  // which 16 rows of the quarter
+  const int et = static_cast<int>(threadIdx.x) - 64;  // 0..kEpiThreads-1
   const int n_o = kRaw ? 0 : *p.n_o;
   const bool overflow = n_o > p.cap;
   const int n_use = overflow ? 0 : n_o;
-  const __half* W = static_cast<const __half*>(p.W);
-  const __half* Xo = static_cast<const __half*>(p.Xo);
+  const int passes = n_use > 0 ? (n_use + kSG - 1) / kSG : 1;  // outlier row groups staged per tile
   __half* Y = static_cast<__half*>(p.Y);
-  const bool y_vec = (p.ldy % 8 == 0) && (reinterpret_cast<uintptr_t>(p.Y) % 16 == 0);
+  const bool y_pair = (p.ldy % 2 == 0) && (reinterpret_cast<uintptr_t>(p.Y) % 4 == 0);
   const bool w_vec = (p.ldw % 8 == 0) && (reinterpret_cast<uintptr_t>(p.W) % 16 == 0);
   const bool c_vec = (p.ldc % 4 == 0) && (reinterpret_cast<uintptr_t>(p.C) % 16 == 0);
+  const bool cs_vec = (reinterpret_cast<uintptr_t>(p.cs) % 16 == 0);
+  const int g = static_cast<int>(lane >> 2), t4 = static_cast<int>(lane & 3);
+  // the pair leader's TMEM-empty barriers collect the arrivals of both CTAs
+  const uint32_t tempty_leader = kPair ? mapa_shared(smem_u32(s.tempty), 0) : smem_u32(s.tempty);
+  // ldmatrix row address of this lane inside a 16 x 16 block of staged W rows
+  const uint32_t wo_lane = smem_u32(s.wo) + 2u * static_cast<uint32_t>(((lane & 7) + 8 * ((lane >> 3) & 1)) *
+                                                                          kWoStride + 8 * (lane >> 4));
 
   uint32_t it = 0;
-  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+  for (int tile = sc.first; tile < sc.num_tiles; tile += sc.stride, ++it) {
     const uint32_t b = it & 1u;
     const uint32_t use = (it >> 1) & 1u;
-    const bool got = wait_or_abort(&s.tfull[b], use, p.status, s.abort);
-    if (!named_bar_and(2, kEpiThreads, got)) break;  // all epilogue threads stop together
-    tc_fence_after();
     int mb, nb;
-    tile_coords(tile, num_m, mb, nb);
-    const int row = mb * BM + static_cast<int>(q * 32 + lane);
-    const bool row_ok = row < p.M;
-    float rsc = 0.0f;
-    if (!kRaw && row_ok) rsc = p.rs[row] * (1.0f / 16129.0f);
+    tile_coords(tile, sc.num_m, mb, nb);
+    const int wrow0 = mb * G::kTileM + (kPair ? static_cast<int>(rank) * BM : 0) + static_cast<int>(q * 32);
+    const int r0 = wrow0 + 16 * ab;  // this warp's 16 rows
+    const uint32_t tacc = tmem_base + ((q * 32u + 16u * ab) << 16) + b * kAccCols;
 
+    // Everything but the accumulator is fetched before waiting for it.
+    float rsc[2] = {0.0f, 0.0f};  // rows g, g + 8
+    uint32_t afr[2][4];           // Xo fragments of the first pass (two k16 steps)
+    if constexpr (!kRaw) {
+      named_bar_sync(1, kEpiThreads);  // the previous tile's readers of the staged data are done
+      stage_scales(p, s, nb, et, cs_vec);
+      stage_outlier_rows(p, s, nb, 0, min(n_use, kSG), et, w_vec);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = r0 + g + 8 * h;
+        if (r < p.M) rsc[h] = __ldg(p.rs + r) * (1.0f / 16129.0f);
+      }
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks)
+        if (16 * ks < min(n_use, kSG)) load_xo_fragment(p, r0, 16 * ks, min(n_use, kSG), lane, afr[ks]);
+    }
+
+    const bool got = wait_or_abort(&s.tfull[b], use, p.status, s.abort);
+    if (!named_bar_and(2, kEpiThreads, got)) break;  // all epilogue threads stop together; staged data visible
+    tc_fence_after();
+
+    if constexpr (kRaw) {
+      // the lane quarter's 32 rows, columns split between its two warps
+      const int row = wrow0 + static_cast<int>(lane);
+      const uint32_t traw = tmem_base + ((q * 32u) << 16) + b * kAccCols;
 #pragma unroll 1
-    for (int c = 0; c < BN / kChunk; ++c) {
-      const int col0 = nb * BN + c * kChunk;
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem_base + ((q * 32u) << 16) + b * kAccCols + c * kChunk, v);
-      tmem_ld_wait();
-
-      if constexpr (kRaw) {
-        if (row_ok) {
+      for (int c = ab * (BN / kChunk / 2); c < (ab + 1) * (BN / kChunk / 2); ++c) {
+        const int col0 = nb * BN + c * kChunk;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(traw + c * kChunk, v);
+        tmem_ld_wait();
+        if (row < p.M) {
           int32_t* dst = p.C + static_cast<int64_t>(row) * p.ldc + col0;
           if (c_vec && col0 + kChunk <= p.N) {
 #pragma unroll
@@ -235,103 +404,130 @@ __device__ void run_epilogue(const GemmArgs& p, const Shared& s, uint32_t tmem_b
               if (col0 + j < p.N) dst[j] = static_cast<int32_t>(v[j]);
           }
         }
-        continue;
-      } else {
-        float y[32];
+      }
+    } else {
+#pragma unroll 1
+      for (int ps = 0; ps < passes; ++ps) {
+        const int t0 = ps * kSG;
+        const int tn = min(kSG, n_use - t0);
+        const int ksteps = tn > 0 ? (tn + 15) / 16 : 0;
+        const bool last = ps == passes - 1;
+        if (ps > 0) {
+          named_bar_sync(1, kEpiThreads);  // the previous pass's rows are no longer read
+          stage_outlier_rows(p, s, nb, t0, tn, et, w_vec);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float csj = (col0 + j < p.N) ? __ldg(p.cs + col0 + j) : 0.0f;
-          y[j] = static_cast<float>(static_cast<int32_t>(v[j])) * rsc * csj;
+          for (int ks = 0; ks < 2; ++ks)
+            if (ks < ksteps) load_xo_fragment(p, r0, t0 + 16 * ks, t0 + tn, lane, afr[ks]);
+          named_bar_sync(1, kEpiThreads);
         }
-        // 16-bit outlier product: y += sum_t Xo[row, t] * W[O[t], cols]
-        for (int t0 = 0; t0 < n_use; t0 += kOutT) {
-          named_bar_sync(1, kEpiThreads);  // previous step's readers are done
-          {
-            const int tt = et >> 2;
-            const int seg = (et & 3) * 8;
-            const int t = t0 + tt;
-            __half h[8];
+        {
+#pragma unroll 1
+          for (int c = 0; c < BN / 64; ++c) {  // 64 accumulator columns at a time
+            const uint32_t taddr = tacc + c * 64;
+            uint32_t v[32];
+            tmem_ld_16x256b_x8(taddr, v);
+            tmem_ld_wait();
+            float d[8][4];
+            if (ps == 0) {
+              // dequantize: acc * rs[row] * cs[col] / 127^2
 #pragma unroll
-            for (int e = 0; e < 8; ++e) h[e] = __ushort_as_half(0);
-            if (t < n_use) {
-              const __half* wr = W + static_cast<int64_t>(p.O[t]) * p.ldw + col0 + seg;
-              if (w_vec && col0 + seg + 8 <= p.N) {
-                const uint4 u = __ldg(reinterpret_cast<const uint4*>(wr));
-                const __half* hp = reinterpret_cast<const __half*>(&u);
+              for (int n = 0; n < 8; ++n) {
+                const float2 c2 = *reinterpret_cast<const float2*>(s.cs + c * 64 + 8 * n + 2 * t4);
+                d[n][0] = i2f_exact(static_cast<int32_t>(v[4 * n + 0])) * rsc[0] * c2.x;
+                d[n][1] = i2f_exact(static_cast<int32_t>(v[4 * n + 1])) * rsc[0] * c2.y;
+                d[n][2] = i2f_exact(static_cast<int32_t>(v[4 * n + 2])) * rsc[1] * c2.x;
+                d[n][3] = i2f_exact(static_cast<int32_t>(v[4 * n + 3])) * rsc[1] * c2.y;
+              }
+            } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) h[e] = hp[e];
-              } else {
+              for (int n = 0; n < 8; ++n)
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                  if (col0 + seg + e < p.N) h[e] = wr[e];
+                for (int e = 0; e < 4; ++e) d[n][e] = __uint_as_float(v[4 * n + e]);
+            }
+            // 16-bit outlier product on the tensor cores: d += Xo[rows, k] * W[O[k], cols]
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+              if (ks < ksteps) {
+#pragma unroll
+                for (int np = 0; np < 4; ++np) {
+                  uint32_t b0, b1, b2, b3;
+                  ldmatrix_x4_trans(wo_lane + 2u * static_cast<uint32_t>(16 * ks * kWoStride + c * 64 + 16 * np),
+                                    b0, b1, b2, b3);
+                  mma_m16n8k16_f16f32(d[2 * np], afr[ks], b0, b1);
+                  mma_m16n8k16_f16f32(d[2 * np + 1], afr[ks], b2, b3);
+                }
               }
             }
+            if (last) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) s.wo[tt * kChunk + seg + e] = h[e];
-          }
-          named_bar_sync(1, kEpiThreads);
-          const int tn = min(kOutT, n_use - t0);
-          for (int tt = 0; tt < tn; ++tt) {
-            const float xo = row_ok ? __half2float(Xo[static_cast<int64_t>(row) * p.ldo + t0 + tt]) : 0.0f;
-            const __half2* wv = reinterpret_cast<const __half2*>(s.wo + tt * kChunk);
+              for (int h = 0; h < 2; ++h) {
+                const int r = r0 + g + 8 * h;
+                if (r < p.M) {
+                  __half* yr = Y + static_cast<int64_t>(r) * p.ldy;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float2 w2 = __half22float2(wv[j]);
-              y[2 * j] = fmaf(xo, w2.x, y[2 * j]);
-              y[2 * j + 1] = fmaf(xo, w2.y, y[2 * j + 1]);
+                  for (int n = 0; n < 8; ++n) {
+                    const int col = nb * BN + c * 64 + 8 * n + 2 * t4;
+                    float y0 = d[n][2 * h], y1 = d[n][2 * h + 1];
+                    if (overflow) y0 = y1 = __int_as_float(0x7fc00000);
+                    if (y_pair && col + 1 < p.N) {
+                      *reinterpret_cast<__half2*>(yr + col) = __floats2half2_rn(y0, y1);
+                    } else {
+                      if (col < p.N) yr[col] = __float2half_rn(y0);
+                      if (col + 1 < p.N) yr[col + 1] = __float2half_rn(y1);
+                    }
+                  }
+                }
+              }
+            } else {
+              // park the partial sum in the accumulator's own TMEM columns
+#pragma unroll
+              for (int n = 0; n < 8; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) v[4 * n + e] = __float_as_uint(d[n][e]);
+              tmem_st_16x256b_x8(taddr, v);
             }
           }
         }
-        if (overflow) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) y[j] = __int_as_float(0x7fc00000);
-        }
-        if (row_ok) {
-          __half* dst = Y + static_cast<int64_t>(row) * p.ldy + col0;
-          if (y_vec && col0 + kChunk <= p.N) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              uint4 u;
-              __half2* h2 = reinterpret_cast<__half2*>(&u);
-              h2[0] = __floats2half2_rn(y[j], y[j + 1]);
-              h2[1] = __floats2half2_rn(y[j + 2], y[j + 3]);
-              h2[2] = __floats2half2_rn(y[j + 4], y[j + 5]);
-              h2[3] = __floats2half2_rn(y[j + 6], y[j + 7]);
-              *reinterpret_cast<uint4*>(dst + j) = u;
-            }
-          } else {
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j < p.N) dst[j] = __float2half_rn(y[j]);
-          }
-        }
+        if (!last) tmem_st_wait();
       }
     }
+    // this warp's TMEM reads of buffer b are complete: free it for the MMA
     tc_fence_before();
-    mbar_arrive(&s.tempty[b]);
+    __syncwarp();
+    if (lane == 0) {
+      if constexpr (kPair)
+        mbar_arrive_cluster(tempty_leader + b * 8u);
+      else
+        mbar_arrive(&s.tempty[b]);
+    }
   }
 }
 
-template <bool kRaw>
+template <bool kRaw, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmArgs p) {
+  using G = Geo<kPair>;
   extern __shared__ uint8_t smem_raw[];
-  const Shared s = carve(smem_raw);
+  const Shared s = carve<kPair>(smem_raw);
   const uint32_t warp = warp_id_sync();
   const uint32_t lane = lane_id();
-  const int num_m = (p.M + BM - 1) / BM;
-  const int num_n = (p.N + BN - 1) / BN;
-  const int num_k = (p.K + BK - 1) / BK;
-  const int num_tiles = num_m * num_n;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  Sched sc;
+  sc.num_m = (p.M + G::kTileM - 1) / G::kTileM;
+  sc.num_k = (p.K + BK - 1) / BK;
+  sc.num_tiles = sc.num_m * ((p.N + BN - 1) / BN);
+  sc.first = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  sc.stride = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < G::kStages; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.tfull[i], 1);
-      mbar_init(&s.tempty[i], kEpiThreads);
+      mbar_init(&s.tempty[i], G::kTmemEmptyArrivals);
     }
     mbar_init(s.drain, 1);
     *s.abort = 0;
@@ -340,61 +536,123 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(s.tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(s.tmem_slot, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(s.tmem_slot, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();  // the peer's barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem_base = *s.tmem_slot;
 
   griddep_wait();  // Xq, rs, O, n_o and Xo are written by the quantize kernel
 
   if (warp == 0) {
-    if (lane == 0) run_producer(&tmA, &tmB, s, num_m, num_tiles, num_k, p.status);
+    if (lane == 0) run_producer<kPair>(&tmA, &tmB, s, sc, rank, p.status);
   } else if (warp == 1) {
-    if (lane == 0) run_mma(s, tmem_base, num_tiles, num_k, p.status);
+    if (lane == 0 && rank == 0) run_mma<kPair>(s, tmem_base, sc, p.status);
   } else {
-    run_epilogue<kRaw>(p, s, tmem_base, num_m, num_tiles, warp, lane);
+    run_epilogue<kRaw, kPair>(p, s, tmem_base, sc, rank, warp, lane);
   }
 
+  tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();  // no CTA leaves while its pair may still signal it
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (kPair)
+      tmem_dealloc_pair(tmem_base, kTmemCols);
+    else
+      tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
-}  // namespace
-
-cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, bool raw_i32,
-                           int num_sms, cudaStream_t stream, bool pdl) {
-  static bool attr_set[2][64] = {};  // per kernel variant and device
-  auto kern = raw_i32 ? gemm_i8_kernel<true> : gemm_i8_kernel<false>;
+template <bool kRaw, bool kPair>
+cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
+                           cudaStream_t stream, bool pdl) {
+  using G = Geo<kPair>;
+  static bool attr_set[64] = {};  // per device
+  static int max_units[64] = {};  // CTAs (or CTA pairs) that fit at once, per device
+  auto kern = gemm_i8_kernel<kRaw, kPair>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[raw_i32][dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::kSmemBytes));
     if (e != cudaSuccess) return e;
-    attr_set[raw_i32][dev] = true;
+    if (kPair) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+      if (e != cudaSuccess) return e;
+    }
+    max_units[dev] = kPair ? num_sms / 2 : num_sms;
+    if (kPair) {
+      // a persistent grid must be co-resident: ask how many pairs fit
+      cudaLaunchAttribute ca;
+      ca.id = cudaLaunchAttributeClusterDimension;
+      ca.val.clusterDim.x = 2;
+      ca.val.clusterDim.y = 1;
+      ca.val.clusterDim.z = 1;
+      cudaLaunchConfig_t oc = {};
+      oc.gridDim = dim3(static_cast<unsigned>(num_sms));
+      oc.blockDim = dim3(kThreads);
+      oc.dynamicSmemBytes = G::kSmemBytes;
+      oc.attrs = &ca;
+      oc.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &oc) == cudaSuccess && n > 0 && n < max_units[dev])
+        max_units[dev] = n;
+      (void)cudaGetLastError();
+    }
+    attr_set[dev] = true;
   }
-  const int num_tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
-  const int grid = num_tiles < num_sms ? num_tiles : num_sms;
+  const int num_tiles = ((a.M + G::kTileM - 1) / G::kTileM) * ((a.N + BN - 1) / BN);
+  const int units = max_units[dev];  // CTAs or CTA pairs that run at once
+  const int grid = (num_tiles < units ? num_tiles : units) * (kPair ? 2 : 1);
 
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int n_attr = 0;
+  if (pdl) {
+    attr[n_attr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n_attr].val.programmaticStreamSerializationAllowed = 1;
+    ++n_attr;
+  }
+  if (kPair) {
+    attr[n_attr].id = cudaLaunchAttributeClusterDimension;
+    attr[n_attr].val.clusterDim.x = 2;
+    attr[n_attr].val.clusterDim.y = 1;
+    attr[n_attr].val.clusterDim.z = 1;
+    ++n_attr;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = G::kSmemBytes;
   cfg.stream = stream;
-  cfg.attrs = pdl ? attr : nullptr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.attrs = n_attr ? attr : nullptr;
+  cfg.numAttrs = n_attr;
   return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
+}
+
+}  // namespace
+
+bool gemm_uses_pair(int M) { return M > BM; }
+
+cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, bool raw_i32,
+                           int num_sms, cudaStream_t stream, bool pdl) {
+  const bool pair = gemm_uses_pair(a.M);
+  if (raw_i32) {
+    return pair ? launch_variant<true, true>(tmA, tmB, a, num_sms, stream, pdl)
+                : launch_variant<true, false>(tmA, tmB, a, num_sms, stream, pdl);
+  }
+  return pair ? launch_variant<false, true>(tmA, tmB, a, num_sms, stream, pdl)
+              : launch_variant<false, false>(tmA, tmB, a, num_sms, stream, pdl);
 }
 
 }  // namespace llmint8

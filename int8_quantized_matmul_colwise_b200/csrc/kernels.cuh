@@ -42,14 +42,21 @@ struct GemmArgs {
   uint32_t* status;
 };
 
-// tmA: Xq [M rows, K cols] int8, tmB: Wq [N rows, K cols] int8, both encoded
-// by encode_operand_map().  raw_i32 selects the accumulator-dump epilogue.
+// Whether the GEMM for M rows runs as CTA pairs (256 x 256 tiles, cta_group::2)
+// rather than single CTAs (128 x 256 tiles).
+bool gemm_uses_pair(int M);
+
+// tmA: Xq [M rows, K cols] int8 in boxes of 128 rows, tmB: Wq [N rows, K cols]
+// int8 in boxes of gemm_b_box_rows(M) rows, 128 bytes along K, 128-byte
+// swizzle.  raw_i32 selects the accumulator-dump epilogue.
 cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, bool raw_i32,
                            int num_sms, cudaStream_t stream, bool pdl);
 
-// Tile sizes of the GEMM (rows of Xq / rows of Wq per tile, K bytes per stage).
+// Tile sizes of the GEMM per CTA (accumulator rows / columns, K bytes per stage).
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 128;
+
+inline unsigned gemm_b_box_rows(int M) { return gemm_uses_pair(M) ? kGemmBN / 2 : kGemmBN; }
 
 }  // namespace llmint8

@@ -19,6 +19,7 @@ namespace llmint8 {
 //    exactly.  __fmul_rn/__fadd_rn keep the compiler from fusing them.
 __device__ __forceinline__ int quantize_exact(float x, float s, float inv_s) {
   const float t = __fmul_rn(127.0f, fabsf(x));
+  if (!(t == t)) return 0;  // NaN input: code 0
   float q = rintf(__fmul_rn(t, inv_s));
   if (__fmul_rn(__fadd_rn(q, 0.5f), s) <= t) {
     q = __fadd_rn(q, 1.0f);
@@ -28,6 +29,18 @@ __device__ __forceinline__ int quantize_exact(float x, float s, float inv_s) {
   q = fminf(q, 127.0f);
   const int qi = __float2int_rz(q);
   return x < 0.0f ? -qi : qi;
+}
+
+// The same code with a cheap common path.  k = fl(127 / s); r = x * k is
+// within 2^-22 relative (|r| <= 127 + 2^-15) of the exact 127 x / s, so when r
+// is farther than 2^-10 from a half-integer, rint(r) is the nearest integer of
+// the exact value and there is no tie: the code is rint(r).  Otherwise (about
+// one value in 500) the exact comparisons of quantize_exact decide.
+__device__ __forceinline__ int quantize_fast(float x, float s, float inv_s, float k) {
+  const float r = __fmul_rn(x, k);
+  const float q = rintf(r);
+  if (fabsf(__fadd_rn(r, -q)) < 0.4990234375f) return __float2int_rz(q);  // 0.5 - 2^-10
+  return quantize_exact(x, s, inv_s);
 }
 
 // Pack four codes (low byte first) into a 32-bit word.
