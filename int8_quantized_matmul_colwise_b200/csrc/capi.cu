@@ -84,9 +84,31 @@ bool encode_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp16 output Y [rows, cols] with row stride ld (elements), written in boxes of
+// 16 rows x 64 columns with the 128-byte swizzle.  Needs 16-byte aligned rows.
+bool encode_output_map(CUtensorMap* map, void* base, int64_t rows, int64_t cols, int64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Y through TMA stores when its rows are 16-byte aligned; direct stores otherwise.
+bool prepare_output(CUtensorMap* map, void* Y, int64_t M, int64_t N, int64_t ldy) {
+  std::memset(map, 0, sizeof(*map));
+  if (ldy % 8 != 0 || !aligned(Y, 16)) return false;
+  return encode_output_map(map, Y, M, N, ldy);
+}
+
 // ------------------------------------------------------------------ workspace
-// [0, 256)        header: status u32 @0, scan counter u32 @4, n_o i32 @8
-// colmax          u32 [K]
+// [0, 256)        header: status u32 @0, n_o i32 @8
+// colmax          u32 [K]                 zero between calls
+// blk_counter     u32 [ceil(K/256)]       zero between calls
 // bitmask         u32 [ceil(K/32)]
 // outlier_idx     i32 [cap]
 // row_scale       f32 [M]
@@ -97,6 +119,7 @@ bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t
   size_t off = 256;
   *colmax = off;
   off = align_up(off + 4 * size_t(K), 256);
+  off = align_up(off + 4 * size_t((K + 255) / 256), 256);  // block counters follow colmax
   *bitmask = off;
   off = align_up(off + 4 * size_t((K + 31) / 32), 256);
   L->status = 0;
@@ -115,12 +138,12 @@ bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t
   return true;
 }
 
-ActWs act_ws(void* ws, size_t colmax_off, size_t bitmask_off) {
+ActWs act_ws(void* ws, size_t colmax_off, size_t bitmask_off, int64_t K) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   ActWs a;
   a.status = reinterpret_cast<uint32_t*>(b);
-  a.counter = reinterpret_cast<uint32_t*>(b + 4);
   a.colmax = reinterpret_cast<uint32_t*>(b + colmax_off);
+  a.blk_counter = reinterpret_cast<uint32_t*>(b + align_up(colmax_off + 4 * size_t(K), 256));
   a.bitmask = reinterpret_cast<uint32_t*>(b + bitmask_off);
   return a;
 }
@@ -195,7 +218,7 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
   llmint8_status st = current_device(nullptr);
   if (st != LLMINT8_OK) return st;
   return cuda_status(launch_quantize_act(X, M, K, ldx, tau, Xq, ldq, row_scale, outlier_idx, outlier_cap,
-                                         n_outlier, Xo, ldo, act_ws(ws, colmax, bitmask),
+                                         n_outlier, Xo, ldo, act_ws(ws, colmax, bitmask, K),
                                          static_cast<cudaStream_t>(stream), true));
 }
 
@@ -232,7 +255,7 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
     return LLMINT8_ERR_CUDA;
 
   cudaError_t e = launch_quantize_act(X, M, K, ldx, tau, xq, L.ldq, rs, O, outlier_cap, n_o, xo, L.ldo,
-                                      act_ws(ws, colmax_off, bitmask_off), s, true);
+                                      act_ws(ws, colmax_off, bitmask_off, K), s, true);
   if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
 
   GemmArgs a = {};
@@ -253,7 +276,9 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
   a.C = nullptr;
   a.ldc = 0;
   a.status = reinterpret_cast<uint32_t*>(b + L.status);
-  return cuda_status(launch_gemm_i8(tmA, tmB, a, false, num_sms, s, true));
+  CUtensorMap tmY;
+  a.y_tma = prepare_output(&tmY, Y, M, N, ldy);
+  return cuda_status(launch_gemm_i8(tmA, tmB, tmY, a, false, num_sms, s, true));
 }
 
 llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* row_scale,
@@ -293,7 +318,9 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
   a.Y = Y;
   a.ldy = ldy;
   a.status = static_cast<uint32_t*>(ws);
-  return cuda_status(launch_gemm_i8(tmA, tmB, a, false, num_sms, static_cast<cudaStream_t>(stream), true));
+  CUtensorMap tmY;
+  a.y_tma = prepare_output(&tmY, Y, M, N, ldy);
+  return cuda_status(launch_gemm_i8(tmA, tmB, tmY, a, false, num_sms, static_cast<cudaStream_t>(stream), true));
 }
 
 llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const int8_t* Wq, int64_t ldk,
@@ -318,7 +345,10 @@ llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const 
   a.C = C;
   a.ldc = ldc;
   a.status = static_cast<uint32_t*>(ws);
-  return cuda_status(launch_gemm_i8(tmA, tmB, a, true, num_sms, static_cast<cudaStream_t>(stream), false));
+  CUtensorMap tmY;
+  std::memset(&tmY, 0, sizeof(tmY));
+  a.y_tma = false;
+  return cuda_status(launch_gemm_i8(tmA, tmB, tmY, a, true, num_sms, static_cast<cudaStream_t>(stream), false));
 }
 
 llmint8_status llmint8_check_status(void* ws, void* stream, uint32_t* flags_out) {

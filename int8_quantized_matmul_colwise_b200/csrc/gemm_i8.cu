@@ -53,7 +53,7 @@ constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kAccCols = BN;
 constexpr uint32_t kTmemCols = 2 * kAccCols;
 constexpr int kChunk = 32;     // accumulator columns per tcgen05.ld (raw int32 epilogue)
-constexpr int kSG = 32;        // outlier rows of W staged per pass over a tile (two k16 MMA steps)
+constexpr int kSG = 16;        // outlier rows of W staged per pass over a tile (one k16 MMA step)
 constexpr int kWoStride = BN + 8;  // halves per staged row: 528 bytes, conflict-free ldmatrix
 
 template <bool kPair>
@@ -67,7 +67,10 @@ struct Geo {
   static constexpr uint32_t kOffB = kOffA + kStages * kBytesA;
   static constexpr uint32_t kOffWo = kOffB + kStages * kBytesB;     // fp16 [kSG][kWoStride]
   static constexpr uint32_t kOffCs = kOffWo + kSG * kWoStride * 2;  // fp32 [BN]
-  static constexpr uint32_t kOffBars = kOffCs + BN * 4;
+  // per epilogue warp, 16 rows x 64 fp16 columns of Y in the 128-byte swizzle
+  static constexpr uint32_t kOffY = (kOffCs + BN * 4 + 1023) & ~1023u;
+  static constexpr uint32_t kYBytes = 16 * 128;
+  static constexpr uint32_t kOffBars = kOffY + kEpiWarps * kYBytes;
   static constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;  // full, empty, tmem full/empty, drain
   static constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
   static constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
@@ -82,6 +85,7 @@ struct Shared {
   uint8_t* b;
   __half* wo;  // outlier rows of W over the tile's columns
   float* cs;  // column scales of the tile
+  uint8_t* ystage;  // Y staging tiles for the TMA store, one per epilogue warp
   uint64_t* full;
   uint64_t* empty;
   uint64_t* tfull;
@@ -100,6 +104,7 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
   s.b = base + G::kOffB;
   s.wo = reinterpret_cast<__half*>(base + G::kOffWo);
   s.cs = reinterpret_cast<float*>(base + G::kOffCs);
+  s.ystage = base + G::kOffY;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + G::kOffBars);
   s.full = bars;
   s.empty = bars + G::kStages;
@@ -330,8 +335,8 @@ __device__ __forceinline__ void load_xo_fragment(const GemmArgs& p, int r0, int 
 }
 
 template <bool kRaw, bool kPair>
-__device__ void run_epilogue(const GemmArgs& p, const Shared& s, uint32_t tmem_base, const Sched& sc,
-                             uint32_t rank, uint32_t warp, uint32_t lane) {
+__device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Shared& s, uint32_t tmem_base,
+                             const Sched& sc, uint32_t rank, uint32_t warp, uint32_t lane) {
   using G = Geo<kPair>;
   const uint32_t q = warp & 3u;             // TMEM lane quarter this warp may access
   const int ab = static_cast<int>(warp - 2) >> 2;  // which 16 rows of the quarter
@@ -351,6 +356,9 @@ __device__ void run_epilogue(const GemmArgs& p, const Shared& s, uint32_t tmem_b
   // ldmatrix row address of this lane inside a 16 x 16 block of staged W rows
   const uint32_t wo_lane = smem_u32(s.wo) + 2u * static_cast<uint32_t>(((lane & 7) + 8 * ((lane >> 3) & 1)) *
                                                                           kWoStride + 8 * (lane >> 4));
+  // this warp's Y staging tile (1024-byte aligned: the 128-byte swizzle repeats every 8 rows)
+  const uint32_t ystage_off = static_cast<uint32_t>(warp - 2) * G::kYBytes;
+  const uint32_t ystage = smem_u32(s.ystage) + ystage_off;
 
   uint32_t it = 0;
   for (int tile = sc.first; tile < sc.num_tiles; tile += sc.stride, ++it) {
@@ -364,7 +372,7 @@ __device__ void run_epilogue(const GemmArgs& p, const Shared& s, uint32_t tmem_b
 
     // Everything but the accumulator is fetched before waiting for it.
     float rsc[2] = {0.0f, 0.0f};  // rows g, g + 8
-    uint32_t afr[2][4];           // Xo fragments of the first pass (two k16 steps)
+    uint32_t afr[4];              // Xo fragment of the first pass
     if constexpr (!kRaw) {
       named_bar_sync(1, kEpiThreads);  // the previous tile's readers of the staged data are done
       stage_scales(p, s, nb, et, cs_vec);
@@ -374,9 +382,7 @@ __device__ void run_epilogue(const GemmArgs& p, const Shared& s, uint32_t tmem_b
         const int r = r0 + g + 8 * h;
         if (r < p.M) rsc[h] = __ldg(p.rs + r) * (1.0f / 16129.0f);
       }
-#pragma unroll
-      for (int ks = 0; ks < 2; ++ks)
-        if (16 * ks < min(n_use, kSG)) load_xo_fragment(p, r0, 16 * ks, min(n_use, kSG), lane, afr[ks]);
+      if (n_use > 0) load_xo_fragment(p, r0, 0, min(n_use, kSG), lane, afr);
     }
 
     const bool got = wait_or_abort(&s.tfull[b], use, p.status, s.abort);
@@ -410,14 +416,11 @@ __device__ void run_epilogue(const GemmArgs& p, const Shared& s, uint32_t tmem_b
       for (int ps = 0; ps < passes; ++ps) {
         const int t0 = ps * kSG;
         const int tn = min(kSG, n_use - t0);
-        const int ksteps = tn > 0 ? (tn + 15) / 16 : 0;
         const bool last = ps == passes - 1;
         if (ps > 0) {
           named_bar_sync(1, kEpiThreads);  // the previous pass's rows are no longer read
           stage_outlier_rows(p, s, nb, t0, tn, et, w_vec);
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks)
-            if (ks < ksteps) load_xo_fragment(p, r0, t0 + 16 * ks, t0 + tn, lane, afr[ks]);
+          load_xo_fragment(p, r0, t0, t0 + tn, lane, afr);
           named_bar_sync(1, kEpiThreads);
         }
         {
@@ -445,20 +448,42 @@ __device__ void run_epilogue(const GemmArgs& p, const Shared& s, uint32_t tmem_b
                 for (int e = 0; e < 4; ++e) d[n][e] = __uint_as_float(v[4 * n + e]);
             }
             // 16-bit outlier product on the tensor cores: d += Xo[rows, k] * W[O[k], cols]
+            if (tn > 0) {
 #pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-              if (ks < ksteps) {
-#pragma unroll
-                for (int np = 0; np < 4; ++np) {
-                  uint32_t b0, b1, b2, b3;
-                  ldmatrix_x4_trans(wo_lane + 2u * static_cast<uint32_t>(16 * ks * kWoStride + c * 64 + 16 * np),
-                                    b0, b1, b2, b3);
-                  mma_m16n8k16_f16f32(d[2 * np], afr[ks], b0, b1);
-                  mma_m16n8k16_f16f32(d[2 * np + 1], afr[ks], b2, b3);
-                }
+              for (int np = 0; np < 4; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4_trans(wo_lane + 2u * static_cast<uint32_t>(c * 64 + 16 * np), b0, b1, b2, b3);
+                mma_m16n8k16_f16f32(d[2 * np], afr, b0, b1);
+                mma_m16n8k16_f16f32(d[2 * np + 1], afr, b2, b3);
               }
             }
-            if (last) {
+            if (last && p.y_tma) {
+              // fp16 fragment -> swizzled staging tile (stmatrix) -> TMA store
+              uint32_t lo[8], hi[8];
+#pragma unroll
+              for (int n = 0; n < 8; ++n) {
+                float y0 = d[n][0], y1 = d[n][1], y2 = d[n][2], y3 = d[n][3];
+                if (overflow) y0 = y1 = y2 = y3 = __int_as_float(0x7fc00000);
+                const __half2 a = __floats2half2_rn(y0, y1), bb = __floats2half2_rn(y2, y3);
+                lo[n] = *reinterpret_cast<const uint32_t*>(&a);
+                hi[n] = *reinterpret_cast<const uint32_t*>(&bb);
+              }
+              if (lane == 0) bulk_wait_read_all();  // the previous store has left the staging tile
+              __syncwarp();
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t rr = (lane & 7) + 8 * ((lane >> 3) & 1);
+                const uint32_t nn = 2 * i + (lane >> 4);
+                stmatrix_x4(ystage + rr * 128u + ((nn ^ (rr & 7)) << 4), lo[2 * i], hi[2 * i], lo[2 * i + 1],
+                            hi[2 * i + 1]);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmY, s.ystage + ystage_off, nb * BN + c * 64, r0);
+                bulk_commit();
+              }
+            } else if (last) {
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
                 const int r = r0 + g + 8 * h;
@@ -501,12 +526,14 @@ __device__ void run_epilogue(const GemmArgs& p, const Shared& s, uint32_t tmem_b
         mbar_arrive(&s.tempty[b]);
     }
   }
+  if (lane == 0) bulk_wait_all();  // Y stores complete before the CTA exits
+  __syncwarp();
 }
 
 template <bool kRaw, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmArgs p) {
+                   const __grid_constant__ CUtensorMap tmY, const GemmArgs p) {
   using G = Geo<kPair>;
   extern __shared__ uint8_t smem_raw[];
   const Shared s = carve<kPair>(smem_raw);
@@ -534,6 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (p.y_tma) tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     if constexpr (kPair) {
@@ -557,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) run_mma<kPair>(s, tmem_base, sc, p.status);
   } else {
-    run_epilogue<kRaw, kPair>(p, s, tmem_base, sc, rank, warp, lane);
+    run_epilogue<kRaw, kPair>(p, tmY, s, tmem_base, sc, rank, warp, lane);
   }
 
   tc_fence_before();
@@ -574,8 +602,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <bool kRaw, bool kPair>
-cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
-                           cudaStream_t stream, bool pdl) {
+cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY,
+                           const GemmArgs& a, int num_sms, cudaStream_t stream, bool pdl) {
   using G = Geo<kPair>;
   static bool attr_set[64] = {};  // per device
   static int max_units[64] = {};  // CTAs (or CTA pairs) that fit at once, per device
@@ -637,22 +665,22 @@ cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const
   cfg.stream = stream;
   cfg.attrs = n_attr ? attr : nullptr;
   cfg.numAttrs = n_attr;
-  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmY, a);
 }
 
 }  // namespace
 
 bool gemm_uses_pair(int M) { return M > BM; }
 
-cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, bool raw_i32,
-                           int num_sms, cudaStream_t stream, bool pdl) {
+cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY,
+                           const GemmArgs& a, bool raw_i32, int num_sms, cudaStream_t stream, bool pdl) {
   const bool pair = gemm_uses_pair(a.M);
   if (raw_i32) {
-    return pair ? launch_variant<true, true>(tmA, tmB, a, num_sms, stream, pdl)
-                : launch_variant<true, false>(tmA, tmB, a, num_sms, stream, pdl);
+    return pair ? launch_variant<true, true>(tmA, tmB, tmY, a, num_sms, stream, pdl)
+                : launch_variant<true, false>(tmA, tmB, tmY, a, num_sms, stream, pdl);
   }
-  return pair ? launch_variant<false, true>(tmA, tmB, a, num_sms, stream, pdl)
-              : launch_variant<false, false>(tmA, tmB, a, num_sms, stream, pdl);
+  return pair ? launch_variant<false, true>(tmA, tmB, tmY, a, num_sms, stream, pdl)
+              : launch_variant<false, false>(tmA, tmB, tmY, a, num_sms, stream, pdl);
 }
 
 }  // namespace llmint8

@@ -10,10 +10,10 @@ namespace llmint8 {
 
 // Scratch the activation kernels keep in the caller's workspace.
 struct ActWs {
-  uint32_t* colmax;   // [K] fp16 bit patterns of the column maxima; zero between calls
-  uint32_t* counter;  // CTA completion counter of the scan kernel; zero between calls
-  uint32_t* bitmask;  // [ceil(K/32)] outlier flags of this call
-  uint32_t* status;   // status word
+  uint32_t* colmax;       // [K] fp16 bit patterns of the column maxima; zero between calls
+  uint32_t* blk_counter;  // [ceil(K/256)] scan CTAs finished per column block; zero between calls
+  uint32_t* bitmask;      // [ceil(K/32)] outlier flags of this call
+  uint32_t* status;       // status word
 };
 
 cudaError_t launch_quantize_weight_colwise(const void* W, int64_t K, int64_t N, int64_t ldw, int8_t* Wq,
@@ -40,6 +40,7 @@ struct GemmArgs {
   int32_t* C;         // int32 [M, ldc] (raw accumulator output mode)
   int64_t ldc;
   uint32_t* status;
+  bool y_tma;         // Y is written through the tmY tensor map (16-byte aligned rows)
 };
 
 // Whether the GEMM for M rows runs as CTA pairs (256 x 256 tiles, cta_group::2)
@@ -49,8 +50,10 @@ bool gemm_uses_pair(int M);
 // tmA: Xq [M rows, K cols] int8 in boxes of 128 rows, tmB: Wq [N rows, K cols]
 // int8 in boxes of gemm_b_box_rows(M) rows, 128 bytes along K, 128-byte
 // swizzle.  raw_i32 selects the accumulator-dump epilogue.
-cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, bool raw_i32,
-                           int num_sms, cudaStream_t stream, bool pdl);
+// tmY: Y [M rows, N cols] fp16 in boxes of 16 rows x 64 columns, 128-byte
+// swizzle (used when a.y_tma).
+cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY,
+                           const GemmArgs& a, bool raw_i32, int num_sms, cudaStream_t stream, bool pdl);
 
 // Tile sizes of the GEMM per CTA (accumulator rows / columns, K bytes per stage).
 constexpr int kGemmBM = 128;

@@ -31,18 +31,6 @@ __device__ __forceinline__ int quantize_exact(float x, float s, float inv_s) {
   return x < 0.0f ? -qi : qi;
 }
 
-// The same code with a cheap common path.  k = fl(127 / s); r = x * k is
-// within 2^-22 relative (|r| <= 127 + 2^-15) of the exact 127 x / s, so when r
-// is farther than 2^-10 from a half-integer, rint(r) is the nearest integer of
-// the exact value and there is no tie: the code is rint(r).  Otherwise (about
-// one value in 500) the exact comparisons of quantize_exact decide.
-__device__ __forceinline__ int quantize_fast(float x, float s, float inv_s, float k) {
-  const float r = __fmul_rn(x, k);
-  const float q = rintf(r);
-  if (fabsf(__fadd_rn(r, -q)) < 0.4990234375f) return __float2int_rz(q);  // 0.5 - 2^-10
-  return quantize_exact(x, s, inv_s);
-}
-
 // Pack four codes (low byte first) into a 32-bit word.
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
   return (uint32_t(a) & 0xFFu) | ((uint32_t(b) & 0xFFu) << 8) | ((uint32_t(c) & 0xFFu) << 16) |

@@ -9,16 +9,17 @@
 // Transformers at Scale" (the outlier feature dimensions are isolated).
 //
 // The outlier set depends on every row, so the work is two kernels:
-//  scan:     column maxima of |X| (atomicMax on fp16 bit patterns, which order
-//            like the values for non-negative halves); the last CTA to finish
-//            turns them into a column bitmask (one warp ballot per 32 columns)
-//            and the ascending outlier list, and returns the maxima to zero
-//            for the next call;
-//  quantize: per row, absmax over non-outlier columns, exact codes, gather.
-//            A row is held in registers by a group of G threads (CPT 16-byte
-//            chunks each), so X is read once and all loads are in flight
-//            together.
-// Both are HBM-bound streaming kernels.
+//  scan:     column maxima of |X| over 64 x 256 tiles, merged with atomicMax
+//            on fp16 bit patterns (non-negative halves order like their bits)
+//            into a workspace array that is zero between calls; the last CTA
+//            of each 256-column block writes that block's outlier bitmask
+//            words (one ballot per 32 columns) and re-zeroes its maxima;
+//  quantize: every CTA issues the loads of its rows, then reads the bitmask
+//            and builds its popcount prefix in shared memory while they are in
+//            flight; CTA 0 writes the ascending outlier list; each row is then
+//            quantized from registers and its outlier values gathered.
+// Both are HBM streaming kernels: one 16-byte load per 8 columns, all of a
+// thread's loads in flight together, no divergent work on the common path.
 #include <cuda_fp16.h>
 
 #include "kernels.cuh"
@@ -32,22 +33,8 @@ namespace {
 constexpr int kScanCols = 256;  // columns per scan CTA (32 lanes x 8)
 constexpr int kScanRows = 64;   // rows per scan CTA (8 warps x 8 rows)
 
-__device__ __forceinline__ void load8_bits(const __half* __restrict__ row, int64_t K, int64_t c, bool vec_ok,
-                                           __half (&h)[8]) {
-  if (vec_ok && c + 8 <= K) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + c));
-    const __half* p = reinterpret_cast<const __half*>(&u);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) h[e] = p[e];
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) h[e] = (c + e < K) ? row[c + e] : __ushort_as_half(0);
-  }
-}
-
-// 8 consecutive fp16 of a row as one 16-byte register quad (zero past K).
-__device__ __forceinline__ uint4 load8_packed(const __half* __restrict__ row, int64_t K, int64_t c, bool vec_ok) {
-  if (vec_ok && c + 8 <= K) return __ldg(reinterpret_cast<const uint4*>(row + c));
+// 8 consecutive fp16 of a row by scalar loads (unaligned rows or a ragged end).
+__device__ __forceinline__ uint4 load8_scalar(const __half* __restrict__ row, int64_t K, int64_t c) {
   uint32_t w[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
@@ -58,9 +45,71 @@ __device__ __forceinline__ uint4 load8_packed(const __half* __restrict__ row, in
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// 8 consecutive fp16 of a row as one 16-byte register quad (zero past K).
+// kVec: rows are 16-byte aligned and K % 8 == 0, so every chunk that starts
+// before K is one aligned 16-byte load (decided on the host).
+template <bool kVec>
+__device__ __forceinline__ uint4 load8_packed(const __half* __restrict__ row, int64_t K, int64_t c) {
+  if constexpr (kVec) return __ldg(reinterpret_cast<const uint4*>(row + c));
+  else return load8_scalar(row, K, c);
+}
+
 __device__ __forceinline__ unsigned short half_bits_at(const uint4& u, int e) {
   const uint32_t w = (e < 2) ? u.x : (e < 4) ? u.y : (e < 6) ? u.z : u.w;
   return static_cast<unsigned short>((e & 1) ? (w >> 16) : (w & 0xFFFFu));
+}
+
+__device__ __forceinline__ uint2 pack8(const int (&q)[8]) {
+  uint2 out;
+  out.x = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+  out.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
+  return out;
+}
+
+// Codes of 8 values (fp16 pairs in u) by the exact comparisons.
+__device__ __forceinline__ uint2 quantize8_exact(uint4 u, float s, float inv) {
+  const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+  int q[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(h2[e]);
+    q[2 * e] = quantize_exact(f.x, s, inv);
+    q[2 * e + 1] = quantize_exact(f.y, s, inv);
+  }
+  return pack8(q);
+}
+
+// Codes of 8 values by rounding x * (127 / s).  With k = fl(127/s) and
+// r = fl(x k), |r - 127x/s| <= 127 (2^-24 + 2^-24)(1 + 2^-24) < 2^-16, so when
+// |r - rint(r)| < 1/2 - 2^-15 the exact value is strictly nearer to rint(r)
+// than to any other integer and rint(r) is its rounding (no tie possible).
+// Otherwise (about one value in 16000, or NaN) tie_risk is set and the caller
+// redoes the chunk with quantize8_exact.
+// rint is taken as t = r + 1.5 * 2^23: for |r| < 2^22 the sum lies in
+// [2^23, 2^24) where the spacing is 1, so it is rounded to the nearest integer
+// (ties to even), t - 1.5 * 2^23 is exact, and the low byte of t's bit pattern
+// is the integer's low byte (two's complement) -- all on the FMA pipe.
+__device__ __forceinline__ uint2 quantize8(uint4 u, float k, bool& tie_risk) {
+  constexpr float kSafe = 0.499969482421875f;  // 1/2 - 2^-15
+  constexpr float kBias = 12582912.0f;         // 1.5 * 2^23
+  const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+  uint32_t t[8];
+  const float2 k2 = make_float2(k, k);
+  const float2 b2 = make_float2(kBias, kBias);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 r = __fmul2_rn(__half22float2(h2[e]), k2);
+    const float2 tb = __fadd2_rn(r, b2);
+    const float2 q = __fadd2_rn(tb, make_float2(-kBias, -kBias));
+    const float2 d = __fadd2_rn(r, make_float2(-q.x, -q.y));
+    tie_risk |= !(fabsf(d.x) < kSafe) | !(fabsf(d.y) < kSafe);  // true for NaN as well
+    t[2 * e] = __float_as_uint(tb.x);
+    t[2 * e + 1] = __float_as_uint(tb.y);
+  }
+  uint2 out;
+  out.x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+  out.y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+  return out;
 }
 
 // Block-wide exclusive prefix sum of one int per thread (256 threads).
@@ -86,14 +135,15 @@ __device__ __forceinline__ int block_exclusive_scan_256(int v, int* s_warp, int&
   return base + inc - v;
 }
 
-// Dynamic shared memory of the last CTA: one bitmask word per 32 columns.
+// ----------------------------------------------------------------- a1: scan
+// Column maxima of |X| over this CTA's 64 rows x 256 columns, merged into the
+// workspace with atomicMax.  The last CTA of a column block (per-block
+// counter) turns the block's 256 maxima into 8 outlier bitmask words and
+// returns the maxima and the counter to zero for the next call.
+template <bool kVec>
 __global__ void __launch_bounds__(256, 4) scan_columns_kernel(const __half* __restrict__ X, int64_t M, int64_t K,
-                                                           int64_t ldx, bool vec_ok, float tau, ActWs ws,
-                                                           int32_t* __restrict__ O, int64_t cap,
-                                                           int32_t* __restrict__ n_out) {
-  extern __shared__ uint32_t s_bits[];
+                                                              int64_t ldx, float tau, ActWs ws) {
   __shared__ uint32_t s_max[8][kScanCols];
-  __shared__ int s_warp[8];
   __shared__ int s_last;
 
   griddep_wait();               // X may come from the previous kernel on the stream
@@ -103,7 +153,7 @@ __global__ void __launch_bounds__(256, 4) scan_columns_kernel(const __half* __re
   const int64_t c = int64_t(blockIdx.x) * kScanCols + 8 * lane;
   const int64_t r0 = int64_t(blockIdx.y) * kScanRows + warp;
   // |x| maxima of 8 columns as 4 half2; __hmax2 returns the non-NaN operand,
-  // so a NaN never wins (it is mapped to 0 below if nothing else was seen).
+  // so a NaN never wins (and is mapped to 0 below if nothing else was seen).
   __half2 m2[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) m2[e] = __half2half2(__ushort_as_half(0));
@@ -112,7 +162,7 @@ __global__ void __launch_bounds__(256, 4) scan_columns_kernel(const __half* __re
 #pragma unroll
     for (int j = 0; j < kScanRows / 8; ++j) {
       const int64_t r = r0 + 8 * j;
-      u[j] = r < M ? load8_packed(X + r * ldx, K, c, vec_ok) : make_uint4(0u, 0u, 0u, 0u);
+      u[j] = r < M ? load8_packed<kVec>(X + r * ldx, K, c) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int j = 0; j < kScanRows / 8; ++j) {
@@ -131,114 +181,85 @@ __global__ void __launch_bounds__(256, 4) scan_columns_kernel(const __half* __re
     s_max[warp][8 * lane + 2 * e + 1] = hi;
   }
   __syncthreads();
-  {
-    uint32_t v = 0;
+  uint32_t v = 0;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v = max(v, s_max[w][threadIdx.x]);
-    const int64_t col = int64_t(blockIdx.x) * kScanCols + threadIdx.x;
-    if (v != 0 && col < K) atomicMax(ws.colmax + col, v);
-  }
+  for (int w = 0; w < 8; ++w) v = max(v, s_max[w][threadIdx.x]);
+  const int64_t col = int64_t(blockIdx.x) * kScanCols + threadIdx.x;
+  if (v != 0 && col < K) atomicMax(ws.colmax + col, v);
 
-  // Last CTA: column flags -> bitmask words and the ascending outlier list.
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned total = gridDim.x * gridDim.y;
-    s_last = (atomicAdd(ws.counter, 1u) == total - 1u) ? 1 : 0;
-  }
+  if (threadIdx.x == 0) s_last = (atomicAdd(ws.blk_counter + blockIdx.x, 1u) == gridDim.y - 1u) ? 1 : 0;
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  const uint32_t mx = col < K ? __ldcg(ws.colmax + col) : 0u;
+  const bool flag = col < K && __half2float(__ushort_as_half(static_cast<unsigned short>(mx))) >= tau;
+  const uint32_t bits = __ballot_sync(0xffffffffu, flag);
+  const int64_t w = int64_t(blockIdx.x) * (kScanCols / 32) + warp;
+  if (lane == 0 && w * 32 < K) ws.bitmask[w] = bits;
+  if (col < K) ws.colmax[col] = 0u;
+  if (threadIdx.x == 0) ws.blk_counter[blockIdx.x] = 0u;
+}
 
+// ----------------------------------------------------------------- a1 -> O
+// The outlier bitmask of this call and its popcount prefix into shared memory
+// (s_mask[w]: columns 32w..32w+31; s_pre[w]: outliers before word w).  CTA 0
+// also writes the ascending outlier list, n_o and the overflow bit.
+__device__ __forceinline__ void build_outlier_set(int64_t K, const ActWs& ws, uint32_t* s_mask, uint32_t* s_pre,
+                                                  int* s_warp, int32_t* __restrict__ O, int64_t cap,
+                                                  int32_t* __restrict__ n_out) {
   const int64_t nwords = (K + 31) / 32;
-  // One coalesced read and one ballot per 32 columns (column = 256 i + 32 warp
-  // + lane, word = 8 i + warp); the loads of 8 rounds are issued together.
-  // The maxima are reset to zero for the next call.
-  constexpr int kBatch = 8;
-  for (int64_t i0 = 0; i0 * 256 < K; i0 += kBatch) {
-    uint32_t v[kBatch];
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const int64_t col = (i0 + i) * 256 + threadIdx.x;
-      v[i] = col < K ? __ldcg(ws.colmax + col) : 0u;
-    }
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const int64_t col = (i0 + i) * 256 + threadIdx.x;
-      const bool flag = col < K && __half2float(__ushort_as_half(static_cast<unsigned short>(v[i]))) >= tau;
-      const uint32_t bits = __ballot_sync(0xffffffffu, flag);
-      const int64_t w = (i0 + i) * 8 + warp;
-      if (lane == 0 && w < nwords) {
-        s_bits[w] = bits;
-        ws.bitmask[w] = bits;
-      }
-      if (col < K) ws.colmax[col] = 0u;
-    }
-  }
-  __syncthreads();
   const int64_t wpt = (nwords + 255) / 256;  // contiguous words per thread, in column order
   const int64_t w0 = int64_t(threadIdx.x) * wpt;
   int cnt = 0;
-  for (int64_t w = w0; w < w0 + wpt && w < nwords; ++w) cnt += __popc(s_bits[w]);
-  int total = 0;
-  int pos = block_exclusive_scan_256(cnt, s_warp, total);
   for (int64_t w = w0; w < w0 + wpt && w < nwords; ++w) {
-    uint32_t bits = s_bits[w];
-    while (bits) {
-      const int b = __ffs(bits) - 1;
-      bits &= bits - 1;
-      if (pos < cap) O[pos] = static_cast<int32_t>(w * 32 + b);
-      ++pos;
-    }
+    const uint32_t b = __ldcg(ws.bitmask + w);
+    s_mask[w] = b;
+    cnt += __popc(b);
   }
-  if (threadIdx.x == 0) {
+  int total = 0;
+  int pre = block_exclusive_scan_256(cnt, s_warp, total);
+  for (int64_t w = w0; w < w0 + wpt && w < nwords; ++w) {
+    s_pre[w] = static_cast<uint32_t>(pre);
+    if (blockIdx.x == 0) {
+      uint32_t bits = s_mask[w];
+      int pos = pre;
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (pos < cap) O[pos] = static_cast<int32_t>(w * 32 + b);
+        ++pos;
+      }
+    }
+    pre += __popc(s_mask[w]);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
     *n_out = total;
-    *ws.counter = 0u;
     if (total > cap) atomicOr(ws.status, kStatusOverflow);
   }
+  __syncthreads();
 }
 
+// ----------------------------------------------------------------- a2-a4
 // Row quantizer: a group of G threads owns one row and holds its CPT chunks
 // of 8 columns in registers (G * CPT * 8 >= K).  256 threads per CTA, 256 / G
-// rows per CTA.
-template <int G, int CPT>
-__global__ void __launch_bounds__(256, 3) quantize_rows_kernel(const __half* __restrict__ X, int64_t M, int64_t K,
-                                                            int64_t ldx, bool vec_ok, ActWs ws,
-                                                            const int32_t* __restrict__ O,
-                                                            const int32_t* __restrict__ n_ptr, int64_t cap,
-                                                            int8_t* __restrict__ Xq, int64_t ldq,
-                                                            float* __restrict__ rs, __half* __restrict__ Xo,
-                                                            int64_t ldo) {
-  extern __shared__ uint32_t s_mask[];  // [nwords] outlier bitmask, then [nwords] exclusive popcount prefix
+// rows per CTA.  Dynamic shared memory: bitmask and prefix, K/32 words each.
+template <int G, int CPT, bool kVec>
+__global__ void __launch_bounds__(256, 4) quantize_rows_kernel(const __half* __restrict__ X, int64_t M, int64_t K,
+                                                               int64_t ldx, float tau, ActWs ws,
+                                                               int32_t* __restrict__ O, int32_t* __restrict__ n_out,
+                                                               int64_t cap, int8_t* __restrict__ Xq, int64_t ldq,
+                                                               float* __restrict__ rs, __half* __restrict__ Xo,
+                                                               int64_t ldo) {
+  extern __shared__ uint32_t s_mask[];
   constexpr int kWarpsPerRow = G / 32;
   constexpr int kRowsPerCta = 256 / G;
   __shared__ float s_part[8];
   __shared__ int s_warp[8];
 
-  griddep_wait();  // the bitmask comes from the scan kernel
+  griddep_wait();  // the column maxima come from the scan kernel
   griddep_launch_dependents();
-
-  const int64_t nwords = (K + 31) / 32;
-  uint32_t* s_pre = s_mask + nwords;
-  {
-    // bitmask into shared memory and, per word, the number of outlier columns
-    // before it: the position in O of a column's outlier value
-    const int64_t wpt = (nwords + 255) / 256;
-    const int64_t w0 = int64_t(threadIdx.x) * wpt;
-    int cnt = 0;
-    for (int64_t w = w0; w < w0 + wpt && w < nwords; ++w) {
-      const uint32_t b = __ldg(ws.bitmask + w);
-      s_mask[w] = b;
-      cnt += __popc(b);
-    }
-    int total = 0;
-    int pre = block_exclusive_scan_256(cnt, s_warp, total);
-    for (int64_t w = w0; w < w0 + wpt && w < nwords; ++w) {
-      s_pre[w] = static_cast<uint32_t>(pre);
-      pre += __popc(s_mask[w]);
-    }
-  }
-  __syncthreads();
 
   const int warp = threadIdx.x >> 5;
   const int gt = threadIdx.x % G;
@@ -246,91 +267,30 @@ __global__ void __launch_bounds__(256, 3) quantize_rows_kernel(const __half* __r
   const bool row_ok = row < M;
   const __half* xr = X + row * ldx;
 
+  // the row loads go out first and overlap the outlier-set construction
   uint4 h[CPT];
 #pragma unroll
   for (int j = 0; j < CPT; ++j) {
     const int64_t c = 8 * (int64_t(gt) + int64_t(j) * G);
-    h[j] = (row_ok && c < K) ? load8_packed(xr, K, c, vec_ok) : make_uint4(0u, 0u, 0u, 0u);
+    h[j] = (row_ok && c < K) ? load8_packed<kVec>(xr, K, c) : make_uint4(0u, 0u, 0u, 0u);
   }
-  // outlier flags of a chunk's 8 columns (chunks past K read as no outliers:
-  // their data is zero)
+  const int64_t nwords = (K + 31) / 32;
+  uint32_t* s_pre = s_mask + nwords;
+  build_outlier_set(K, ws, s_mask, s_pre, s_warp, O, cap, n_out);
+
+  // outlier flags of chunk j's 8 columns (chunks past K: none, data is zero)
   auto flags = [&](int j) -> uint32_t {
     const int64_t c = 8 * (int64_t(gt) + int64_t(j) * G);
     return c < K ? (s_mask[c >> 5] >> (c & 31)) & 0xFFu : 0u;
   };
-  // a2: absmax over the non-outlier columns; packed half2 max on chunks
-  // without outliers, element-wise on the rare chunks that have some
-  __half2 m2 = __half2half2(__ushort_as_half(0));
+  uint32_t any_outlier = 0;
 #pragma unroll
-  for (int j = 0; j < CPT; ++j) {
-    const uint32_t om = flags(j);
-    const __half2* h2 = reinterpret_cast<const __half2*>(&h[j]);
-    if (om == 0u) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(h2[e]));
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (!((om >> e) & 1u)) {
-          const __half a = __habs(__ushort_as_half(half_bits_at(h[j], e)));
-          m2 = __hmax2(m2, __halves2half2(a, a));
-        }
-      }
-    }
-  }
-  float m = fmaxf(__low2float(m2), __high2float(m2));
-  m = (m == m) ? m : 0.0f;  // all-NaN row segment
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if constexpr (kWarpsPerRow > 1) {
-    if ((threadIdx.x & 31) == 0) s_part[warp] = m;
-    __syncthreads();
-    const int wg0 = (warp / kWarpsPerRow) * kWarpsPerRow;
-#pragma unroll
-    for (int w = 0; w < kWarpsPerRow; ++w) m = fmaxf(m, s_part[wg0 + w]);
-  }
-  if (!row_ok) return;
-  const float s = m;
-  const float inv = s > 0.0f ? __frcp_rn(s) : 0.0f;
-  const float k = s > 0.0f ? __fdiv_rn(127.0f, s) : 0.0f;
-  if (gt == 0) rs[row] = s;
-
-  // a3: codes; outlier columns are zeroed first (0 quantizes to 0); columns
-  // [K, ldq) are written as zero
-  int8_t* qr = Xq + row * ldq;
-#pragma unroll
-  for (int j = 0; j < CPT; ++j) {
-    const int64_t c = 8 * (int64_t(gt) + int64_t(j) * G);
-    if (c < ldq) {
-      const uint32_t om = flags(j);
-      uint4 u = h[j];
-      if (om != 0u) {
-        uint32_t* w = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          w[e] &= (((om >> (2 * e)) & 1u) ? 0u : 0xFFFFu) | (((om >> (2 * e + 1)) & 1u) ? 0u : 0xFFFF0000u);
-      }
-      const __half2* h2 = reinterpret_cast<const __half2*>(&u);
-      int q[8];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(h2[e]);
-        q[2 * e] = quantize_fast(f.x, s, inv, k);
-        q[2 * e + 1] = quantize_fast(f.y, s, inv, k);
-      }
-      uint2 out;
-      out.x = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
-      out.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
-      *reinterpret_cast<uint2*>(qr + c) = out;
-    }
-  }
-  // ldq may exceed G * CPT * 8 only by the zero padding beyond K
-  for (int64_t c = 8 * (int64_t(gt) + int64_t(CPT) * G); c < ldq; c += 8 * G)
-    *reinterpret_cast<uint2*>(qr + c) = make_uint2(0u, 0u);
+  for (int j = 0; j < CPT; ++j) any_outlier |= flags(j);
 
   // a4: gather X[row, O[t]] for the outlier product, from the registers: the
   // outlier column c sits at position prefix(word) + popcount(lower bits).
-  if (Xo != nullptr) {
+  // Outlier columns are then zeroed in the registers (0 quantizes to 0).
+  if (any_outlier != 0u) {
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
       const uint32_t om = flags(j);
@@ -343,40 +303,94 @@ __global__ void __launch_bounds__(256, 3) quantize_rows_kernel(const __half* __r
           if ((om >> e) & 1u) {
             const int b = static_cast<int>((c & 31) + e);
             const int64_t pos = base + __popc(word & ((1u << b) - 1u));
-            if (pos < cap) Xo[row * ldo + pos] = __ushort_as_half(half_bits_at(h[j], e));
+            if (Xo != nullptr && row_ok && pos < cap) Xo[row * ldo + pos] = __ushort_as_half(half_bits_at(h[j], e));
           }
         }
+        uint32_t* w = reinterpret_cast<uint32_t*>(&h[j]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          w[e] &= (((om >> (2 * e)) & 1u) ? 0u : 0xFFFFu) | (((om >> (2 * e + 1)) & 1u) ? 0u : 0xFFFF0000u);
       }
     }
   }
+
+  // a2: absmax over the non-outlier columns (outliers and padding are zero now)
+  __half2 m2 = __half2half2(__ushort_as_half(0));
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) {
+    const __half2* h2 = reinterpret_cast<const __half2*>(&h[j]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(h2[e]));
+  }
+  float m = fmaxf(__low2float(m2), __high2float(m2));
+  m = (m == m) ? m : 0.0f;  // all-NaN row segment
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if constexpr (kWarpsPerRow > 1) {
+    if ((threadIdx.x & 31) == 0) s_part[warp] = m;
+    __syncthreads();
+    const int wg0 = (warp / kWarpsPerRow) * kWarpsPerRow;
+#pragma unroll
+    for (int w = 0; w < kWarpsPerRow; ++w) m = fmaxf(m, s_part[wg0 + w]);
+  }
+  const float s = m;
+  const float inv = s > 0.0f ? __frcp_rn(s) : 0.0f;
+  const float k = s > 0.0f ? __fdiv_rn(127.0f, s) : 0.0f;
+
+  if (row_ok) {
+    if (gt == 0) rs[row] = s;
+    // a3: codes; columns [K, ldq) are written as zero
+    int8_t* qr = Xq + row * ldq;
+    uint32_t risk = 0;  // chunks that need the exact rounding
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int64_t c = 8 * (int64_t(gt) + int64_t(j) * G);
+      if (c < ldq) {
+        bool tie_risk = false;
+        *reinterpret_cast<uint2*>(qr + c) = quantize8(h[j], k, tie_risk);
+        risk |= static_cast<uint32_t>(tie_risk) << j;
+      }
+    }
+    if (risk != 0u) {  // rare: redo those chunks exactly
+#pragma unroll
+      for (int j = 0; j < CPT; ++j)
+        if ((risk >> j) & 1u)
+          *reinterpret_cast<uint2*>(qr + 8 * (int64_t(gt) + int64_t(j) * G)) = quantize8_exact(h[j], s, inv);
+    }
+    // ldq may exceed G * CPT * 8 only by the zero padding beyond K
+    for (int64_t c = 8 * (int64_t(gt) + int64_t(CPT) * G); c < ldq; c += 8 * G)
+      *reinterpret_cast<uint2*>(qr + c) = make_uint2(0u, 0u);
+  }
 }
 
-// Fallback for very long rows (K > 16384): two passes over the row.
+// Rows too long for the register-resident kernel (K > 16384): one CTA per row,
+// two passes over the row.
 __global__ void __launch_bounds__(256) quantize_rows_long_kernel(const __half* __restrict__ X, int64_t M,
-                                                                 int64_t K, int64_t ldx, bool vec_ok, ActWs ws,
-                                                                 const int32_t* __restrict__ O,
-                                                                 const int32_t* __restrict__ n_ptr, int64_t cap,
+                                                                 int64_t K, int64_t ldx, float tau, ActWs ws,
+                                                                 int32_t* __restrict__ O,
+                                                                 int32_t* __restrict__ n_out, int64_t cap,
                                                                  int8_t* __restrict__ Xq, int64_t ldq,
                                                                  float* __restrict__ rs, __half* __restrict__ Xo,
                                                                  int64_t ldo) {
   extern __shared__ uint32_t s_mask[];
   __shared__ float s_part[8];
+  __shared__ int s_warp[8];
   griddep_wait();
   griddep_launch_dependents();
   const int64_t nwords = (K + 31) / 32;
-  for (int64_t w = threadIdx.x; w < nwords; w += blockDim.x) s_mask[w] = ws.bitmask[w];
-  __syncthreads();
+  uint32_t* s_pre = s_mask + nwords;
+  build_outlier_set(K, ws, s_mask, s_pre, s_warp, O, cap, n_out);
+
   const int64_t row = blockIdx.x;
   const __half* xr = X + row * ldx;
   const int64_t nchunks = (K + 7) / 8;
   float m = 0.0f;
   for (int64_t ch = threadIdx.x; ch < nchunks; ch += 256) {
-    __half h[8];
-    load8_bits(xr, K, 8 * ch, vec_ok, h);
+    const uint4 u = load8_scalar(xr, K, 8 * ch);
     const uint32_t mw = s_mask[(8 * ch) >> 5] >> ((8 * ch) & 31);
 #pragma unroll
     for (int e = 0; e < 8; ++e)
-      if (!((mw >> e) & 1u)) m = fmaxf(m, fabsf(__half2float(h[e])));
+      if (!((mw >> e) & 1u)) m = fmaxf(m, fabsf(__half2float(__ushort_as_half(half_bits_at(u, e)))));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -392,38 +406,45 @@ __global__ void __launch_bounds__(256) quantize_rows_long_kernel(const __half* _
     const int64_t c = 8 * ch;
     int q[8];
     if (c < K) {
-      __half h[8];
-      load8_bits(xr, K, c, vec_ok, h);
+      const uint4 u = load8_scalar(xr, K, c);
       const uint32_t mw = s_mask[c >> 5] >> (c & 31);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const bool keep = (c + e < K) && !((mw >> e) & 1u) && s > 0.0f;
-        q[e] = keep ? quantize_exact(__half2float(h[e]), s, inv) : 0;
+        q[e] = keep ? quantize_exact(__half2float(__ushort_as_half(half_bits_at(u, e))), s, inv) : 0;
       }
     } else {
 #pragma unroll
       for (int e = 0; e < 8; ++e) q[e] = 0;
     }
-    uint2 out;
-    out.x = pack4(q[0], q[1], q[2], q[3]);
-    out.y = pack4(q[4], q[5], q[6], q[7]);
-    *reinterpret_cast<uint2*>(qr + c) = out;
+    *reinterpret_cast<uint2*>(qr + c) = pack8(q);
   }
   if (Xo != nullptr) {
-    const int n_o = *n_ptr;
-    const int64_t n_gather = n_o < cap ? n_o : cap;
-    for (int64_t t = threadIdx.x; t < n_gather; t += 256) Xo[row * ldo + t] = xr[O[t]];
+    // positions come from the local bitmask and prefix (O itself is written by CTA 0)
+    for (int64_t w = threadIdx.x; w < nwords; w += 256) {
+      uint32_t bits = s_mask[w];
+      int64_t pos = s_pre[w];
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (pos < cap) Xo[row * ldo + pos] = xr[w * 32 + b];
+        ++pos;
+      }
+    }
   }
 }
 
 template <int G, int CPT>
 cudaError_t launch_rows(cudaLaunchConfig_t& cfg, int64_t M, const __half* x, int64_t K, int64_t ldx, bool vec_ok,
-                        ActWs ws, const int32_t* O, const int32_t* n, int64_t cap, int8_t* Xq, int64_t ldq,
+                        float tau, ActWs ws, int32_t* O, int32_t* n, int64_t cap, int8_t* Xq, int64_t ldq,
                         float* rs, __half* xo, int64_t ldo) {
   constexpr int rows_per_cta = 256 / G;
   cfg.gridDim = dim3(static_cast<unsigned>((M + rows_per_cta - 1) / rows_per_cta));
-  return cudaLaunchKernelEx(&cfg, quantize_rows_kernel<G, CPT>, x, M, K, ldx, vec_ok, ws, O, n, cap, Xq, ldq, rs,
-                            xo, ldo);
+  if (vec_ok)
+    return cudaLaunchKernelEx(&cfg, quantize_rows_kernel<G, CPT, true>, x, M, K, ldx, tau, ws, O, n, cap, Xq, ldq,
+                              rs, xo, ldo);
+  return cudaLaunchKernelEx(&cfg, quantize_rows_kernel<G, CPT, false>, x, M, K, ldx, tau, ws, O, n, cap, Xq, ldq,
+                            rs, xo, ldo);
 }
 
 }  // namespace
@@ -432,7 +453,7 @@ cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx
                                 int64_t ldq, float* rs, int32_t* O, int64_t cap, int32_t* n_out, void* Xo,
                                 int64_t ldo, ActWs ws, cudaStream_t stream, bool pdl) {
   const __half* x = static_cast<const __half*>(X);
-  const bool vec_ok = (ldx % 8 == 0) && (reinterpret_cast<uintptr_t>(X) % 16 == 0);
+  const bool vec_ok = (ldx % 8 == 0) && (K % 8 == 0) && (reinterpret_cast<uintptr_t>(X) % 16 == 0);
   const size_t mask_bytes = static_cast<size_t>((K + 31) / 32) * sizeof(uint32_t);
 
   cudaLaunchAttribute attr[1];
@@ -447,34 +468,35 @@ cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx
 
   cfg.gridDim = dim3(static_cast<unsigned>((K + kScanCols - 1) / kScanCols),
                      static_cast<unsigned>((M + kScanRows - 1) / kScanRows));
-  cfg.dynamicSmemBytes = mask_bytes;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, scan_columns_kernel, x, M, K, ldx, vec_ok, tau, ws, O, cap, n_out);
+  cfg.dynamicSmemBytes = 0;
+  cudaError_t e = vec_ok ? cudaLaunchKernelEx(&cfg, scan_columns_kernel<true>, x, M, K, ldx, tau, ws)
+                         : cudaLaunchKernelEx(&cfg, scan_columns_kernel<false>, x, M, K, ldx, tau, ws);
   if (e != cudaSuccess) return e;
 
   cfg.dynamicSmemBytes = 2 * mask_bytes;  // bitmask + popcount prefix
   __half* xo = static_cast<__half*>(Xo);
-  const int32_t* Oc = O;
-  const int32_t* nc = n_out;
   // Row groups: G threads x CPT chunks of 8 columns >= K.  Small M spreads a
   // row over more threads (fewer chunks each) to shorten the critical path.
-  const bool small_m = M < 512;
   const int64_t chunks = (K + 7) / 8;
-  if (small_m) {
-    if (chunks <= 32 * 2) return launch_rows<32, 2>(cfg, M, x, K, ldx, vec_ok, ws, Oc, nc, cap, Xq, ldq, rs, xo, ldo);
-    if (chunks <= 64 * 2) return launch_rows<64, 2>(cfg, M, x, K, ldx, vec_ok, ws, Oc, nc, cap, Xq, ldq, rs, xo, ldo);
-    if (chunks <= 128 * 2) return launch_rows<128, 2>(cfg, M, x, K, ldx, vec_ok, ws, Oc, nc, cap, Xq, ldq, rs, xo, ldo);
-    if (chunks <= 256 * 2) return launch_rows<256, 2>(cfg, M, x, K, ldx, vec_ok, ws, Oc, nc, cap, Xq, ldq, rs, xo, ldo);
-    if (chunks <= 256 * 4) return launch_rows<256, 4>(cfg, M, x, K, ldx, vec_ok, ws, Oc, nc, cap, Xq, ldq, rs, xo, ldo);
-    if (chunks <= 256 * 8) return launch_rows<256, 8>(cfg, M, x, K, ldx, vec_ok, ws, Oc, nc, cap, Xq, ldq, rs, xo, ldo);
+#define LLMINT8_ROWS(G, CPT) \
+  return launch_rows<G, CPT>(cfg, M, x, K, ldx, vec_ok, tau, ws, O, n_out, cap, Xq, ldq, rs, xo, ldo)
+  if (M < 512) {
+    if (chunks <= 32 * 2) LLMINT8_ROWS(32, 2);
+    if (chunks <= 64 * 2) LLMINT8_ROWS(64, 2);
+    if (chunks <= 128 * 2) LLMINT8_ROWS(128, 2);
+    if (chunks <= 256 * 2) LLMINT8_ROWS(256, 2);
+    if (chunks <= 256 * 4) LLMINT8_ROWS(256, 4);
+    if (chunks <= 256 * 8) LLMINT8_ROWS(256, 8);
   } else {
-    if (chunks <= 32 * 8) return launch_rows<32, 8>(cfg, M, x, K, ldx, vec_ok, ws, Oc, nc, cap, Xq, ldq, rs, xo, ldo);
-    if (chunks <= 64 * 8) return launch_rows<64, 8>(cfg, M, x, K, ldx, vec_ok, ws, Oc, nc, cap, Xq, ldq, rs, xo, ldo);
-    if (chunks <= 128 * 8) return launch_rows<128, 8>(cfg, M, x, K, ldx, vec_ok, ws, Oc, nc, cap, Xq, ldq, rs, xo, ldo);
-    if (chunks <= 256 * 8) return launch_rows<256, 8>(cfg, M, x, K, ldx, vec_ok, ws, Oc, nc, cap, Xq, ldq, rs, xo, ldo);
+    if (chunks <= 32 * 8) LLMINT8_ROWS(32, 8);
+    if (chunks <= 64 * 8) LLMINT8_ROWS(64, 8);
+    if (chunks <= 128 * 8) LLMINT8_ROWS(128, 8);
+    if (chunks <= 256 * 8) LLMINT8_ROWS(256, 8);
   }
+#undef LLMINT8_ROWS
   cfg.gridDim = dim3(static_cast<unsigned>(M));
-  return cudaLaunchKernelEx(&cfg, quantize_rows_long_kernel, x, M, K, ldx, vec_ok, ws, Oc, nc, cap, Xq, ldq, rs,
-                            xo, ldo);
+  return cudaLaunchKernelEx(&cfg, quantize_rows_long_kernel, x, M, K, ldx, tau, ws, O, n_out, cap, Xq, ldq, rs, xo,
+                            ldo);
 }
 
 }  // namespace llmint8
