@@ -175,6 +175,29 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
                                   const float* col_scale, const void* W, int64_t ldw, int64_t M, int64_t N,
                                   int64_t K, void* Y, int64_t ldy, void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of llmint8_quantize_act_rowwise_outliers (the
+ * pages have no counterpart: this serves callers of this library that cannot
+ * give it a device workspace -- an engine that plans all device memory up
+ * front, or code that may not call cudaMalloc at call time because it would
+ * synchronise the device or break a latency budget).  Same arguments and
+ * outputs, minus the workspace; the scratch (status word, column maxima,
+ * per-block counters, outlier bitmask) lives in a 256 KiB device array inside
+ * the library, which every GPU it is used on keeps until the process exits.
+ *   K <= LLMINT8_NOALLOC_MAX_K, otherwise LLMINT8_ERR_WORKSPACE and nothing
+ *   runs.  Nothing is allocated: no cudaMalloc, cudaFree or allocating library
+ *   call.  The first call on a device looks up the array's device address and
+ *   zero-fills it on `stream`; make that first call before any stream capture.
+ *   All calls share the array: calls that overlap on the GPU (different
+ *   streams or host threads) race and must be ordered by the caller.  The
+ *   status word is not reported; an outlier overflow shows as
+ *   *n_outlier > outlier_cap. */
+#define LLMINT8_NOALLOC_MAX_K 61440
+llmint8_status llmint8_quantize_act_rowwise_outliers_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
+                                                             float tau, int8_t* Xq, int64_t ldq, float* row_scale,
+                                                             int32_t* outlier_idx, int64_t outlier_cap,
+                                                             int32_t* n_outlier, void* Xo, int64_t ldo,
+                                                             void* stream);
+
 /* Synchronise `stream`, read the status word of `ws`, clear it, and return
  * LLMINT8_OK, LLMINT8_ERR_OUTLIER_OVERFLOW or LLMINT8_ERR_TIMEOUT (timeout
  * wins).  `flags_out` (host, may be NULL) receives the raw bits. */

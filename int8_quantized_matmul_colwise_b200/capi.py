@@ -69,6 +69,8 @@ SIGNATURES = {
                                    _SZ, _P]),
     "llmint8_mixed_gemm": (_ST, [_P, _I64, _P, _P, _P, _I64, _P, _I64, _P, _I64, _P, _P, _I64, _I64, _I64,
                                  _I64, _P, _I64, _P, _SZ, _P]),
+    "llmint8_quantize_act_rowwise_outliers_noalloc": (_ST, [_P, _I64, _I64, _I64, _F, _P, _I64, _P, _P, _I64, _P,
+                                                            _P, _I64, _P]),
     "llmint8_check_status": (_ST, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "llmint8_debug_int8_gemm_i32": (_ST, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64, _P, _SZ, _P]),
 }
