@@ -74,8 +74,9 @@ const char* llmint8_status_string(llmint8_status s);
  * is caller-owned device memory, 256-byte aligned, zero-filled once before its
  * first use (llmint8_workspace_init or any memset); the library leaves the
  * parts that must start at zero back at zero.  It holds the status word, the
- * column maxima, the outlier set, the row scales, Xq and the gathered outlier
- * columns of X.  Returns 0 for invalid sizes. */
+ * column maxima, the outlier set, the row scales, Xq, the gathered outlier
+ * columns of X and, for M <= 32, the split-K sums of the decode GEMM.
+ * Returns 0 for invalid sizes. */
 size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K, int64_t outlier_cap);
 
 /* Zero-fill `ws` (cudaMemsetAsync on `stream`). */
@@ -151,7 +152,8 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
  *   Y, ldy     fp16 [M, N] written, row stride ldy >= N.
  *   ws         workspace of at least llmint8_workspace_size(M, N, K, cap).
  * Runs three kernels on `stream` (scan/max, quantize/gather, int8 tcgen05
- * GEMM with the dequantize + outlier epilogue); no host synchronisation. */
+ * GEMM with the dequantize + outlier epilogue; for M <= 32 a split-K GEMM
+ * that streams Wq on all SMs); no host synchronisation. */
 llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
                                     int64_t ldk, const float* col_scale, const void* W, int64_t ldw,
                                     int64_t N, float tau, int64_t outlier_cap, void* Y, int64_t ldy,
@@ -166,7 +168,11 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
  *   outlier_idx      int32 [outlier_cap], n_outlier int32 [1] (device)
  *   Xo, ldo          fp16 [M, ldo], ldo >= outlier_cap
  *   Wq, ldk, col_scale, W, ldw, Y, ldy  as for llmint8_mixed_matmul
- *   ws               at least 256 bytes (status word).
+ *   ws               at least 256 bytes (status word).  For M <= 32 the GEMM
+ *                    splits K across CTAs when ws also holds its reduction
+ *                    scratch (a workspace of llmint8_workspace_size(M, N, K,
+ *                    outlier_cap) bytes, zero-filled once, does); the scratch is
+ *                    the end of ws and is left at zero.
  * If n_outlier > outlier_cap, Y is NaN-filled (the status bit was set by the
  * quantize call).  One kernel launch (the tcgen05 GEMM). */
 llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* row_scale,
@@ -207,7 +213,8 @@ llmint8_status llmint8_check_status(void* ws, void* stream, uint32_t* flags_out)
  * computed by the same tcgen05 kernel as llmint8_mixed_matmul (the epilogue
  * stores the raw accumulator instead of dequantizing).
  *   Xq int8 [M, ldq], Wq int8 [N, ldk] (ld % 16 == 0, 16-byte aligned),
- *   C int32 [M, ldc] written, ldc >= N.  `ws` supplies the status word. */
+ *   C int32 [M, ldc] written, ldc >= N.  `ws` supplies the status word (and,
+ *   for M <= 32, the split-K scratch as for llmint8_mixed_gemm). */
 llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const int8_t* Wq, int64_t ldk,
                                            int64_t M, int64_t N, int64_t K, int32_t* C, int64_t ldc,
                                            void* ws, size_t ws_bytes, void* stream);

@@ -106,7 +106,7 @@ def debug_int8_gemm_i32(Xq, Wq, K: int, stream=None):
     import torch
     M, N = Xq.size(0), Wq.size(0)
     C = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
-    ws = torch.zeros(256, dtype=torch.uint8, device=Xq.device)
+    ws = empty_workspace(M, N, K, 1, device=Xq.device)  # status word + decode split-K scratch
     llmint8_debug_int8_gemm_i32(Xq, Wq, K, C, ws, stream)
     return C
 

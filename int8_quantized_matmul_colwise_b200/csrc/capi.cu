@@ -114,7 +114,9 @@ bool prepare_output(CUtensorMap* map, void* Y, int64_t M, int64_t N, int64_t ldy
 // row_scale       f32 [M]
 // xq              i8  [M, ldq]
 // xo              f16 [M, ldo]
-bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t* colmax, size_t* bitmask) {
+// decode          (M <= kDecodeMaxM) split-K partial sums + tile counters, zero between calls
+bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t* colmax, size_t* bitmask,
+                 int64_t N = 0, size_t* decode = nullptr) {
   if (M < 1 || K < 1 || K > kMaxK || cap < 0 || cap > K) return false;
   size_t off = 256;
   *colmax = off;
@@ -134,8 +136,18 @@ bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t
   L->ldo = round_up(cap > 0 ? cap : 1, 8);
   L->xo = off;
   off = align_up(off + 2 * size_t(M) * size_t(L->ldo), 256);
+  if (decode) *decode = off;
+  if (M <= kDecodeMaxM && N > 0) off += decode_scratch_bytes(static_cast<int>(M), static_cast<int>(N));
   L->total = off;
   return true;
+}
+
+// Xq and Wq maps of the decode kernel: Wq is the MMA's A operand (128-row boxes),
+// Xq its B operand (boxes of the padded row count).
+bool encode_decode_maps(CUtensorMap* tmA, CUtensorMap* tmB, const int8_t* Wq, int64_t N, int64_t ldk,
+                        const int8_t* Xq, int64_t M, int64_t ldq, int64_t K) {
+  return encode_operand_map(tmA, Wq, N, K, ldk, 128) &&
+         encode_operand_map(tmB, Xq, M, K, ldq, static_cast<uint32_t>(decode_rows_padded(static_cast<int>(M))));
 }
 
 ActWs act_ws(void* ws, size_t colmax_off, size_t bitmask_off, int64_t K) {
@@ -172,8 +184,8 @@ const char* llmint8_status_string(llmint8_status s) {
 llmint8_status llmint8_workspace_layout(int64_t M, int64_t N, int64_t K, int64_t outlier_cap,
                                         llmint8_ws_layout* out) {
   if (!out || N < 1) return LLMINT8_ERR_INVALID_ARG;
-  size_t c, b;
-  if (!make_layout(M, K, outlier_cap, out, &c, &b)) return LLMINT8_ERR_INVALID_ARG;
+  size_t c, b, d;
+  if (!make_layout(M, K, outlier_cap, out, &c, &b, N, &d)) return LLMINT8_ERR_INVALID_ARG;
   return LLMINT8_OK;
 }
 
@@ -235,8 +247,8 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
   if (!aligned(Wq, 16) || !aligned(X, 2) || !aligned(W, 2) || !aligned(Y, 2) || !aligned(col_scale, 4))
     return LLMINT8_ERR_INVALID_ARG;
   llmint8_ws_layout L;
-  size_t colmax_off, bitmask_off;
-  if (!make_layout(M, K, outlier_cap, &L, &colmax_off, &bitmask_off)) return LLMINT8_ERR_INVALID_ARG;
+  size_t colmax_off, bitmask_off, decode_off;
+  if (!make_layout(M, K, outlier_cap, &L, &colmax_off, &bitmask_off, N, &decode_off)) return LLMINT8_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return LLMINT8_ERR_WORKSPACE;
   int num_sms = 0;
   llmint8_status st = current_device(&num_sms);
@@ -249,14 +261,43 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
   int32_t* n_o = reinterpret_cast<int32_t*>(b + L.n_outlier);
   void* xo = b + L.xo;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool decode = M <= kDecodeMaxM;
 
   CUtensorMap tmA, tmB;
-  if (!encode_operand_map(&tmA, xq, M, K, L.ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, gemm_b_box_rows(static_cast<int>(M))))
+  if (decode) {
+    if (!encode_decode_maps(&tmA, &tmB, Wq, N, ldk, xq, M, L.ldq, K)) return LLMINT8_ERR_CUDA;
+  } else if (!encode_operand_map(&tmA, xq, M, K, L.ldq, kGemmBM) ||
+             !encode_operand_map(&tmB, Wq, N, K, ldk, gemm_b_box_rows(static_cast<int>(M)))) {
     return LLMINT8_ERR_CUDA;
+  }
 
   cudaError_t e = launch_quantize_act(X, M, K, ldx, tau, xq, L.ldq, rs, O, outlier_cap, n_o, xo, L.ldo,
                                       act_ws(ws, colmax_off, bitmask_off, K), s, true);
   if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+
+  if (decode) {
+    DecodeArgs d = {};
+    d.M = static_cast<int>(M);
+    d.N = static_cast<int>(N);
+    d.K = static_cast<int>(K);
+    decode_split(d.M, d.N, d.K, num_sms, true, &d.splits, &d.kb_per_split);
+    d.rs = rs;
+    d.cs = col_scale;
+    d.Xo = xo;
+    d.ldo = L.ldo;
+    d.O = O;
+    d.n_o = n_o;
+    d.cap = static_cast<int>(outlier_cap);
+    d.W = W;
+    d.ldw = ldw;
+    d.Y = Y;
+    d.ldy = ldy;
+    d.partial = reinterpret_cast<int32_t*>(b + decode_off);
+    d.tile_counter = reinterpret_cast<uint32_t*>(
+        b + decode_off + align_up(size_t(N) * size_t(decode_rows_padded(d.M)) * 4, 256));
+    d.status = reinterpret_cast<uint32_t*>(b + L.status);
+    return cuda_status(launch_gemm_i8_decode(tmA, tmB, d, false, s, true));
+  }
 
   GemmArgs a = {};
   a.M = static_cast<int>(M);
@@ -300,6 +341,34 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
   llmint8_status st = current_device(&num_sms);
   if (st != LLMINT8_OK) return st;
   CUtensorMap tmA, tmB;
+  if (M <= kDecodeMaxM) {
+    if (!encode_decode_maps(&tmA, &tmB, Wq, N, ldk, Xq, M, ldq, K)) return LLMINT8_ERR_CUDA;
+    DecodeArgs d = {};
+    d.M = static_cast<int>(M);
+    d.N = static_cast<int>(N);
+    d.K = static_cast<int>(K);
+    // split-K needs its scratch after the status block of the workspace
+    const bool can_split = ws_bytes >= 256 + decode_scratch_bytes(d.M, d.N);
+    decode_split(d.M, d.N, d.K, num_sms, can_split, &d.splits, &d.kb_per_split);
+    d.rs = row_scale;
+    d.cs = col_scale;
+    d.Xo = Xo;
+    d.ldo = ldo;
+    d.O = outlier_idx;
+    d.n_o = n_outlier;
+    d.cap = static_cast<int>(outlier_cap);
+    d.W = W;
+    d.ldw = ldw;
+    d.Y = Y;
+    d.ldy = ldy;
+    // the split-K scratch is the last decode_scratch_bytes of the workspace
+    // (the decode region of a workspace sized by llmint8_workspace_size)
+    uint8_t* b = static_cast<uint8_t*>(ws) + (can_split ? (ws_bytes - decode_scratch_bytes(d.M, d.N)) / 256 * 256 : 256);
+    d.partial = reinterpret_cast<int32_t*>(b);
+    d.tile_counter = reinterpret_cast<uint32_t*>(b + align_up(size_t(N) * size_t(decode_rows_padded(d.M)) * 4, 256));
+    d.status = static_cast<uint32_t*>(ws);
+    return cuda_status(launch_gemm_i8_decode(tmA, tmB, d, false, static_cast<cudaStream_t>(stream), true));
+  }
   if (!encode_operand_map(&tmA, Xq, M, K, ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, gemm_b_box_rows(static_cast<int>(M))))
     return LLMINT8_ERR_CUDA;
   GemmArgs a = {};
@@ -336,6 +405,24 @@ llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const 
   llmint8_status st = current_device(&num_sms);
   if (st != LLMINT8_OK) return st;
   CUtensorMap tmA, tmB;
+  if (M <= kDecodeMaxM) {
+    if (!encode_decode_maps(&tmA, &tmB, Wq, N, ldk, Xq, M, ldq, K)) return LLMINT8_ERR_CUDA;
+    DecodeArgs d = {};
+    d.M = static_cast<int>(M);
+    d.N = static_cast<int>(N);
+    d.K = static_cast<int>(K);
+    const bool can_split = ws_bytes >= 256 + decode_scratch_bytes(d.M, d.N);
+    decode_split(d.M, d.N, d.K, num_sms, can_split, &d.splits, &d.kb_per_split);
+    d.C = C;
+    d.ldc = ldc;
+    // the split-K scratch is the last decode_scratch_bytes of the workspace
+    // (the decode region of a workspace sized by llmint8_workspace_size)
+    uint8_t* b = static_cast<uint8_t*>(ws) + (can_split ? (ws_bytes - decode_scratch_bytes(d.M, d.N)) / 256 * 256 : 256);
+    d.partial = reinterpret_cast<int32_t*>(b);
+    d.tile_counter = reinterpret_cast<uint32_t*>(b + align_up(size_t(N) * size_t(decode_rows_padded(d.M)) * 4, 256));
+    d.status = static_cast<uint32_t*>(ws);
+    return cuda_status(launch_gemm_i8_decode(tmA, tmB, d, true, static_cast<cudaStream_t>(stream), false));
+  }
   if (!encode_operand_map(&tmA, Xq, M, K, ldq, kGemmBM) || !encode_operand_map(&tmB, Wq, N, K, ldk, gemm_b_box_rows(static_cast<int>(M))))
     return LLMINT8_ERR_CUDA;
   GemmArgs a = {};

@@ -62,4 +62,45 @@ constexpr int kGemmBK = 128;
 
 inline unsigned gemm_b_box_rows(int M) { return gemm_uses_pair(M) ? kGemmBN / 2 : kGemmBN; }
 
+// ------------------------------------------------------------------ decode GEMM (M <= kDecodeMaxM)
+constexpr int kDecodeMaxM = 32;
+
+struct DecodeArgs {
+  int M, N, K;
+  int splits;        // K slices per 128-row tile of Wq
+  int kb_per_split;  // 128-byte K blocks per slice
+  const float* rs;
+  const float* cs;
+  const void* Xo;
+  int64_t ldo;
+  const int32_t* O;
+  const int32_t* n_o;
+  int cap;
+  const void* W;
+  int64_t ldw;
+  void* Y;
+  int64_t ldy;
+  int32_t* C;  // raw int32 output mode
+  int64_t ldc;
+  int32_t* partial;         // int32 [N, NP] split-K sums, zero between calls (splits > 1)
+  uint32_t* tile_counter;   // [ceil(N/128)] slices finished per tile, zero between calls
+  uint32_t* status;
+};
+
+// Rows of X padded to the MMA's N (16 or 32).
+int decode_rows_padded(int M);
+// K slices per tile so that tiles x slices CTAs cover num_sms (1 if !can_split).
+void decode_split(int M, int N, int K, int num_sms, bool can_split, int* splits, int* kb_per_split);
+// Scratch bytes of the split-K reduction: partial sums + per-tile counters.
+inline size_t decode_scratch_bytes(int M, int N) {
+  const size_t partial = size_t(N) * size_t(M <= 16 ? 16 : 32) * 4;
+  const size_t counters = size_t((N + 127) / 128) * 4;
+  return ((partial + 255) / 256) * 256 + ((counters + 255) / 256) * 256;
+}
+// tmA: Wq [N rows, K cols] int8 in boxes of 128 rows x 128 bytes; tmB: Xq
+// [M rows, K cols] in boxes of decode_rows_padded(M) rows x 128 bytes (both
+// 128-byte swizzle).
+cudaError_t launch_gemm_i8_decode(const CUtensorMap& tmA, const CUtensorMap& tmB, const DecodeArgs& a, bool raw_i32,
+                                  cudaStream_t stream, bool pdl);
+
 }  // namespace llmint8

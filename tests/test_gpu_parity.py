@@ -155,7 +155,9 @@ def test_activation_strided_rows(L):
 # ------------------------------------------------------------------ a5: int8 GEMM (raw accumulator)
 
 GEMM_SHAPES = [(128, 256, 128), (1, 1, 1), (5, 7, 3), (3, 33, 24), (129, 257, 520), (1, 1001, 1000),
-               (1000, 1000, 1000), (300, 600, 4096), (2047, 4095, 4100), (256, 512, 8192)]
+               (1000, 1000, 1000), (300, 600, 4096), (2047, 4095, 4100), (256, 512, 8192),
+               # decode kernel (M <= 32): split-K over all SMs, uneven K-block split, both padded widths
+               (8, 4096, 4096), (16, 4096, 4100), (17, 1000, 1000), (32, 4095, 2048), (33, 520, 256)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
@@ -276,6 +278,26 @@ def test_repeat_calls_are_deterministic_and_reuse_workspace(L):
     L.mixed_matmul(dev(wl.make_x(wl.get("ragged_129x257x520"))[::-1].copy()), Wq, cs, Wd, 3.0, ws=ws)
     c = host(L.mixed_matmul(Xd, Wq, cs, Wd, w.tau, ws=ws)).view(np.uint16)
     assert np.array_equal(a, b) and np.array_equal(a, c)
+    assert_status_ok(L, ws)
+
+
+def test_decode_repeat_calls_leave_split_k_scratch_at_zero(L):
+    """Decode-shaped calls reduce split-K partial sums in the workspace and
+    must leave it at zero: repeated calls through one workspace agree."""
+    w = wl.get("decode_m8")
+    X, W = wl.make_inputs(w)
+    Wd = dev(W)
+    Wq, cs = L.quantize_weight_colwise(Wd)
+    ws = L.empty_workspace(w.M, w.N, w.K, w.K)
+    Xd = dev(X)
+    ys = [host(L.mixed_matmul(Xd, Wq, cs, Wd, w.tau, ws=ws)).view(np.uint16) for _ in range(3)]
+    assert np.array_equal(ys[0], ys[1]) and np.array_equal(ys[0], ys[2])
+    r = oracle.mixed_matmul(X, W, w.tau)
+    y_close(ys[0].view(np.float16), r["Y"])
+    # the split entry points on the same data (mixed_gemm with a full-size workspace)
+    act = L.quantize_act_rowwise_outliers(Xd, w.tau)
+    y2 = host(L.mixed_gemm(act, Wq, cs, Wd, ws=L.empty_workspace(w.M, w.N, w.K, w.K))).view(np.uint16)
+    assert np.array_equal(y2, ys[0])
     assert_status_ok(L, ws)
 
 
