@@ -46,6 +46,10 @@ def parse_args():
     ap.add_argument("--workload", default="ffn_6p7b_prefill")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the supplementary decode-shape measurement")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture the K timed steps in one CUDA graph (small, launch-bound workloads)")
     return ap.parse_args()
 
 
@@ -245,6 +249,58 @@ def config_of(wl_, n_o, extra=None):
     return c
 
 
+# ------------------------------------------------------------------ decode shapes
+def measure_decode(L, torch, dev, peaks, names=("decode_m1", "decode_m8", "decode_m32"), reps=20):
+    """Decode-shaped calls of llmint8_mixed_matmul (M <= 32, HBM-bound on
+    streaming Wq): per-call time from a CUDA graph of one pass over rotating
+    weight copies (together > 3x L2, so every call streams Wq from HBM),
+    replayed `reps` times between CUDA events on the replaying stream."""
+    import workloads as wl
+    out = {}
+    for name in names:
+        w = wl.get(name)
+        X_np, W_np = wl.make_inputs(w)
+        W = torch.from_numpy(W_np).to(dev)
+        X = torch.from_numpy(X_np).to(dev)
+        Wq0, cs0 = L.quantize_weight_colwise(W)
+        n_sets = max(2, math.ceil(3 * L2_BYTES / Wq0.numel()))
+        sets = [(Wq0.clone(), cs0.clone(), torch.empty((w.M, w.N), dtype=torch.float16, device=dev),
+                 L.empty_workspace(w.M, w.N, w.K, w.K, device=dev)) for _ in range(n_sets)]
+        del Wq0, cs0
+
+        def one_pass(on):
+            for (q, c, y, ws) in sets:
+                L.llmint8_mixed_matmul(X, q, c, W, w.tau, w.K, y, ws, on)
+
+        for _ in range(3):
+            one_pass(torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            one_pass(torch.cuda.current_stream())
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) * 1e-3 / (reps * n_sets)
+        st, flags = L.llmint8_check_status(sets[0][3])
+        if st != 0:
+            raise RuntimeError(f"device status after the {name} run: {st} flags={flags}")
+        n_o = int(L.workspace_views(sets[0][3], w.M, w.N, w.K, w.K)["n_outlier"].item())
+        byts = algorithmic_bytes(w.M, w.N, w.K, n_o)
+        out[name] = {"M": w.M, "N": w.N, "K": w.K, "us_per_call": t * 1e6, "achieved_gbs": byts / t / 1e9,
+                     "frac_hbm": byts / t / 1e9 / peaks["hbm_gbs"],
+                     "roofline_us": byts / (peaks["hbm_gbs"] * 1e9) * 1e6, "algorithmic_bytes": byts,
+                     "kernels_per_call": L.llmint8_mixed_matmul_kernels(X, w.N), "n_outlier": n_o,
+                     "timing": f"CUDA graph of {n_sets} calls on rotating Wq copies, replayed {reps}x"}
+        del sets, g
+    return out
+
+
 # ------------------------------------------------------------------ our arm
 def source_digest(path):
     with open(path, "rb") as f:
@@ -305,9 +361,9 @@ def run_ours(args, wl_, dist):
         })
     stream = torch.cuda.current_stream()
 
-    def step(i):
+    def step(i, on=stream):
         s = sets[i % n_sets]
-        L.llmint8_mixed_matmul(s["X"], s["Wq"], s["cs"], W, wl_.tau, cap, s["Y"], s["ws"], stream)
+        L.llmint8_mixed_matmul(s["X"], s["Wq"], s["cs"], W, wl_.tau, cap, s["Y"], s["ws"], on)
 
     clocks = ClockSampler(torch.cuda.current_device()).start()
     for i in range(args.warmup):
@@ -318,6 +374,16 @@ def run_ours(args, wl_, dist):
         raise RuntimeError(f"device status after warm-up: {st} flags={flags}")
     views = L.workspace_views(sets[0]["ws"], M, N, K, cap)
     n_o = int(views["n_outlier"].item())
+    n_kern = L.llmint8_mixed_matmul_kernels(sets[0]["X"], N)  # 1: the one-kernel decode path
+
+    graph = None
+    if args.graph:  # the K timed steps as one CUDA graph, captured before the timed region
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):  # captured on torch's side stream, replayed on `stream`
+            for i in range(args.steps):
+                step(i, torch.cuda.current_stream())
+        graph.replay()
+        torch.cuda.synchronize()
 
     # ---- timed region: exactly K steps, inputs resident in HBM
     dist.barrier(torch)
@@ -325,8 +391,11 @@ def run_ours(args, wl_, dist):
     ev_a, ev_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_host0 = time.perf_counter()
     ev_a.record(stream)
-    for i in range(args.steps):
-        step(i)
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(args.steps):
+            step(i)
     ev_b.record(stream)
     torch.cuda.synchronize()
     t_host1 = time.perf_counter()
@@ -338,50 +407,63 @@ def run_ours(args, wl_, dist):
     value = dist.world * ops * args.steps / (el_ms / 1e3) / 1e12
     ms_per_step = el_ms / args.steps
 
-    # ---- per-kernel durations (same inputs, split entry points, events on the launching stream)
-    acts = []
-    for s in sets:
-        acts.append({
-            "Xq": torch.empty((M, L.round_up(K, 16)), dtype=torch.int8, device=dev),
-            "row_scale": torch.empty(M, dtype=torch.float32, device=dev),
-            "outlier_idx": torch.empty(cap, dtype=torch.int32, device=dev),
-            "n_outlier": torch.empty(1, dtype=torch.int32, device=dev),
-            "Xo": torch.empty((M, cap), dtype=torch.float16, device=dev),
-        })
-    n_k = max(10, min(args.steps, 200))
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-            torch.cuda.Event(enable_timing=True)) for _ in range(n_k)]
-    for rep in range(2):  # first pass warms up
-        for i in range(n_k):
-            s, a = sets[i % n_sets], acts[i % n_sets]
-            if rep:
-                evs[i][0].record(stream)
-            L.llmint8_quantize_act_rowwise_outliers(s["X"], wl_.tau, a["Xq"], a["row_scale"], a["outlier_idx"],
-                                                    a["n_outlier"], a["Xo"], s["ws"], stream)
-            if rep:
-                evs[i][1].record(stream)
-            L.llmint8_mixed_gemm(a["Xq"], a["row_scale"], a["outlier_idx"], a["n_outlier"], a["Xo"], s["Wq"],
-                                 s["cs"], W, K, s["Y"], s["ws"], stream)
-            if rep:
-                evs[i][2].record(stream)
-        torch.cuda.synchronize()
-    t_quant = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) * 1e3  # us
-    t_gemm = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) * 1e3
-    t_gemm = dist.max(torch, t_gemm)
-    gemm_tops = ops / (t_gemm * 1e-6) / 1e12
-
-    traffic = recorded_traffic(wl_.name)
-    roofline = {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TFLOP/s",
-                "frac": gemm_tops / int8_peak, "traffic": traffic,
-                "kernel": "gemm_i8_kernel (tcgen05 kind::i8 + dequant/outlier epilogue)",
-                "peak_note": f"int8 dense = {INT8_PER_BF16:g} x bf16 burst {peaks['bf16_tflops']:.1f} TFLOP/s "
-                             f"({peaks['source']}); algorithmic ops per launch = 2MNK = {ops:.4g}"}
     byts = algorithmic_bytes(M, N, K, n_o)
-    t_roof = max(ops / (int8_peak * 1e12), byts / (peaks["hbm_gbs"] * 1e9))
-    path = {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step * 1e-3),
-            "algorithmic_bytes": byts, "int8_peak_tops": int8_peak, "hbm_gbs": peaks["hbm_gbs"],
-            "scan_quantize_us": t_quant, "gemm_us": t_gemm,
-            "scan_quantize_gbs": (2 * M * K + M * K) / (t_quant * 1e-6) / 1e9}
+    if n_kern == 1:
+        # one kernel per step: its duration is the step's, taken over the timed region
+        t_step = ms_per_step * 1e-3
+        gbs = byts / t_step / 1e9
+        roofline = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                    "kernel": "decode_fused_kernel (a1-a7 in one kernel: cluster split-K, tcgen05 kind::i8)",
+                    "peak_note": f"measured HBM copy bandwidth ({peaks['source']}); algorithmic bytes per launch "
+                                 f"= 2MK + NK + 2*n_o*N + 4(M+N) + 2MN = {byts}"}
+        path = {"t_roof_us": byts / (peaks["hbm_gbs"] * 1e9) * 1e6, "t_step_us": ms_per_step * 1e3,
+                "frac": byts / (peaks["hbm_gbs"] * 1e9) / t_step, "algorithmic_bytes": byts,
+                "int8_peak_tops": int8_peak, "hbm_gbs": peaks["hbm_gbs"]}
+    else:
+        # ---- per-kernel durations (same inputs, split entry points, events on the launching stream)
+        acts = []
+        for s in sets:
+            acts.append({
+                "Xq": torch.empty((M, L.round_up(K, 16)), dtype=torch.int8, device=dev),
+                "row_scale": torch.empty(M, dtype=torch.float32, device=dev),
+                "outlier_idx": torch.empty(cap, dtype=torch.int32, device=dev),
+                "n_outlier": torch.empty(1, dtype=torch.int32, device=dev),
+                "Xo": torch.empty((M, cap), dtype=torch.float16, device=dev),
+            })
+        n_k = max(10, min(args.steps, 200))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                torch.cuda.Event(enable_timing=True)) for _ in range(n_k)]
+        for rep in range(2):  # first pass warms up
+            for i in range(n_k):
+                s, a = sets[i % n_sets], acts[i % n_sets]
+                if rep:
+                    evs[i][0].record(stream)
+                L.llmint8_quantize_act_rowwise_outliers(s["X"], wl_.tau, a["Xq"], a["row_scale"], a["outlier_idx"],
+                                                        a["n_outlier"], a["Xo"], s["ws"], stream)
+                if rep:
+                    evs[i][1].record(stream)
+                L.llmint8_mixed_gemm(a["Xq"], a["row_scale"], a["outlier_idx"], a["n_outlier"], a["Xo"], s["Wq"],
+                                     s["cs"], W, K, s["Y"], s["ws"], stream)
+                if rep:
+                    evs[i][2].record(stream)
+            torch.cuda.synchronize()
+        t_quant = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) * 1e3  # us
+        t_gemm = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) * 1e3
+        t_gemm = dist.max(torch, t_gemm)
+        gemm_tops = ops / (t_gemm * 1e-6) / 1e12
+
+        traffic = recorded_traffic(wl_.name)
+        roofline = {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TFLOP/s",
+                    "frac": gemm_tops / int8_peak, "traffic": traffic,
+                    "kernel": "gemm_i8_kernel (tcgen05 kind::i8 + dequant/outlier epilogue)",
+                    "peak_note": f"int8 dense = {INT8_PER_BF16:g} x bf16 burst {peaks['bf16_tflops']:.1f} TFLOP/s "
+                                 f"({peaks['source']}); algorithmic ops per launch = 2MNK = {ops:.4g}"}
+        t_roof = max(ops / (int8_peak * 1e12), byts / (peaks["hbm_gbs"] * 1e9))
+        path = {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step * 1e-3),
+                "algorithmic_bytes": byts, "int8_peak_tops": int8_peak, "hbm_gbs": peaks["hbm_gbs"],
+                "scan_quantize_us": t_quant, "gemm_us": t_gemm,
+                "scan_quantize_gbs": (2 * M * K + M * K) / (t_quant * 1e-6) / 1e9}
 
     # ---- end to end through the public API with host buffers
     Xh = torch.from_numpy(X_np).pin_memory()
@@ -424,10 +506,14 @@ def run_ours(args, wl_, dist):
             "l2": f"{n_sets} rotating input sets (X, Wq, Y, workspace) of {per_set / 2**20:.0f} MiB each "
                   f"> 3x L2; consecutive steps touch different buffers",
             "weight_quant_ms_offline": wq_ms, "workspace_bytes": ws_bytes,
-            "launch": "llmint8_mixed_matmul: 3 kernels chained with programmatic dependent launch"}),
+            "launch": ("llmint8_mixed_matmul: 1 kernel (a1-a7 fused)" if n_kern == 1 else
+                       "llmint8_mixed_matmul: 3 kernels chained with programmatic dependent launch") +
+                      ("; the K steps replayed from one CUDA graph" if args.graph else "")}),
         "roofline": roofline, "path_roofline": path, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": 3 * args.steps, "clocks": clk,
+        "gpu_launches": n_kern * args.steps, "clocks": clk,
     }
+    if not args.no_decode and M > 32:
+        line["decode"] = measure_decode(L, torch, dev, peaks)
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()

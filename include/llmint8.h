@@ -153,11 +153,22 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
  *   ws         workspace of at least llmint8_workspace_size(M, N, K, cap).
  * Runs three kernels on `stream` (scan/max, quantize/gather, int8 tcgen05
  * GEMM with the dequantize + outlier epilogue; for M <= 32 a split-K GEMM
- * that streams Wq on all SMs); no host synchronisation. */
+ * that streams Wq on all SMs).  For M <= 32 with K % 8 == 0, ldx % 8 == 0,
+ * X 16-byte aligned and K <= 16384 (and N, K small enough that each CTA's
+ * share of Xq fits in 32 KB of shared memory), one kernel does all of it:
+ * CTA clusters split K, exchange outlier flags and row maxima through
+ * distributed shared memory and reduce their int32 partial sums there.  The
+ * workspace then receives the same Xq, row scales, O, n_o and Xo.  No host
+ * synchronisation. */
 llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
                                     int64_t ldk, const float* col_scale, const void* W, int64_t ldw,
                                     int64_t N, float tau, int64_t outlier_cap, void* Y, int64_t ldy,
                                     void* ws, size_t ws_bytes, void* stream);
+
+/* Number of kernels llmint8_mixed_matmul launches on the current device for
+ * these arguments (1 on the one-kernel decode path, else 3; 0 for invalid
+ * sizes or no supported device).  Host-only query. */
+int llmint8_mixed_matmul_kernels(int64_t M, int64_t N, int64_t K, int64_t ldx, const void* X);
 
 /* Steps a5-a7 alone, on an activation already quantized by
  * llmint8_quantize_act_rowwise_outliers (so that one quantized X can feed

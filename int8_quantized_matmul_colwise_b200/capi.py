@@ -72,6 +72,7 @@ SIGNATURES = {
     "llmint8_quantize_act_rowwise_outliers_noalloc": (_ST, [_P, _I64, _I64, _I64, _F, _P, _I64, _P, _P, _I64, _P,
                                                             _P, _I64, _P]),
     "llmint8_check_status": (_ST, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
+    "llmint8_mixed_matmul_kernels": (ctypes.c_int, [_I64, _I64, _I64, _I64, _P]),
     "llmint8_debug_int8_gemm_i32": (_ST, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64, _P, _SZ, _P]),
 }
 
@@ -239,6 +240,12 @@ def llmint8_check_status(ws, stream=None) -> Tuple[int, int]:
     flags = ctypes.c_uint32(0)
     st = lib().llmint8_check_status(_ptr(ws), _stream(stream), ctypes.byref(flags))
     return int(st), int(flags.value)
+
+
+def llmint8_mixed_matmul_kernels(X, N: int) -> int:
+    """Kernels llmint8_mixed_matmul launches for this X and N (1 or 3)."""
+    M, K = X.shape
+    return int(lib().llmint8_mixed_matmul_kernels(M, N, K, _ld(X), _ptr(X)))
 
 
 def llmint8_debug_int8_gemm_i32(Xq, Wq, K: int, C, ws, stream=None):

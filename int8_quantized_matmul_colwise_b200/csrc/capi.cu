@@ -164,6 +164,15 @@ llmint8_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK
 
 bool valid_tau(float tau) { return !std::isnan(tau) && tau >= 0.0f; }
 
+// Whether llmint8_mixed_matmul runs the one-kernel decode path for these
+// arguments (then *splits, *kb_per receive its plan).
+bool use_fused_decode(int64_t M, int64_t N, int64_t K, int64_t ldx, const void* X, int num_sms, int* splits,
+                      int* kb_per, int* stages) {
+  return M <= kDecodeMaxM && K % 8 == 0 && ldx % 8 == 0 && aligned(X, 16) &&
+         decode_fused_plan(static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), num_sms, splits, kb_per,
+                           stages);
+}
+
 }  // namespace
 
 extern "C" {
@@ -187,6 +196,15 @@ llmint8_status llmint8_workspace_layout(int64_t M, int64_t N, int64_t K, int64_t
   size_t c, b, d;
   if (!make_layout(M, K, outlier_cap, out, &c, &b, N, &d)) return LLMINT8_ERR_INVALID_ARG;
   return LLMINT8_OK;
+}
+
+int llmint8_mixed_matmul_kernels(int64_t M, int64_t N, int64_t K, int64_t ldx, const void* X) {
+  if (!X || M < 1 || N < 1 || K < 1 || K > kMaxK || ldx < K || M > (int64_t(1) << 31) - 1 ||
+      N > (int64_t(1) << 31) - 1)
+    return 0;
+  int num_sms = 0, s = 0, kb = 0, stages = 0;
+  if (current_device(&num_sms) != LLMINT8_OK) return 0;
+  return use_fused_decode(M, N, K, ldx, X, num_sms, &s, &kb, &stages) ? 1 : 3;
 }
 
 size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K, int64_t outlier_cap) {
@@ -262,6 +280,38 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
   void* xo = b + L.xo;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool decode = M <= kDecodeMaxM;
+
+  // Decode calls whose X rows allow 16-byte loads: the whole path in one kernel.
+  int f_splits = 0, f_kb = 0, f_stages = 0;
+  if (use_fused_decode(M, N, K, ldx, X, num_sms, &f_splits, &f_kb, &f_stages)) {
+    CUtensorMap tmW;
+    if (!encode_operand_map(&tmW, Wq, N, K, ldk, 128)) return LLMINT8_ERR_CUDA;
+    FusedArgs f = {};
+    f.X = X;
+    f.ldx = ldx;
+    f.M = static_cast<int>(M);
+    f.N = static_cast<int>(N);
+    f.K = static_cast<int>(K);
+    f.tau = tau;
+    f.cs = col_scale;
+    f.W = W;
+    f.ldw = ldw;
+    f.Y = Y;
+    f.ldy = ldy;
+    f.Xq = xq;
+    f.ldq = L.ldq;
+    f.rs = rs;
+    f.O = O;
+    f.n_out = n_o;
+    f.Xo = xo;
+    f.ldo = L.ldo;
+    f.cap = static_cast<int>(outlier_cap);
+    f.status = reinterpret_cast<uint32_t*>(b + L.status);
+    f.splits = f_splits;
+    f.kb_per = f_kb;
+    f.stages = f_stages;
+    return cuda_status(launch_decode_fused(tmW, f, s, true));
+  }
 
   CUtensorMap tmA, tmB;
   if (decode) {

@@ -579,6 +579,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *s.tmem_slot;
 
   griddep_wait();  // Xq, rs, O, n_o and Xo are written by the quantize kernel
+  // The next launch on the stream may get resident now: every kernel of this
+  // library waits (griddepcontrol.wait) for this grid to complete before it
+  // touches memory this grid reads or writes.
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) run_producer<kPair>(&tmA, &tmB, s, sc, rank, p.status);

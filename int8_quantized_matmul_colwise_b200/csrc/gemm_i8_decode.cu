@@ -52,25 +52,6 @@ struct GeoD {
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
-__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* status,
-                                             volatile int* abort) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t n = 0;
-  while (true) {
-    if (mbar_try_wait(a, parity)) return true;
-    if ((++n & 63u) == 0u) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(status, kStatusTimeout);
-        *abort = 1;
-        return false;
-      }
-    }
-  }
-}
-
 __device__ __forceinline__ void red_add_s32(int32_t* p, int32_t v) {
   asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -193,6 +174,10 @@ __global__ void __launch_bounds__(kThreadsD, 1)
   }
 
   griddep_wait();  // Xq, rs, O, n_o and Xo are written by the quantize kernel
+  // The next launch on the stream may get resident now: every kernel of this
+  // library waits (griddepcontrol.wait) for this grid to complete before it
+  // touches memory this grid reads or writes.
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -203,7 +188,7 @@ __global__ void __launch_bounds__(kThreadsD, 1)
       for (int i = kStagesD; i < nkb && ok; ++i) {
         const int st = i % kStagesD;
         const uint32_t ph = static_cast<uint32_t>(i / kStagesD - 1) & 1u;
-        if (!wait_bounded(&empty[st], ph, p.status, abort)) {
+        if (!mbar_wait_abortable(&empty[st], ph, p.status, abort)) {
           ok = false;
           break;
         }
@@ -225,7 +210,7 @@ __global__ void __launch_bounds__(kThreadsD, 1)
       for (int i = 0; i < nkb; ++i) {
         const int st = i % kStagesD;
         const uint32_t ph = static_cast<uint32_t>(i / kStagesD) & 1u;
-        if (!wait_bounded(&full[st], ph, p.status, abort)) {
+        if (!mbar_wait_abortable(&full[st], ph, p.status, abort)) {
           ok = false;
           break;
         }
@@ -275,7 +260,7 @@ __global__ void __launch_bounds__(kThreadsD, 1)
     int32_t acc[NP];
     bool got = true;
     if (nkb > 0) {
-      got = wait_bounded(tfull, 0, p.status, abort);
+      got = mbar_wait_abortable(tfull, 0, p.status, abort);
       got = named_bar_and(2, 128, got);  // also makes s_rs / s_xo visible
       if (got) {
         tc_fence_after();

@@ -103,4 +103,38 @@ inline size_t decode_scratch_bytes(int M, int N) {
 cudaError_t launch_gemm_i8_decode(const CUtensorMap& tmA, const CUtensorMap& tmB, const DecodeArgs& a, bool raw_i32,
                                   cudaStream_t stream, bool pdl);
 
+// ------------------------------------------------------------------ fused decode path (a1-a7, one kernel)
+constexpr int kFusedMaxK = 16384;     // longest K the fused kernel takes
+constexpr int kFusedXqBytes = 32768;  // quantized activation a CTA keeps in shared memory
+
+struct FusedArgs {
+  const void* X;  // fp16 [M, ldx], rows 16-byte aligned, K % 8 == 0
+  int64_t ldx;
+  int M, N, K;
+  float tau;
+  const float* cs;
+  const void* W;  // fp16 [K, ldw]: outlier rows
+  int64_t ldw;
+  void* Y;
+  int64_t ldy;
+  int8_t* Xq;  // workspace outputs, written by the first cluster
+  int64_t ldq;
+  float* rs;
+  int32_t* O;
+  int32_t* n_out;
+  void* Xo;
+  int64_t ldo;
+  int cap;
+  uint32_t* status;
+  int splits;  // CTAs per tile (cluster size): 1, 2, 4 or 8
+  int kb_per;  // 128-column K blocks per CTA (a power of two)
+  int stages;  // Wq ring depth: 4 (two CTAs per SM) or 8
+};
+
+// Cluster size and K blocks per CTA for a decode call; false if the fused
+// kernel does not take this shape (the caller then runs the three-kernel path).
+bool decode_fused_plan(int M, int N, int K, int num_sms, int* splits, int* kb_per, int* stages);
+// tmA: Wq [N rows, K cols] int8, boxes of 128 rows x 128 bytes, 128-byte swizzle.
+cudaError_t launch_decode_fused(const CUtensorMap& tmA, const FusedArgs& a, cudaStream_t stream, bool pdl);
+
 }  // namespace llmint8

@@ -44,4 +44,83 @@ __device__ __forceinline__ uint32_t abs_bits(__half h) {
   return b > 0x7C00u ? 0u : b;
 }
 
+// 8 consecutive fp16 of a row by scalar loads (unaligned rows or a ragged end).
+__device__ __forceinline__ uint4 load8_scalar(const __half* __restrict__ row, int64_t K, int64_t c) {
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t lo = (c + 2 * e < K) ? __half_as_ushort(row[c + 2 * e]) : 0u;
+    const uint32_t hi = (c + 2 * e + 1 < K) ? __half_as_ushort(row[c + 2 * e + 1]) : 0u;
+    w[e] = lo | (hi << 16);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// 8 consecutive fp16 of a row as one 16-byte register quad (zero past K).
+// kVec: rows are 16-byte aligned and K % 8 == 0, so every chunk that starts
+// before K is one aligned 16-byte load (decided on the host).
+template <bool kVec>
+__device__ __forceinline__ uint4 load8_packed(const __half* __restrict__ row, int64_t K, int64_t c) {
+  if constexpr (kVec) return __ldg(reinterpret_cast<const uint4*>(row + c));
+  else return load8_scalar(row, K, c);
+}
+
+__device__ __forceinline__ unsigned short half_bits_at(const uint4& u, int e) {
+  const uint32_t w = (e < 2) ? u.x : (e < 4) ? u.y : (e < 6) ? u.z : u.w;
+  return static_cast<unsigned short>((e & 1) ? (w >> 16) : (w & 0xFFFFu));
+}
+
+__device__ __forceinline__ uint2 pack8(const int (&q)[8]) {
+  uint2 out;
+  out.x = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+  out.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
+  return out;
+}
+
+// Codes of 8 values (fp16 pairs in u) by the exact comparisons.
+__device__ __forceinline__ uint2 quantize8_exact(uint4 u, float s, float inv) {
+  const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+  int q[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(h2[e]);
+    q[2 * e] = quantize_exact(f.x, s, inv);
+    q[2 * e + 1] = quantize_exact(f.y, s, inv);
+  }
+  return pack8(q);
+}
+
+// Codes of 8 values by rounding x * (127 / s).  With k = fl(127/s) and
+// r = fl(x k), |r - 127x/s| <= 127 (2^-24 + 2^-24)(1 + 2^-24) < 2^-16, so when
+// |r - rint(r)| < 1/2 - 2^-15 the exact value is strictly nearer to rint(r)
+// than to any other integer and rint(r) is its rounding (no tie possible).
+// Otherwise (about one value in 16000, or NaN) tie_risk is set and the caller
+// redoes the chunk with quantize8_exact.
+// rint is taken as t = r + 1.5 * 2^23: for |r| < 2^22 the sum lies in
+// [2^23, 2^24) where the spacing is 1, so it is rounded to the nearest integer
+// (ties to even), t - 1.5 * 2^23 is exact, and the low byte of t's bit pattern
+// is the integer's low byte (two's complement) -- all on the FMA pipe.
+__device__ __forceinline__ uint2 quantize8(uint4 u, float k, bool& tie_risk) {
+  constexpr float kSafe = 0.499969482421875f;  // 1/2 - 2^-15
+  constexpr float kBias = 12582912.0f;         // 1.5 * 2^23
+  const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+  uint32_t t[8];
+  const float2 k2 = make_float2(k, k);
+  const float2 b2 = make_float2(kBias, kBias);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 r = __fmul2_rn(__half22float2(h2[e]), k2);
+    const float2 tb = __fadd2_rn(r, b2);
+    const float2 q = __fadd2_rn(tb, make_float2(-kBias, -kBias));
+    const float2 d = __fadd2_rn(r, make_float2(-q.x, -q.y));
+    tie_risk |= !(fabsf(d.x) < kSafe) | !(fabsf(d.y) < kSafe);  // true for NaN as well
+    t[2 * e] = __float_as_uint(tb.x);
+    t[2 * e + 1] = __float_as_uint(tb.y);
+  }
+  uint2 out;
+  out.x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+  out.y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+  return out;
+}
+
 }  // namespace llmint8

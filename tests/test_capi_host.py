@@ -99,3 +99,11 @@ def test_binding_refuses_host_tensors():
     W = torch.zeros(8, 8, dtype=torch.float16)
     with pytest.raises(ValueError):
         L.llmint8_quantize_weight_colwise(W, torch.zeros(8, 16, dtype=torch.int8), torch.zeros(8))
+
+
+def test_kernel_count_query_rejects_invalid_sizes(lib):
+    f = lib.llmint8_mixed_matmul_kernels
+    assert f(0, 16, 16, 16, 0x1000) == 0        # M < 1
+    assert f(4, 16, 16, 8, 0x1000) == 0         # ldx < K
+    assert f(4, 16, 16, 16, None) == 0          # no X
+    assert f(4, 16, 200000, 200000, 0x1000) == 0  # K beyond the int32 accumulator bound

@@ -215,6 +215,9 @@ def check_path(L, X, W, tau, rows=None, cap=None):
     assert np.array_equal(host(v["outlier_idx"])[:n], r["O"])
     assert np.array_equal(host(v["row_scale"]), r["rs"])
     assert np.array_equal(host(v["xq"])[:, :K], r["Xq"])
+    assert not host(v["xq"])[:, K:].any()
+    if n <= (K if cap is None else cap):  # the gathered outlier columns, bit for bit
+        assert np.array_equal(host(v["xo"])[:, :n].view(np.uint16), X[:, r["O"]].view(np.uint16))
     assert np.array_equal(host(cs), cs_ref)
     Yg = host(Y)
     Yg = Yg if rows is None else Yg[rows]
@@ -282,8 +285,9 @@ def test_repeat_calls_are_deterministic_and_reuse_workspace(L):
 
 
 def test_decode_repeat_calls_leave_split_k_scratch_at_zero(L):
-    """Decode-shaped calls reduce split-K partial sums in the workspace and
-    must leave it at zero: repeated calls through one workspace agree."""
+    """Decode-shaped calls: the one-kernel path of mixed_matmul and the split
+    entry points (whose split-K GEMM reduces partial sums in the workspace and
+    must leave them at zero) agree bit for bit over repeated calls."""
     w = wl.get("decode_m8")
     X, W = wl.make_inputs(w)
     Wd = dev(W)
@@ -296,9 +300,62 @@ def test_decode_repeat_calls_leave_split_k_scratch_at_zero(L):
     y_close(ys[0].view(np.float16), r["Y"])
     # the split entry points on the same data (mixed_gemm with a full-size workspace)
     act = L.quantize_act_rowwise_outliers(Xd, w.tau)
-    y2 = host(L.mixed_gemm(act, Wq, cs, Wd, ws=L.empty_workspace(w.M, w.N, w.K, w.K))).view(np.uint16)
-    assert np.array_equal(y2, ys[0])
+    ws2 = L.empty_workspace(w.M, w.N, w.K, w.K)
+    for _ in range(3):
+        y2 = host(L.mixed_gemm(act, Wq, cs, Wd, ws=ws2)).view(np.uint16)
+        assert np.array_equal(y2, ys[0])
     assert_status_ok(L, ws)
+    assert_status_ok(L, ws2)
+
+
+# (M, N, K) of decode calls: a single CTA; clusters of 8 with empty K slices;
+# Xq padding (K % 16 == 8); 16 K blocks per CTA (Wq ring refills); N too wide
+# for the one-kernel path (three kernels); a 2-row call at the decode size.
+DECODE_SHAPES = [(1, 128, 128), (5, 300, 1032), (17, 520, 2056), (24, 129, 264), (9, 2048, 16384),
+                 (32, 1024, 8192), (16, 16384, 4096), (2, 4096, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
+def test_decode_shapes(L, M, N, K):
+    rng = np.random.default_rng(M * 1000003 + N * 1009 + K)
+    X, W, _ = wl.random_small(rng, M, K, N, max(1, K // 700))
+    check_path(L, X, W, 6.0)
+
+
+def test_decode_every_column_an_outlier_and_overflow(L):
+    """tau = 0: all 512 columns are outliers, more than the epilogue stages
+    (it walks the bitmask for the rest); a cap below n_o gives NaN and the
+    overflow bit."""
+    rng = np.random.default_rng(77)
+    X, W, _ = wl.random_small(rng, 4, 512, 256, 2)
+    Yg, r = check_path(L, X, W, 0.0)
+    assert r["O"].size == 512
+    Y, ws, v, _, (st, flags) = run_path(L, X, W, 6.0, cap=1)
+    assert st == 5 and flags & 1
+    assert int(host(v["n_outlier"])[0]) == 2
+    assert np.isnan(host(Y).astype(np.float32)).all()
+
+
+def test_decode_unaligned_rows_take_the_three_kernel_path(L):
+    """X rows that are not 16-byte aligned (ldx = K + 1) go through the
+    scan / quantize / split-K GEMM kernels; same results."""
+    M, N, K = 8, 1000, 1000
+    rng = np.random.default_rng(5)
+    X, W, _ = wl.random_small(rng, M, K, N, 3)
+    Xw = np.zeros((M, K + 1), np.float16)
+    Xw[:, :K] = X
+    Xd = dev(Xw)[:, :K]
+    Wd = dev(W)
+    Wq, cs = L.quantize_weight_colwise(Wd)
+    ws = L.empty_workspace(M, N, K, K)
+    Y = host(L.mixed_matmul(Xd, Wq, cs, Wd, 6.0, ws=ws))
+    assert_status_ok(L, ws)
+    r = oracle.mixed_matmul(X, W, 6.0)
+    v = L.workspace_views(ws, M, N, K, K)
+    assert np.array_equal(host(v["xq"])[:, :K], r["Xq"])
+    y_close(Y, r["Y"])
+    Ya = host(L.mixed_matmul(dev(X), Wq, cs, Wd, 6.0))  # the one-kernel path, same bits
+    assert np.array_equal(Ya.view(np.uint16), Y.view(np.uint16))
 
 
 # ------------------------------------------------------------------ full-size workloads (sampled rows)
