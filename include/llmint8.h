@@ -130,7 +130,13 @@ llmint8_status llmint8_quantize_weight_colwise(const void* W, int64_t K, int64_t
  *   Xo          optional fp16 [M, ldo] (NULL to skip): Xo[i,t] = X[i,O[t]]
  *               for t < min(n_o, cap); ldo >= outlier_cap.
  *   ws          workspace (see llmint8_workspace_size).
- * All outputs are device-side; nothing is copied to the host. */
+ * All outputs are device-side; nothing is copied to the host.  When X's rows
+ * are 16-byte aligned (ldx % 8 == 0, K % 8 == 0) and X fits in shared memory
+ * spread over the SMs (at most 16 rows and 200 KB per SM), the step is one
+ * persistent kernel: X is read once, the CTAs meet at a grid barrier between
+ * the column scan and the row quantization, and no other kernel may hold SMs
+ * for long on other streams meanwhile (the barrier gives up after 2 s and sets
+ * LLMINT8_STATUS_TIMEOUT).  Otherwise two kernels (column scan, rows). */
 llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, int64_t K, int64_t ldx,
                                                      float tau, int8_t* Xq, int64_t ldq, float* row_scale,
                                                      int32_t* outlier_idx, int64_t outlier_cap,
@@ -217,7 +223,9 @@ llmint8_status llmint8_quantize_act_rowwise_outliers_noalloc(const void* X, int6
 
 /* Synchronise `stream`, read the status word of `ws`, clear it, and return
  * LLMINT8_OK, LLMINT8_ERR_OUTLIER_OVERFLOW or LLMINT8_ERR_TIMEOUT (timeout
- * wins).  `flags_out` (host, may be NULL) receives the raw bits. */
+ * wins).  `flags_out` (host, may be NULL) receives the raw bits.  After a
+ * timeout the workspace's internal counters may be left non-zero: zero it
+ * (llmint8_workspace_init) before its next use. */
 llmint8_status llmint8_check_status(void* ws, void* stream, uint32_t* flags_out);
 
 /* Test hook for step a5 alone: C[i,j] = sum_k Xq[i,k] * Wq[j,k] as int32,

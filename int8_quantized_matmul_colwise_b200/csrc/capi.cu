@@ -124,6 +124,7 @@ bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t
   off = align_up(off + 4 * size_t((K + 255) / 256), 256);  // block counters follow colmax
   *bitmask = off;
   off = align_up(off + 4 * size_t((K + 31) / 32), 256);
+  off += act_fused_bytes(K);  // the one-kernel activation step's counters and bitmasks
   L->status = 0;
   L->n_outlier = 8;
   L->outlier_idx = off;
@@ -157,6 +158,7 @@ ActWs act_ws(void* ws, size_t colmax_off, size_t bitmask_off, int64_t K) {
   a.colmax = reinterpret_cast<uint32_t*>(b + colmax_off);
   a.blk_counter = reinterpret_cast<uint32_t*>(b + align_up(colmax_off + 4 * size_t(K), 256));
   a.bitmask = reinterpret_cast<uint32_t*>(b + bitmask_off);
+  a.fused = reinterpret_cast<uint32_t*>(b + align_up(bitmask_off + 4 * size_t((K + 31) / 32), 256));
   return a;
 }
 
@@ -245,11 +247,12 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
   size_t colmax, bitmask;
   if (!make_layout(M, K, outlier_cap, &L, &colmax, &bitmask)) return LLMINT8_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return LLMINT8_ERR_WORKSPACE;
-  llmint8_status st = current_device(nullptr);
+  int num_sms = 0;
+  llmint8_status st = current_device(&num_sms);
   if (st != LLMINT8_OK) return st;
   return cuda_status(launch_quantize_act(X, M, K, ldx, tau, Xq, ldq, row_scale, outlier_idx, outlier_cap,
                                          n_outlier, Xo, ldo, act_ws(ws, colmax, bitmask, K),
-                                         static_cast<cudaStream_t>(stream), true));
+                                         static_cast<cudaStream_t>(stream), true, num_sms));
 }
 
 llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
@@ -322,7 +325,7 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
   }
 
   cudaError_t e = launch_quantize_act(X, M, K, ldx, tau, xq, L.ldq, rs, O, outlier_cap, n_o, xo, L.ldo,
-                                      act_ws(ws, colmax_off, bitmask_off, K), s, true);
+                                      act_ws(ws, colmax_off, bitmask_off, K), s, true, num_sms);
   if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
 
   if (decode) {

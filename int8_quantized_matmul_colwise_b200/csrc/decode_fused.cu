@@ -140,31 +140,6 @@ __device__ __noinline__ int outlier_at(int t, const uint32_t* s_mask, const uint
   return lo * 32 + __ffs(bits) - 1;
 }
 
-// Maximum of R per-lane values over `width` lanes (a power of two >= R),
-// halving the vector at each step: after the call the lane holds the maximum
-// of row `row` over its width lanes (lanes that agree on the low bits below
-// width / R hold the same row).
-template <int R>
-__device__ __forceinline__ float rows_max_transposed(float (&v)[R], int width, int lane, int& row) {
-  int o = width >> 1;
-  row = 0;
-#pragma unroll
-  for (int half = R >> 1; half > 0; half >>= 1) {
-    const bool up = (lane & o) != 0;
-#pragma unroll
-    for (int j = 0; j < half; ++j) {
-      const float mine = up ? v[j + half] : v[j];
-      const float other = up ? v[j] : v[j + half];
-      v[j] = fmaxf(mine, __shfl_xor_sync(0xffffffffu, other, o));
-    }
-    row += up ? half : 0;
-    o >>= 1;
-  }
-  float x = v[0];
-  for (; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-  return x;
-}
-
 template <int NP, int R, int MINB>
 __global__ void __launch_bounds__(kThreadsF, MINB)
     decode_fused_kernel(const __grid_constant__ CUtensorMap tmA, const FusedArgs p) {
@@ -664,6 +639,9 @@ cudaError_t launch_fused_variant(const CUtensorMap& tmA, const FusedArgs& a, cud
   const LayoutF lo(NP, a.kb_per, a.stages, (a.K + 31) / 32);
   if (static_cast<int>(lo.total) > smem_set[dev]) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(lo.total));
+    if (e != cudaSuccess) return e;
+    // all of the SM's unified memory as shared memory, so that two CTAs fit
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     smem_set[dev] = static_cast<int>(lo.total);
   }

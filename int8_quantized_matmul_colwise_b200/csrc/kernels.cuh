@@ -14,14 +14,25 @@ struct ActWs {
   uint32_t* blk_counter;  // [ceil(K/256)] scan CTAs finished per column block; zero between calls
   uint32_t* bitmask;      // [ceil(K/32)] outlier flags of this call
   uint32_t* status;       // status word
+  // One-kernel activation step (optional, nullptr: not used): a 64-bit grid
+  // arrival counter followed by two outlier bitmasks of ceil(K/32) words each
+  // (this call ORs into one, zeroes the other for the next call); zero-filled
+  // once with the workspace.
+  uint32_t* fused = nullptr;
 };
+
+// Bytes of ActWs::fused for K columns (256-byte multiple).
+inline size_t act_fused_bytes(int64_t K) { return (16 + 8 * size_t((K + 31) / 32) + 255) / 256 * 256; }
 
 cudaError_t launch_quantize_weight_colwise(const void* W, int64_t K, int64_t N, int64_t ldw, int8_t* Wq,
                                            int64_t ldk, float* col_scale, cudaStream_t stream);
 
+// num_sms > 0 and ws.fused set: shapes whose X fits in shared memory across
+// the SMs run as one persistent kernel (grid barrier between the column scan
+// and the row quantization); otherwise two kernels.
 cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx, float tau, int8_t* Xq,
                                 int64_t ldq, float* rs, int32_t* O, int64_t cap, int32_t* n_out, void* Xo,
-                                int64_t ldo, ActWs ws, cudaStream_t stream, bool pdl);
+                                int64_t ldo, ActWs ws, cudaStream_t stream, bool pdl, int num_sms = 0);
 
 // Everything the GEMM epilogue needs besides the two tensor maps.
 struct GemmArgs {

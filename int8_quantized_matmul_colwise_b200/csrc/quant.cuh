@@ -123,4 +123,29 @@ __device__ __forceinline__ uint2 quantize8(uint4 u, float k, bool& tie_risk) {
   return out;
 }
 
+// Maximum of R per-lane values over `width` lanes (a power of two >= R),
+// halving the vector at each step: after the call the lane holds the maximum
+// of row `row` over its width lanes (lanes that agree on the low bits below
+// width / R hold the same row).
+template <int R>
+__device__ __forceinline__ float rows_max_transposed(float (&v)[R], int width, int lane, int& row) {
+  int o = width >> 1;
+  row = 0;
+#pragma unroll
+  for (int half = R >> 1; half > 0; half >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < half; ++j) {
+      const float mine = up ? v[j + half] : v[j];
+      const float other = up ? v[j] : v[j + half];
+      v[j] = fmaxf(mine, __shfl_xor_sync(0xffffffffu, other, o));
+    }
+    row += up ? half : 0;
+    o >>= 1;
+  }
+  float x = v[0];
+  for (; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
 }  // namespace llmint8

@@ -284,6 +284,258 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_kernel(const __half* __r
   }
 }
 
+// ----------------------------------------------------------------- a1-a4 in one kernel
+// For shapes whose X fits in shared memory spread over the SMs: one CTA per SM
+// (all resident), each holding a block of rows.  Phase 1 bulk-copies the rows
+// into shared memory and ORs the rows' outlier flags (|x| >= tau) into the
+// call's global bitmask, one atomic per non-zero 32-column word; after a grid
+// barrier, phase 2 reads the bitmask and its prefix, and one warp per row takes
+// the row maximum over the non-outlier columns, the codes and the outlier
+// gather straight from shared memory.  X is read from HBM once.
+//
+// ws.fused: word 0 counts the CTAs that reached the grid barrier (the last one
+// returns it to zero), word 1 is the call generation g (the last CTA bumps
+// it, which releases the others), words 4.. hold bitmask buffers 0 and 1 of
+// ceil(K/32) words.  A call of generation g ORs into buffer g & 1 and zeroes
+// buffer (g + 1) & 1, which the previous call used and the next will use.
+constexpr int kActFusedThreads = 512;
+constexpr int kActFusedMaxRows = 16;  // rows per CTA
+constexpr size_t kActFusedSmemMax = 200 * 1024;
+
+__global__ void __launch_bounds__(kActFusedThreads, 2)
+    act_fused_kernel(const __half* __restrict__ X, int64_t M, int64_t K, int64_t ldx, float tau, ActWs ws,
+                     int32_t* __restrict__ O, int32_t* __restrict__ n_out, int64_t cap, int8_t* __restrict__ Xq,
+                     int64_t ldq, float* __restrict__ rs, __half* __restrict__ Xo, int64_t ldo, int rows_per) {
+  extern __shared__ __align__(128) uint8_t smem_a[];
+  const int nwords = static_cast<int>((K + 31) / 32);
+  const int nchunks = static_cast<int>(K / 8);  // K % 8 == 0 on this path
+  __half* s_x = reinterpret_cast<__half*>(smem_a);  // [rows_per][K]
+  uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem_a + size_t(rows_per) * size_t(K) * 2);
+  uint32_t* s_pre = s_mask + nwords;
+  __shared__ uint64_t bar;
+  __shared__ int s_warp[kActFusedThreads / 32];
+  __shared__ uint32_t s_gen;
+  __shared__ uint32_t s_rmax[kActFusedMaxRows];
+  __shared__ float s_k[kActFusedMaxRows];
+  __shared__ float s_inv[kActFusedMaxRows];
+  __shared__ int s_ok;
+
+  const int tid = static_cast<int>(threadIdx.x);
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int64_t r0 = int64_t(blockIdx.x) * rows_per;
+  const int nr = static_cast<int>(min(int64_t(rows_per), M - r0));
+  uint32_t* arrived = ws.fused;
+  uint32_t* generation = ws.fused + 1;
+
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  if (tid < kActFusedMaxRows) s_rmax[tid] = 0u;
+  griddep_wait();  // X may be written by the preceding kernel
+  griddep_launch_dependents();
+  if (tid == 0) {
+    s_gen = ld_acquire_gpu_u32(generation);
+    // phase 1 input: this CTA's rows, one bulk copy each
+    mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nr) * static_cast<uint32_t>(K) * 2u);
+    for (int r = 0; r < nr; ++r)
+      bulk_load_1d(s_x + size_t(r) * size_t(K), X + (r0 + r) * ldx, static_cast<uint32_t>(K) * 2u, &bar);
+  }
+  __syncthreads();
+  const uint32_t gen = s_gen;
+  uint32_t* buf = ws.fused + 4 + (gen & 1u) * uint32_t(nwords);
+  uint32_t* other = ws.fused + 4 + ((gen + 1u) & 1u) * uint32_t(nwords);
+  if (blockIdx.x == 0) {
+    for (int w = tid; w < nwords; w += kActFusedThreads) other[w] = 0u;
+  }
+  const bool loaded = mbar_wait(&bar, 0, ws.status);
+
+  // a1 for this CTA's rows: OR of (|x| >= tau) per column, one word per 4 lanes
+  for (int ch0 = 0; ch0 < nchunks; ch0 += kActFusedThreads) {
+    const int ch = ch0 + tid;
+    uint32_t fl = 0;
+    if (ch < nchunks && loaded) {
+      for (int r = 0; r < nr; ++r) {
+        const uint4 u = *reinterpret_cast<const uint4*>(s_x + size_t(r) * size_t(K) + 8 * ch);
+        const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(__habs2(h2[e]));
+          fl |= (f.x >= tau ? 1u : 0u) << (2 * e);
+          fl |= (f.y >= tau ? 1u : 0u) << (2 * e + 1);
+        }
+      }
+    }
+    uint32_t word = fl << ((8 * ch) & 31);
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    word |= __shfl_xor_sync(0xffffffffu, word, 2);
+    if ((ch & 3) == 0 && ch < nchunks && word != 0u) atomicOr(buf + (ch >> 2), word);
+  }
+
+  // grid barrier (every CTA of the grid is resident: one per SM, at most the
+  // SM count); bounded
+  __syncthreads();
+  if (tid == 0) {
+    int ok = 1;
+    if (atom_add_acq_rel_gpu_u32(arrived, 1u) == gridDim.x - 1u) {
+      *arrived = 0u;                         // for the next call
+      st_release_gpu_u32(generation, gen + 1u);  // releases the others
+    } else {
+      const uint64_t t0 = globaltimer_ns();
+      uint32_t n = 0;
+      while (ld_acquire_gpu_u32(generation) == gen) {
+        if ((++n & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+          atomicOr(ws.status, kStatusTimeout);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    s_ok = ok && loaded;
+  }
+  __syncthreads();
+
+  // phase 2: the call's bitmask and its popcount prefix
+  int cnt = 0;
+  const int wpt = (nwords + kActFusedThreads - 1) / kActFusedThreads;
+  const int w0 = tid * wpt;
+  for (int w = w0; w < w0 + wpt && w < nwords; ++w) {
+    const uint32_t b = __ldcg(buf + w);
+    s_mask[w] = b;
+    cnt += __popc(b);
+  }
+  int x = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  int before = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < kActFusedThreads / 32; ++w) {
+    before += w < warp ? s_warp[w] : 0;
+    total += s_warp[w];
+  }
+  int pos = before + x - cnt;
+  for (int w = w0; w < w0 + wpt && w < nwords; ++w) {
+    s_pre[w] = static_cast<uint32_t>(pos);
+    if (blockIdx.x == 0) {
+      uint32_t bits = s_mask[w];
+      int q = pos;
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (q < cap) O[q] = w * 32 + b;
+        ++q;
+      }
+    }
+    pos += __popc(s_mask[w]);
+  }
+  if (blockIdx.x == 0 && tid == 0) {
+    *n_out = total;
+    if (total > cap) atomicOr(ws.status, kStatusOverflow);
+  }
+  __syncthreads();
+
+  // a2-a4, thread <-> 8-column chunk for all rows of the CTA (as in phase 1):
+  // row maxima over the non-outlier columns (transposed warp reduction, one
+  // shared atomic max per row and warp), then codes and the outlier gather.
+  float pm[kActFusedMaxRows];
+#pragma unroll
+  for (int r = 0; r < kActFusedMaxRows; ++r) pm[r] = 0.0f;
+  for (int ch = tid; ch < nchunks; ch += kActFusedThreads) {
+    const uint32_t fl = (s_mask[ch >> 2] >> ((ch & 3) * 8)) & 0xFFu;
+    const uint32_t k0 = ((fl & 1u) ? 0u : 0xFFFFu) | ((fl & 2u) ? 0u : 0xFFFF0000u);
+    const uint32_t k1 = ((fl & 4u) ? 0u : 0xFFFFu) | ((fl & 8u) ? 0u : 0xFFFF0000u);
+    const uint32_t k2 = ((fl & 16u) ? 0u : 0xFFFFu) | ((fl & 32u) ? 0u : 0xFFFF0000u);
+    const uint32_t k3 = ((fl & 64u) ? 0u : 0xFFFFu) | ((fl & 128u) ? 0u : 0xFFFF0000u);
+#pragma unroll
+    for (int r = 0; r < kActFusedMaxRows; ++r) {
+      if (r < nr) {
+        uint4 u = *reinterpret_cast<const uint4*>(s_x + size_t(r) * size_t(K) + 8 * ch);
+        u.x &= k0;
+        u.y &= k1;
+        u.z &= k2;
+        u.w &= k3;
+        const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+        __half2 m2 = __hmax2(__habs2(h2[0]), __habs2(h2[1]));
+        m2 = __hmax2(m2, __hmax2(__habs2(h2[2]), __habs2(h2[3])));
+        pm[r] = fmaxf(pm[r], fmaxf(__low2float(m2), __high2float(m2)));  // NaN never wins
+      }
+    }
+  }
+  int prow = 0;
+  const float pmax = rows_max_transposed<kActFusedMaxRows>(pm, 32, lane, prow);
+  if ((lane & 1) == 0 && prow < nr) atomicMax(&s_rmax[prow], __float_as_uint(pmax));
+  __syncthreads();
+  if (tid < nr) {
+    const float sc = __uint_as_float(s_rmax[tid]);
+    rs[r0 + tid] = sc;
+    s_k[tid] = sc > 0.0f ? __fdiv_rn(127.0f, sc) : 0.0f;
+    s_inv[tid] = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+  }
+  __syncthreads();
+  if (s_ok) {
+    for (int ch = tid; ch < nchunks; ch += kActFusedThreads) {
+      const uint32_t fl = (s_mask[ch >> 2] >> ((ch & 3) * 8)) & 0xFFu;
+      const uint32_t k0 = ((fl & 1u) ? 0u : 0xFFFFu) | ((fl & 2u) ? 0u : 0xFFFF0000u);
+      const uint32_t k1 = ((fl & 4u) ? 0u : 0xFFFFu) | ((fl & 8u) ? 0u : 0xFFFF0000u);
+      const uint32_t k2 = ((fl & 16u) ? 0u : 0xFFFFu) | ((fl & 32u) ? 0u : 0xFFFF0000u);
+      const uint32_t k3 = ((fl & 64u) ? 0u : 0xFFFFu) | ((fl & 128u) ? 0u : 0xFFFF0000u);
+      uint32_t risk_rows = 0;
+#pragma unroll
+      for (int r = 0; r < kActFusedMaxRows; ++r) {
+        if (r < nr) {
+          uint4 u = *reinterpret_cast<const uint4*>(s_x + size_t(r) * size_t(K) + 8 * ch);
+          u.x &= k0;
+          u.y &= k1;
+          u.z &= k2;
+          u.w &= k3;
+          bool risk = false;
+          const uint2 code = quantize8(u, s_k[r], risk);
+          risk_rows |= static_cast<uint32_t>(risk) << r;
+          *reinterpret_cast<uint2*>(Xq + (r0 + r) * ldq + 8 * ch) = code;
+        }
+      }
+      if (risk_rows != 0u) {  // rare: a value within 2^-15 of a rounding boundary; redo its chunk exactly
+#pragma unroll 1
+        for (int r = 0; r < nr; ++r) {
+          if ((risk_rows >> r) & 1u) {
+            uint4 u = *reinterpret_cast<const uint4*>(s_x + size_t(r) * size_t(K) + 8 * ch);
+            u.x &= k0;
+            u.y &= k1;
+            u.z &= k2;
+            u.w &= k3;
+            *reinterpret_cast<uint2*>(Xq + (r0 + r) * ldq + 8 * ch) = quantize8_exact(u, __uint_as_float(s_rmax[r]), s_inv[r]);
+          }
+        }
+      }
+      if (fl != 0u && Xo != nullptr) {  // a4: gather the outlier values
+        const int b0 = (8 * ch) & 31;
+        const uint32_t wd = s_mask[ch >> 2];
+        const int base = static_cast<int>(s_pre[ch >> 2]);
+#pragma unroll 1
+        for (int e = 0; e < 8; ++e) {
+          if ((fl >> e) & 1u) {
+            const int q = base + __popc(wd & ((1u << (b0 + e)) - 1u));
+            if (q < cap) {
+#pragma unroll 1
+              for (int r = 0; r < nr; ++r) Xo[(r0 + r) * ldo + q] = s_x[size_t(r) * size_t(K) + 8 * ch + e];
+            }
+          }
+        }
+      }
+    }
+    // Xq columns [K, ldq) are zero
+    const int pad = static_cast<int>((ldq - K) / 8);
+    for (int i = tid; i < pad * nr; i += kActFusedThreads)
+      *reinterpret_cast<uint2*>(Xq + (r0 + i / pad) * ldq + K + 8 * (i % pad)) = make_uint2(0u, 0u);
+  }
+}
+
 // Rows too long for the register-resident kernel (K > 16384): one CTA per row,
 // two passes over the row.
 __global__ void __launch_bounds__(256) quantize_rows_long_kernel(const __half* __restrict__ X, int64_t M,
@@ -372,7 +624,7 @@ cudaError_t launch_rows(cudaLaunchConfig_t& cfg, int64_t M, const __half* x, int
 
 cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx, float tau, int8_t* Xq,
                                 int64_t ldq, float* rs, int32_t* O, int64_t cap, int32_t* n_out, void* Xo,
-                                int64_t ldo, ActWs ws, cudaStream_t stream, bool pdl) {
+                                int64_t ldo, ActWs ws, cudaStream_t stream, bool pdl, int num_sms) {
   const __half* x = static_cast<const __half*>(X);
   const bool vec_ok = (ldx % 8 == 0) && (K % 8 == 0) && (reinterpret_cast<uintptr_t>(X) % 16 == 0);
   const size_t mask_bytes = static_cast<size_t>((K + 31) / 32) * sizeof(uint32_t);
@@ -386,6 +638,35 @@ cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx
   cfg.stream = stream;
   cfg.attrs = pdl ? attr : nullptr;
   cfg.numAttrs = pdl ? 1 : 0;
+
+  // One kernel when X fits in shared memory over at most num_sms CTAs.
+  if (ws.fused != nullptr && num_sms > 0 && vec_ok) {
+    const int64_t rows_per = (M + num_sms - 1) / num_sms;
+    const size_t smem = size_t(rows_per) * size_t(K) * 2 + 2 * mask_bytes;
+    if (rows_per <= kActFusedMaxRows && smem <= kActFusedSmemMax) {
+      static int smem_set[64] = {};
+      int dev = 0;
+      cudaError_t e = cudaGetDevice(&dev);
+      if (e != cudaSuccess) return e;
+      if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+      if (static_cast<int>(smem) > smem_set[dev]) {
+        e = cudaFuncSetAttribute(act_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kActFusedSmemMax));
+        if (e != cudaSuccess) return e;
+        // all of the SM's unified memory as shared memory: the next call's
+        // CTAs can then be resident next to this call's
+        e = cudaFuncSetAttribute(act_fused_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        smem_set[dev] = static_cast<int>(kActFusedSmemMax);
+      }
+      cfg.blockDim = dim3(kActFusedThreads);
+      cfg.gridDim = dim3(static_cast<unsigned>((M + rows_per - 1) / rows_per));
+      cfg.dynamicSmemBytes = smem;
+      return cudaLaunchKernelEx(&cfg, act_fused_kernel, x, M, K, ldx, tau, ws, O, n_out, cap, Xq, ldq, rs,
+                                static_cast<__half*>(Xo), ldo, static_cast<int>(rows_per));
+    }
+  }
 
   cfg.gridDim = dim3(static_cast<unsigned>((K + kScanCols - 1) / kScanCols),
                      static_cast<unsigned>((M + kScanRows - 1) / kScanRows));

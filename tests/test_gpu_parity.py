@@ -141,6 +141,34 @@ def test_exact_quantizer_every_fp16_value(L, s):
     check_act(L, X, np.inf)
 
 
+def test_activation_workspace_reuse_across_shapes(L):
+    """One workspace for calls of several row counts (the one-kernel step's
+    grid barrier and its two alternating bitmasks) and for a call whose rows
+    are not 16-byte aligned (the two-kernel step): every call bit-exact."""
+    K, M_max = 512, 300
+    ws = L.empty_workspace(M_max, 1, K, K)
+    rng = np.random.default_rng(31)
+    for M, tau, strided in [(129, 6.0, False), (16, 6.0, False), (300, 3.0, False), (40, 6.0, True),
+                            (129, 6.0, False), (1, 0.0, False), (129, np.inf, False)]:
+        X, _, _ = wl.random_small(rng, M, K, 1, 3)
+        if strided:
+            wide = np.zeros((M, K + 1), np.float16)
+            wide[:, :K] = X
+            Xd = dev(wide)[:, :K]
+        else:
+            Xd = dev(X)
+        out = L.quantize_act_rowwise_outliers(Xd, tau, ws=ws)
+        O, rs, Xq = oracle.quantize_activation(X, tau)
+        n = int(host(out["n_outlier"])[0])
+        assert n == O.size
+        assert np.array_equal(host(out["outlier_idx"])[:n], O)
+        assert np.array_equal(host(out["row_scale"]), rs)
+        assert np.array_equal(host(out["Xq"])[:, :K], Xq)
+        Xo_ref, _ = oracle.gather_outliers(X, O)
+        assert np.array_equal(host(out["Xo"])[:, :n].view(np.uint16), Xo_ref.view(np.uint16))
+    assert_status_ok(L, ws)
+
+
 def test_activation_strided_rows(L):
     X = wl.make_x(wl.get("tiny"))
     wide = np.zeros((X.shape[0], X.shape[1] + 40), np.float16)
