@@ -286,45 +286,56 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_kernel(const __half* __r
 
 // ----------------------------------------------------------------- a1-a4 in one kernel
 // For shapes whose X fits in shared memory spread over the SMs: one CTA per SM
-// (all resident), each holding a block of rows.  Phase 1 bulk-copies the rows
-// into shared memory and ORs the rows' outlier flags (|x| >= tau) into the
-// call's global bitmask, one atomic per non-zero 32-column word; after a grid
-// barrier, phase 2 reads the bitmask and its prefix, and one warp per row takes
-// the row maximum over the non-outlier columns, the codes and the outlier
-// gather straight from shared memory.  X is read from HBM once.
+// (all resident), each holding a block of rows.  The CTA bulk-copies its rows
+// into shared memory; thread t then holds R of those rows for one 8-column
+// chunk in registers for the whole kernel (chunks padded to a multiple of 32
+// so that a warp never straddles two row groups).  Phase 1 ORs the rows'
+// outlier flags (column maxima >= tau) into the call's global bitmask, one
+// atomic per non-zero 32-column word; after a grid barrier, phase 2 reads the
+// call's bitmask and its prefix, gathers the outlier values, zeroes them, takes
+// the row maxima (transposed warp reduction, one shared atomic max per row and
+// warp) and writes the codes.  X is read from HBM once.
 //
 // ws.fused: word 0 counts the CTAs that reached the grid barrier (the last one
 // returns it to zero), word 1 is the call generation g (the last CTA bumps
 // it, which releases the others), words 4.. hold bitmask buffers 0 and 1 of
 // ceil(K/32) words.  A call of generation g ORs into buffer g & 1 and zeroes
 // buffer (g + 1) & 1, which the previous call used and the next will use.
-constexpr int kActFusedThreads = 512;
+constexpr int kActFusedThreads = 1024;
 constexpr int kActFusedMaxRows = 16;  // rows per CTA
 constexpr size_t kActFusedSmemMax = 200 * 1024;
 
-__global__ void __launch_bounds__(kActFusedThreads, 2)
+template <int R>
+__global__ void __launch_bounds__(kActFusedThreads, 1)
     act_fused_kernel(const __half* __restrict__ X, int64_t M, int64_t K, int64_t ldx, float tau, ActWs ws,
                      int32_t* __restrict__ O, int32_t* __restrict__ n_out, int64_t cap, int8_t* __restrict__ Xq,
-                     int64_t ldq, float* __restrict__ rs, __half* __restrict__ Xo, int64_t ldo, int rows_per) {
+                     int64_t ldq, float* __restrict__ rs, __half* __restrict__ Xo, int64_t ldo, int rows_per,
+                     int cpad) {
   extern __shared__ __align__(128) uint8_t smem_a[];
   const int nwords = static_cast<int>((K + 31) / 32);
   const int nchunks = static_cast<int>(K / 8);  // K % 8 == 0 on this path
   __half* s_x = reinterpret_cast<__half*>(smem_a);  // [rows_per][K]
   uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem_a + size_t(rows_per) * size_t(K) * 2);
-  uint32_t* s_pre = s_mask + nwords;
+  uint32_t* s_pre = s_mask + ((nwords + 3) & ~3);
+  uint4* s_cm = reinterpret_cast<uint4*>(s_pre + ((nwords + 3) & ~3));  // [kActFusedThreads] column maxima
   __shared__ uint64_t bar;
   __shared__ int s_warp[kActFusedThreads / 32];
   __shared__ uint32_t s_gen;
+  __shared__ int s_ok;
   __shared__ uint32_t s_rmax[kActFusedMaxRows];
   __shared__ float s_k[kActFusedMaxRows];
   __shared__ float s_inv[kActFusedMaxRows];
-  __shared__ int s_ok;
 
   const int tid = static_cast<int>(threadIdx.x);
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int64_t r0 = int64_t(blockIdx.x) * rows_per;
   const int nr = static_cast<int>(min(int64_t(rows_per), M - r0));
+  const int groups = kActFusedThreads / cpad;  // row groups; the host's plan gives R * groups >= rows_per
+  const int cc = tid % cpad;                    // this thread's chunk
+  const int g = tid / cpad;
+  const bool col_ok = cc < nchunks && g < groups;
+  const int m0 = g * R;                         // its first row (of the CTA's)
   uint32_t* arrived = ws.fused;
   uint32_t* generation = ws.fused + 1;
 
@@ -337,7 +348,7 @@ __global__ void __launch_bounds__(kActFusedThreads, 2)
   griddep_launch_dependents();
   if (tid == 0) {
     s_gen = ld_acquire_gpu_u32(generation);
-    // phase 1 input: this CTA's rows, one bulk copy each
+    // this CTA's rows, one bulk copy each
     mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nr) * static_cast<uint32_t>(K) * 2u);
     for (int r = 0; r < nr; ++r)
       bulk_load_1d(s_x + size_t(r) * size_t(K), X + (r0 + r) * ldx, static_cast<uint32_t>(K) * 2u, &bar);
@@ -351,35 +362,53 @@ __global__ void __launch_bounds__(kActFusedThreads, 2)
   }
   const bool loaded = mbar_wait(&bar, 0, ws.status);
 
-  // a1 for this CTA's rows: OR of (|x| >= tau) per column, one word per 4 lanes
-  for (int ch0 = 0; ch0 < nchunks; ch0 += kActFusedThreads) {
-    const int ch = ch0 + tid;
-    uint32_t fl = 0;
-    if (ch < nchunks && loaded) {
-      for (int r = 0; r < nr; ++r) {
-        const uint4 u = *reinterpret_cast<const uint4*>(s_x + size_t(r) * size_t(K) + 8 * ch);
-        const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+  // this thread's rows of its chunk, kept in registers to the end
+  uint4 h[R];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(__habs2(h2[e]));
-          fl |= (f.x >= tau ? 1u : 0u) << (2 * e);
-          fl |= (f.y >= tau ? 1u : 0u) << (2 * e + 1);
-        }
-      }
-    }
-    uint32_t word = fl << ((8 * ch) & 31);
-    word |= __shfl_xor_sync(0xffffffffu, word, 1);
-    word |= __shfl_xor_sync(0xffffffffu, word, 2);
-    if ((ch & 3) == 0 && ch < nchunks && word != 0u) atomicOr(buf + (ch >> 2), word);
-  }
+  for (int r = 0; r < R; ++r)
+    h[r] = (loaded && col_ok && m0 + r < nr) ? *reinterpret_cast<const uint4*>(s_x + size_t(m0 + r) * size_t(K) + 8 * cc)
+                                             : make_uint4(0u, 0u, 0u, 0u);
 
-  // grid barrier (every CTA of the grid is resident: one per SM, at most the
-  // SM count); bounded
+  // a1 (this CTA's rows): column maxima, then over the row groups
+  __half2 cm[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) cm[e] = __half2half2(__ushort_as_half(0));
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const __half2* h2 = reinterpret_cast<const __half2*>(&h[r]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) cm[e] = __hmax2(cm[e], __habs2(h2[e]));  // NaN never wins
+  }
+  if (groups > 1) {
+    s_cm[tid] = *reinterpret_cast<const uint4*>(cm);
+    __syncthreads();
+    for (int gg = 0; gg < groups; ++gg) {
+      const uint4 o = s_cm[gg * cpad + cc];
+      const __half2* o2 = reinterpret_cast<const __half2*>(&o);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cm[e] = __hmax2(cm[e], o2[e]);
+    }
+  }
+  uint32_t fl = 0;
+  if (col_ok) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(cm[e]);
+      fl |= (f.x >= tau ? 1u : 0u) << (2 * e);
+      fl |= (f.y >= tau ? 1u : 0u) << (2 * e + 1);
+    }
+  }
+  uint32_t word = fl << ((8 * cc) & 31);
+  word |= __shfl_xor_sync(0xffffffffu, word, 1);
+  word |= __shfl_xor_sync(0xffffffffu, word, 2);
+  if (g == 0 && col_ok && (cc & 3) == 0 && word != 0u) atomicOr(buf + (cc >> 2), word);
+
+  // grid barrier (every CTA of the grid is resident: at most one per SM); bounded
   __syncthreads();
   if (tid == 0) {
     int ok = 1;
     if (atom_add_acq_rel_gpu_u32(arrived, 1u) == gridDim.x - 1u) {
-      *arrived = 0u;                         // for the next call
+      *arrived = 0u;                             // for the next call
       st_release_gpu_u32(generation, gen + 1u);  // releases the others
     } else {
       const uint64_t t0 = globaltimer_ns();
@@ -401,9 +430,9 @@ __global__ void __launch_bounds__(kActFusedThreads, 2)
   const int wpt = (nwords + kActFusedThreads - 1) / kActFusedThreads;
   const int w0 = tid * wpt;
   for (int w = w0; w < w0 + wpt && w < nwords; ++w) {
-    const uint32_t b = __ldcg(buf + w);
-    s_mask[w] = b;
-    cnt += __popc(b);
+    const uint32_t bw = __ldcg(buf + w);
+    s_mask[w] = bw;
+    cnt += __popc(bw);
   }
   int x = cnt;
 #pragma unroll
@@ -426,9 +455,9 @@ __global__ void __launch_bounds__(kActFusedThreads, 2)
       uint32_t bits = s_mask[w];
       int q = pos;
       while (bits) {
-        const int b = __ffs(bits) - 1;
+        const int bb = __ffs(bits) - 1;
         bits &= bits - 1;
-        if (q < cap) O[q] = w * 32 + b;
+        if (q < cap) O[q] = w * 32 + bb;
         ++q;
       }
     }
@@ -440,36 +469,49 @@ __global__ void __launch_bounds__(kActFusedThreads, 2)
   }
   __syncthreads();
 
-  // a2-a4, thread <-> 8-column chunk for all rows of the CTA (as in phase 1):
-  // row maxima over the non-outlier columns (transposed warp reduction, one
-  // shared atomic max per row and warp), then codes and the outlier gather.
-  float pm[kActFusedMaxRows];
+  // a4: gather this thread's outlier values; then zero them (0 quantizes to 0)
+  const uint32_t gfl = col_ok ? (s_mask[cc >> 2] >> ((cc & 3) * 8)) & 0xFFu : 0u;
+  if (gfl != 0u) {
+    if (Xo != nullptr) {
+      const int b0 = (8 * cc) & 31;
+      const uint32_t wd = s_mask[cc >> 2];
+      const int base = static_cast<int>(s_pre[cc >> 2]);
+#pragma unroll 1
+      for (int e = 0; e < 8; ++e) {
+        if ((gfl >> e) & 1u) {
+          const int q = base + __popc(wd & ((1u << (b0 + e)) - 1u));
+          if (q < cap) {
 #pragma unroll
-  for (int r = 0; r < kActFusedMaxRows; ++r) pm[r] = 0.0f;
-  for (int ch = tid; ch < nchunks; ch += kActFusedThreads) {
-    const uint32_t fl = (s_mask[ch >> 2] >> ((ch & 3) * 8)) & 0xFFu;
-    const uint32_t k0 = ((fl & 1u) ? 0u : 0xFFFFu) | ((fl & 2u) ? 0u : 0xFFFF0000u);
-    const uint32_t k1 = ((fl & 4u) ? 0u : 0xFFFFu) | ((fl & 8u) ? 0u : 0xFFFF0000u);
-    const uint32_t k2 = ((fl & 16u) ? 0u : 0xFFFFu) | ((fl & 32u) ? 0u : 0xFFFF0000u);
-    const uint32_t k3 = ((fl & 64u) ? 0u : 0xFFFFu) | ((fl & 128u) ? 0u : 0xFFFF0000u);
-#pragma unroll
-    for (int r = 0; r < kActFusedMaxRows; ++r) {
-      if (r < nr) {
-        uint4 u = *reinterpret_cast<const uint4*>(s_x + size_t(r) * size_t(K) + 8 * ch);
-        u.x &= k0;
-        u.y &= k1;
-        u.z &= k2;
-        u.w &= k3;
-        const __half2* h2 = reinterpret_cast<const __half2*>(&u);
-        __half2 m2 = __hmax2(__habs2(h2[0]), __habs2(h2[1]));
-        m2 = __hmax2(m2, __hmax2(__habs2(h2[2]), __habs2(h2[3])));
-        pm[r] = fmaxf(pm[r], fmaxf(__low2float(m2), __high2float(m2)));  // NaN never wins
+            for (int r = 0; r < R; ++r)
+              if (m0 + r < nr) Xo[(r0 + m0 + r) * ldo + q] = __ushort_as_half(half_bits_at(h[r], e));
+          }
+        }
       }
     }
+    const uint32_t k0 = ((gfl & 1u) ? 0u : 0xFFFFu) | ((gfl & 2u) ? 0u : 0xFFFF0000u);
+    const uint32_t k1 = ((gfl & 4u) ? 0u : 0xFFFFu) | ((gfl & 8u) ? 0u : 0xFFFF0000u);
+    const uint32_t k2 = ((gfl & 16u) ? 0u : 0xFFFFu) | ((gfl & 32u) ? 0u : 0xFFFF0000u);
+    const uint32_t k3 = ((gfl & 64u) ? 0u : 0xFFFFu) | ((gfl & 128u) ? 0u : 0xFFFF0000u);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      h[r].x &= k0;
+      h[r].y &= k1;
+      h[r].z &= k2;
+      h[r].w &= k3;
+    }
+  }
+
+  // a2: row maxima over the non-outlier columns
+  float pm[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const __half2* h2 = reinterpret_cast<const __half2*>(&h[r]);
+    const __half2 m2 = __hmax2(__hmax2(__habs2(h2[0]), __habs2(h2[1])), __hmax2(__habs2(h2[2]), __habs2(h2[3])));
+    pm[r] = fmaxf(__low2float(m2), __high2float(m2));
   }
   int prow = 0;
-  const float pmax = rows_max_transposed<kActFusedMaxRows>(pm, 32, lane, prow);
-  if ((lane & 1) == 0 && prow < nr) atomicMax(&s_rmax[prow], __float_as_uint(pmax));
+  const float pmax = rows_max_transposed<R>(pm, 32, lane, prow);
+  if ((lane & (32 / R - 1)) == 0 && g < groups && m0 + prow < nr) atomicMax(&s_rmax[m0 + prow], __float_as_uint(pmax));
   __syncthreads();
   if (tid < nr) {
     const float sc = __uint_as_float(s_rmax[tid]);
@@ -478,58 +520,31 @@ __global__ void __launch_bounds__(kActFusedThreads, 2)
     s_inv[tid] = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
   }
   __syncthreads();
-  if (s_ok) {
-    for (int ch = tid; ch < nchunks; ch += kActFusedThreads) {
-      const uint32_t fl = (s_mask[ch >> 2] >> ((ch & 3) * 8)) & 0xFFu;
-      const uint32_t k0 = ((fl & 1u) ? 0u : 0xFFFFu) | ((fl & 2u) ? 0u : 0xFFFF0000u);
-      const uint32_t k1 = ((fl & 4u) ? 0u : 0xFFFFu) | ((fl & 8u) ? 0u : 0xFFFF0000u);
-      const uint32_t k2 = ((fl & 16u) ? 0u : 0xFFFFu) | ((fl & 32u) ? 0u : 0xFFFF0000u);
-      const uint32_t k3 = ((fl & 64u) ? 0u : 0xFFFFu) | ((fl & 128u) ? 0u : 0xFFFF0000u);
-      uint32_t risk_rows = 0;
+
+  // a3: codes
+  if (s_ok && col_ok) {
+    int8_t* q = Xq + (r0 + m0) * ldq + 8 * cc;
+    uint32_t risk_rows = 0;
 #pragma unroll
-      for (int r = 0; r < kActFusedMaxRows; ++r) {
-        if (r < nr) {
-          uint4 u = *reinterpret_cast<const uint4*>(s_x + size_t(r) * size_t(K) + 8 * ch);
-          u.x &= k0;
-          u.y &= k1;
-          u.z &= k2;
-          u.w &= k3;
-          bool risk = false;
-          const uint2 code = quantize8(u, s_k[r], risk);
-          risk_rows |= static_cast<uint32_t>(risk) << r;
-          *reinterpret_cast<uint2*>(Xq + (r0 + r) * ldq + 8 * ch) = code;
-        }
+    for (int r = 0; r < R; ++r) {
+      if (m0 + r < nr) {
+        bool risk = false;
+        const uint2 code = quantize8(h[r], s_k[m0 + r], risk);
+        risk_rows |= static_cast<uint32_t>(risk) << r;
+        *reinterpret_cast<uint2*>(q) = code;
       }
-      if (risk_rows != 0u) {  // rare: a value within 2^-15 of a rounding boundary; redo its chunk exactly
-#pragma unroll 1
-        for (int r = 0; r < nr; ++r) {
-          if ((risk_rows >> r) & 1u) {
-            uint4 u = *reinterpret_cast<const uint4*>(s_x + size_t(r) * size_t(K) + 8 * ch);
-            u.x &= k0;
-            u.y &= k1;
-            u.z &= k2;
-            u.w &= k3;
-            *reinterpret_cast<uint2*>(Xq + (r0 + r) * ldq + 8 * ch) = quantize8_exact(u, __uint_as_float(s_rmax[r]), s_inv[r]);
-          }
-        }
-      }
-      if (fl != 0u && Xo != nullptr) {  // a4: gather the outlier values
-        const int b0 = (8 * ch) & 31;
-        const uint32_t wd = s_mask[ch >> 2];
-        const int base = static_cast<int>(s_pre[ch >> 2]);
-#pragma unroll 1
-        for (int e = 0; e < 8; ++e) {
-          if ((fl >> e) & 1u) {
-            const int q = base + __popc(wd & ((1u << (b0 + e)) - 1u));
-            if (q < cap) {
-#pragma unroll 1
-              for (int r = 0; r < nr; ++r) Xo[(r0 + r) * ldo + q] = s_x[size_t(r) * size_t(K) + 8 * ch + e];
-            }
-          }
-        }
-      }
+      q += ldq;
     }
-    // Xq columns [K, ldq) are zero
+    if (risk_rows != 0u) {  // rare: a value within 2^-15 of a rounding boundary; redo its chunk exactly
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        if ((risk_rows >> r) & 1u)
+          *reinterpret_cast<uint2*>(Xq + (r0 + m0 + r) * ldq + 8 * cc) =
+              quantize8_exact(h[r], __uint_as_float(s_rmax[m0 + r]), s_inv[m0 + r]);
+    }
+  }
+  // Xq columns [K, ldq) are zero
+  if (s_ok) {
     const int pad = static_cast<int>((ldq - K) / 8);
     for (int i = tid; i < pad * nr; i += kActFusedThreads)
       *reinterpret_cast<uint2*>(Xq + (r0 + i / pad) * ldq + K + 8 * (i % pad)) = make_uint2(0u, 0u);
@@ -642,29 +657,31 @@ cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx
   // One kernel when X fits in shared memory over at most num_sms CTAs.
   if (ws.fused != nullptr && num_sms > 0 && vec_ok) {
     const int64_t rows_per = (M + num_sms - 1) / num_sms;
-    const size_t smem = size_t(rows_per) * size_t(K) * 2 + 2 * mask_bytes;
-    if (rows_per <= kActFusedMaxRows && smem <= kActFusedSmemMax) {
-      static int smem_set[64] = {};
+    const int64_t cpad = ((K / 8) + 31) / 32 * 32;  // chunks padded to whole warps
+    const int64_t groups = cpad <= kActFusedThreads ? kActFusedThreads / cpad : 0;
+    const int64_t r = groups > 0 ? (rows_per + groups - 1) / groups : 0;
+    const size_t smem = size_t(rows_per) * size_t(K) * 2 + 2 * ((mask_bytes + 15) / 16 * 16) +
+                        size_t(kActFusedThreads) * 16;
+    if (groups > 0 && r <= 8 && rows_per <= kActFusedMaxRows && smem <= kActFusedSmemMax) {
+      const int rt = r <= 1 ? 1 : r <= 2 ? 2 : r <= 4 ? 4 : 8;
+      auto kern = rt == 1 ? act_fused_kernel<1> : rt == 2 ? act_fused_kernel<2> : rt == 4 ? act_fused_kernel<4>
+                                                                                            : act_fused_kernel<8>;
+      static bool attr_set[4][64] = {};
+      const int ri = rt == 1 ? 0 : rt == 2 ? 1 : rt == 4 ? 2 : 3;
       int dev = 0;
       cudaError_t e = cudaGetDevice(&dev);
       if (e != cudaSuccess) return e;
       if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-      if (static_cast<int>(smem) > smem_set[dev]) {
-        e = cudaFuncSetAttribute(act_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kActFusedSmemMax));
+      if (!attr_set[ri][dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kActFusedSmemMax));
         if (e != cudaSuccess) return e;
-        // all of the SM's unified memory as shared memory: the next call's
-        // CTAs can then be resident next to this call's
-        e = cudaFuncSetAttribute(act_fused_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        smem_set[dev] = static_cast<int>(kActFusedSmemMax);
+        attr_set[ri][dev] = true;
       }
       cfg.blockDim = dim3(kActFusedThreads);
       cfg.gridDim = dim3(static_cast<unsigned>((M + rows_per - 1) / rows_per));
       cfg.dynamicSmemBytes = smem;
-      return cudaLaunchKernelEx(&cfg, act_fused_kernel, x, M, K, ldx, tau, ws, O, n_out, cap, Xq, ldq, rs,
-                                static_cast<__half*>(Xo), ldo, static_cast<int>(rows_per));
+      return cudaLaunchKernelEx(&cfg, kern, x, M, K, ldx, tau, ws, O, n_out, cap, Xq, ldq, rs,
+                                static_cast<__half*>(Xo), ldo, static_cast<int>(rows_per), static_cast<int>(cpad));
     }
   }
 
