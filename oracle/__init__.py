@@ -61,6 +61,7 @@ def _load():
             "oracle_gather_outliers": (None, [P, I64, I64, P, I64, P, P, I64, P]),
             "oracle_int8_matmul": (None, [P, P, I64, I64, P, I64, P]),
             "oracle_mixed_output": (None, [P, P, P, P, I64, P, I64, P, I64, P, I64, P, P]),
+            "oracle_dequantize_weight": (None, [P, I64, I64, P, P]),
             "oracle_num_threads": (ctypes.c_int, []),
         }
         for name, (res, args) in sig.items():
@@ -204,6 +205,16 @@ def mixed_output(acc: np.ndarray, rs: np.ndarray, cs: np.ndarray, X: np.ndarray,
     return Y.view(np.float16), Yd
 
 
+def dequantize_weight(Wq: np.ndarray, cs: np.ndarray) -> np.ndarray:
+    """fp16 [K, N]: the weight recovered from its int8 form, Wq * cs / 127
+    rounded once to fp16 (the outlier rows when no fp16 weight is kept)."""
+    Wq = _c(Wq, np.int8)
+    K, N = Wq.shape
+    out = np.empty((K, N), np.uint16)
+    _load().oracle_dequantize_weight(_p(Wq), K, N, _p(_c(cs, np.float32)), _p(out))
+    return out.view(np.float16)
+
+
 def quantize_weight(W: np.ndarray):
     """a0 as one call: (Wq [K, N] int8, cs [N] fp32)."""
     cs = col_scales(W)
@@ -218,15 +229,18 @@ def quantize_activation(X: np.ndarray, tau: float):
 
 
 def mixed_matmul(X: np.ndarray, W: np.ndarray, tau: float, rows: Optional[np.ndarray] = None,
-                 weight: Optional[tuple] = None) -> Dict[str, np.ndarray]:
+                 weight: Optional[tuple] = None, int8_weight: bool = False) -> Dict[str, np.ndarray]:
     """The whole path a0..a7; returns every intermediate.
 
     ``rows`` restricts a5-a7 to those rows (a1 still scans all rows, as the
-    definition requires).  ``weight`` may pass a precomputed (Wq, cs)."""
+    definition requires).  ``weight`` may pass a precomputed (Wq, cs).
+    ``int8_weight``: the outlier product uses the weight recovered from its
+    int8 form (dequantize_weight) instead of the fp16 W."""
     Wq, cs = quantize_weight(W) if weight is None else weight
     O, rs, Xq = quantize_activation(X, tau)
     acc = int8_matmul(Xq, Wq, rows)
-    Y, Yd = mixed_output(acc, rs, cs, X, W, O, rows)
+    Wout = dequantize_weight(Wq, cs) if int8_weight else W
+    Y, Yd = mixed_output(acc, rs, cs, X, Wout, O, rows)
     return {"O": O, "rs": rs, "Xq": Xq, "Wq": Wq, "cs": cs, "acc": acc, "Y": Y, "Yd": Yd}
 
 

@@ -305,6 +305,24 @@ void oracle_mixed_output(const int64_t* acc, const float* rs, const float* cs, c
     }
 }
 
+/* ------------------------------------------------------------------ */
+/* The 16-bit weight rows recovered from the int8 weight, for callers     */
+/* that keep only the int8 form: the point of the method is halving the   */
+/* weight memory ("LLM.int8()" arXiv abstract: inference memory cut by    */
+/* half; "What is 8-bit LLM quantization?", How much memory can it save:  */
+/* 14 GB of fp16 weights become 7 GB of int8).  Each value is the         */
+/* column's dequantized code, Wq * cs / 127, rounded once to fp16.        */
+/* ------------------------------------------------------------------ */
+
+/* Wd[k,j] = fp16_RNE(Wq[k,j] * cs[j] / 127), evaluated in double. */
+void oracle_dequantize_weight(const int8_t* Wq, int64_t K, int64_t N, const float* cs, uint16_t* Wd)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k < K; ++k)
+        for (int64_t j = 0; j < N; ++j)
+            Wd[k * N + j] = oracle_double_to_half((double)Wq[k * N + j] * (double)cs[j] / 127.0);
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

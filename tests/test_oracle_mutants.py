@@ -26,6 +26,8 @@ MUTANTS = {
     "outlier_columns_not_zeroed": ("Xq[i * K + k] = mask[k] ? 0 :", "Xq[i * K + k] ="),
     "row_scale_wrong_index": ("(double)rs[i] * (double)cs[j]", "(double)rs[r] * (double)cs[j]"),
     "codec_ties_to_odd": ("fmod(r, 2.0) != 0.0", "fmod(r, 2.0) == 0.0"),
+    "dequantized_weight_scale_128": ("(double)Wq[k * N + j] * (double)cs[j] / 127.0",
+                                     "(double)Wq[k * N + j] * (double)cs[j] / 128.0"),
     "weight_scale_first_rows_only": ("for (int64_t k = 0; k < K; ++k) {\n            float a = fabsf(half_to_float(W[k * N + j]));",
                                      "for (int64_t k = 0; k < (K + 1) / 2; ++k) {\n            float a = fabsf(half_to_float(W[k * N + j]));"),
 }

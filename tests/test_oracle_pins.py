@@ -358,3 +358,58 @@ def test_chunked_weight_draw_equals_single_draw():
     rng = np.random.default_rng(w.seed + 100)
     b = (rng.standard_normal((37, 29), dtype=np.float32) * np.float32(w.w_sigma)).astype(np.float16)
     assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
+# ------------------------------------------------------------------ int8-only weights
+# The outlier product may use the weight recovered from its int8 form
+# (Wq * cs / 127, rounded once to fp16) instead of a kept fp16 copy.
+
+def _ulp16(v: np.ndarray) -> np.ndarray:
+    """Spacing of fp16 values at magnitude v (normal or subnormal)."""
+    v = np.maximum(np.abs(v.astype(np.float64)), 2.0 ** -14)
+    return 2.0 ** (np.floor(np.log2(v)) - 10)
+
+
+@pytest.mark.parametrize("name,X,W", _problems())
+def test_dequantized_weight_within_half_step(name, X, W):
+    """|Wd - W| <= cs/254 (the codes' rounding) + half an fp16 ulp at cs (the
+    one fp16 rounding); |Wd| <= cs and Wd has the sign of its code."""
+    Wq, cs = oracle.quantize_weight(W)
+    Wd = oracle.dequantize_weight(Wq, cs).astype(np.float64)
+    c = cs.astype(np.float64)[None, :]
+    assert np.all(np.abs(Wd - W.astype(np.float64)) <= c / 254 + _ulp16(c) / 2)
+    assert np.all(np.abs(Wd) <= c)
+    assert np.all(np.sign(Wd) == np.sign(Wq))
+
+
+def test_dequantized_weight_is_exact_on_code_valued_weights():
+    """W = q * 2^-j with a +-127 * 2^-j entry in every column: cs = 127 * 2^-j,
+    the codes are q and the recovered weight is W itself, so the int8-only
+    outlier product equals the fp16 one bit for bit."""
+    rng = np.random.default_rng(41)
+    K, N = 96, 40
+    q = rng.integers(-127, 128, (K, N))
+    q[rng.integers(0, K, N), np.arange(N)] = rng.choice([-127, 127], N)
+    for j in (0, 3, 7):
+        W = (q * 2.0 ** -j).astype(np.float16)
+        Wq, cs = oracle.quantize_weight(W)
+        assert np.array_equal(Wq.astype(np.int64), q)
+        Wd = oracle.dequantize_weight(Wq, cs)
+        assert np.array_equal(Wd.view(np.uint16), W.view(np.uint16))
+        X, _, _ = wl.random_small(rng, 9, K, 1, 4)
+        a = oracle.mixed_matmul(X, W, 6.0)
+        b = oracle.mixed_matmul(X, W, 6.0, int8_weight=True)
+        assert a["O"].size > 0
+        assert np.array_equal(a["Y"].view(np.uint16), b["Y"].view(np.uint16))
+
+
+@pytest.mark.parametrize("name,X,W", _problems())
+def test_int8_weight_reading_at_tau_limits(name, X, W):
+    """tau = +inf: no outlier product, both readings give the same Y; tau = 0:
+    Y is the fp16 matmul of X with the recovered weight."""
+    a = oracle.mixed_matmul(X, W, np.inf)
+    b = oracle.mixed_matmul(X, W, np.inf, int8_weight=True)
+    assert np.array_equal(a["Y"].view(np.uint16), b["Y"].view(np.uint16))
+    r = oracle.mixed_matmul(X, W, 0.0, int8_weight=True)
+    Wd = oracle.dequantize_weight(*oracle.quantize_weight(W)).astype(np.float64)
+    assert np.allclose(r["Yd"], X.astype(np.float64) @ Wd, rtol=1e-12, atol=1e-12)
