@@ -60,7 +60,7 @@ def _load():
             "oracle_quantize_cols": (None, [P, I64, I64, P, P]),
             "oracle_gather_outliers": (None, [P, I64, I64, P, I64, P, P, I64, P]),
             "oracle_int8_matmul": (None, [P, P, I64, I64, P, I64, P]),
-            "oracle_mixed_output": (None, [P, P, P, P, I64, P, I64, P, I64, P, I64, P, P]),
+            "oracle_mixed_output": (None, [P, P, P, P, I64, P, I64, P, I64, P, P, I64, P, P]),
             "oracle_dequantize_weight": (None, [P, I64, I64, P, P]),
             "oracle_num_threads": (ctypes.c_int, []),
         }
@@ -187,8 +187,8 @@ def int8_matmul(Xq: np.ndarray, Wq: np.ndarray, rows: Optional[np.ndarray] = Non
 
 
 def mixed_output(acc: np.ndarray, rs: np.ndarray, cs: np.ndarray, X: np.ndarray, W: np.ndarray,
-                 O: np.ndarray, rows: Optional[np.ndarray] = None):
-    """a6+a7: (Y fp16, Yd float64) for the selected rows."""
+                 O: np.ndarray, rows: Optional[np.ndarray] = None, bias: Optional[np.ndarray] = None):
+    """a6+a7: (Y fp16, Yd float64) for the selected rows; optional fp16 bias [N]."""
     acc = _c(acc, np.int64)
     Xb = _bits16(X)
     Wb = _bits16(W)
@@ -200,8 +200,9 @@ def mixed_output(acc: np.ndarray, rs: np.ndarray, cs: np.ndarray, X: np.ndarray,
     assert acc.shape == (n, N)
     Yd = np.empty((n, N), np.float64)
     Y = np.empty((n, N), np.uint16)
+    bb = None if bias is None else _bits16(np.asarray(bias, np.float16).reshape(N))
     _load().oracle_mixed_output(_p(acc), _p(_c(rs, np.float32)), _p(_c(cs, np.float32)), _p(Xb), K,
-                                _p(Wb), N, _p(O), O.size, _p(rr), n, _p(Yd), _p(Y))
+                                _p(Wb), N, _p(O), O.size, _p(bb), _p(rr), n, _p(Yd), _p(Y))
     return Y.view(np.float16), Yd
 
 
@@ -229,18 +230,20 @@ def quantize_activation(X: np.ndarray, tau: float):
 
 
 def mixed_matmul(X: np.ndarray, W: np.ndarray, tau: float, rows: Optional[np.ndarray] = None,
-                 weight: Optional[tuple] = None, int8_weight: bool = False) -> Dict[str, np.ndarray]:
+                 weight: Optional[tuple] = None, int8_weight: bool = False,
+                 bias: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """The whole path a0..a7; returns every intermediate.
 
     ``rows`` restricts a5-a7 to those rows (a1 still scans all rows, as the
     definition requires).  ``weight`` may pass a precomputed (Wq, cs).
     ``int8_weight``: the outlier product uses the weight recovered from its
-    int8 form (dequantize_weight) instead of the fp16 W."""
+    int8 form (dequantize_weight) instead of the fp16 W.  ``bias``: fp16 [N]
+    added to every row (a linear layer's X W + b)."""
     Wq, cs = quantize_weight(W) if weight is None else weight
     O, rs, Xq = quantize_activation(X, tau)
     acc = int8_matmul(Xq, Wq, rows)
     Wout = dequantize_weight(Wq, cs) if int8_weight else W
-    Y, Yd = mixed_output(acc, rs, cs, X, Wout, O, rows)
+    Y, Yd = mixed_output(acc, rs, cs, X, Wout, O, rows, bias)
     return {"O": O, "rs": rs, "Xq": Xq, "Wq": Wq, "cs": cs, "acc": acc, "Y": Y, "Yd": Yd}
 
 

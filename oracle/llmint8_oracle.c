@@ -281,12 +281,15 @@ void oracle_int8_matmul(const int8_t* Xq, const int8_t* Wq, int64_t N, int64_t K
 /* ------------------------------------------------------------------ */
 
 /* For each selected row i = rows[r]:
- *   Yd[r,j] = acc[r,j] * rs[i] * cs[j] / 127^2 + sum_t X[i,O[t]] * W[O[t],j]
+ *   Yd[r,j] = acc[r,j] * rs[i] * cs[j] / 127^2 + sum_t X[i,O[t]] * W[O[t],j] (+ b[j])
  *   Y[r,j]  = fp16_RNE(Yd[r,j])
- * evaluated in double, outlier terms added in ascending column order. */
+ * evaluated in double, outlier terms added in ascending column order.  The
+ * optional bias b (fp16 [N], NULL for none) is the linear layer's: a layer's
+ * output is X W + b ("LLM.int8()" arXiv abstract: the method replaces the
+ * feed-forward and attention projection layers), added last. */
 void oracle_mixed_output(const int64_t* acc, const float* rs, const float* cs, const uint16_t* X,
                          int64_t ldx, const uint16_t* W, int64_t N, const int32_t* O, int64_t n_o,
-                         const int64_t* rows, int64_t n_rows, double* Yd, uint16_t* Y)
+                         const uint16_t* bias, const int64_t* rows, int64_t n_rows, double* Yd, uint16_t* Y)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < n_rows; ++r) {
@@ -300,6 +303,9 @@ void oracle_mixed_output(const int64_t* acc, const float* rs, const float* cs, c
             for (int64_t j = 0; j < N; ++j)
                 yd[j] += x * oracle_half_to_double(w[j]);
         }
+        if (bias)
+            for (int64_t j = 0; j < N; ++j)
+                yd[j] += oracle_half_to_double(bias[j]);
         for (int64_t j = 0; j < N; ++j)
             Y[r * N + j] = oracle_double_to_half(yd[j]);
     }

@@ -413,3 +413,27 @@ def test_int8_weight_reading_at_tau_limits(name, X, W):
     r = oracle.mixed_matmul(X, W, 0.0, int8_weight=True)
     Wd = oracle.dequantize_weight(*oracle.quantize_weight(W)).astype(np.float64)
     assert np.allclose(r["Yd"], X.astype(np.float64) @ Wd, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ linear-layer bias
+
+def test_bias_alone_when_x_is_zero():
+    """X = 0: no codes, no outliers, acc = 0, so every row of Y is the bias
+    itself (exact in fp16), with the bias indexed by output column."""
+    rng = np.random.default_rng(5)
+    M, K, N = 7, 40, 23
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float16)
+    b = (rng.standard_normal(N) * 3).astype(np.float16)
+    r = oracle.mixed_matmul(np.zeros((M, K), np.float16), W, 6.0, bias=b)
+    assert np.array_equal(r["Y"].view(np.uint16), np.broadcast_to(b.view(np.uint16), (M, N)))
+
+
+@pytest.mark.parametrize("name,X,W", _problems())
+def test_bias_on_the_fp16_matmul(name, X, W):
+    """tau = 0 (every column an outlier): Y is the fp16 rounding of X W + b,
+    X W summed in double."""
+    rng = np.random.default_rng(X.shape[0] * 7 + W.shape[1])
+    b = (rng.standard_normal(W.shape[1]) * 0.5).astype(np.float16)
+    r = oracle.mixed_matmul(X, W, 0.0, bias=b)
+    exact = X.astype(np.float64) @ W.astype(np.float64) + b.astype(np.float64)[None, :]
+    assert np.allclose(r["Yd"], exact, rtol=1e-12, atol=1e-12)
