@@ -150,7 +150,11 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
  *   Wq, ldk    int8 [N, ldk] and
  *   col_scale  fp32 [N] from llmint8_quantize_weight_colwise.
  *   W, ldw     fp16 [K, N] row-major, row stride ldw >= N: only the rows in O
- *              are read (the 16-bit outlier product).
+ *              are read (the 16-bit outlier product).  W may be NULL (ldw
+ *              ignored) when no fp16 copy of the weight is kept: the outlier
+ *              rows are then recovered from Wq, W~[k, j] = fp16_RNE(Wq[j, k]
+ *              * cs[j] / 127), so the weight lives in memory as int8 only
+ *              ("LLM.int8()" arXiv abstract: inference memory halved).
  *   tau        threshold (>= 0 or +inf).
  *   outlier_cap  bound on n_o the workspace is sized for; outlier_cap = K is
  *              always enough.  If n_o > outlier_cap, Y is filled with NaN and

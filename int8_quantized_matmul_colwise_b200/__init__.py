@@ -61,12 +61,14 @@ def quantize_act_rowwise_outliers(X, tau: float = 6.0, outlier_cap: Optional[int
     llmint8_quantize_act_rowwise_outliers(X, tau, out["Xq"], out["row_scale"], out["outlier_idx"],
                                           out["n_outlier"], out["Xo"], ws, stream)
     out["ws"] = ws
+    out["K"] = K
     return out
 
 
 def mixed_matmul(X, Wq, col_scale, W, tau: float = 6.0, outlier_cap: Optional[int] = None, Y=None, ws=None,
                  stream=None):
-    """Y = X . W by the LLM.int8() decomposition (fp16 [M, N])."""
+    """Y = X . W by the LLM.int8() decomposition (fp16 [M, N]).  W = None:
+    no fp16 weight kept, the outlier rows are recovered from Wq."""
     import torch
     M, K = X.shape
     N = Wq.size(0)
@@ -84,7 +86,7 @@ def mixed_gemm(act: Dict[str, object], Wq, col_scale, W, Y=None, ws=None, stream
     import torch
     Xq = act["Xq"]
     M, N = Xq.size(0), Wq.size(0)
-    K = W.size(0)
+    K = W.size(0) if W is not None else int(act["K"])  # W None: int8-only weight
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=Xq.device)
     if ws is None:

@@ -206,12 +206,13 @@ def llmint8_mixed_matmul(X, Wq, col_scale, W, tau: float, outlier_cap: int, Y, w
     _rowmajor(X, "X", torch.float16)
     _rowmajor(Wq, "Wq", torch.int8)
     _rowmajor(col_scale, "col_scale", torch.float32, 1)
-    _rowmajor(W, "W", torch.float16)
+    if W is not None:  # None: no fp16 weight kept, the outlier rows come from Wq
+        _rowmajor(W, "W", torch.float16)
     _rowmajor(Y, "Y", torch.float16)
     M, K = X.shape
     N = Wq.size(0)
     _check(lib().llmint8_mixed_matmul(
-        _ptr(X), M, K, _ld(X), _ptr(Wq), _ld(Wq), _ptr(col_scale), _ptr(W), _ld(W), N, float(tau),
+        _ptr(X), M, K, _ld(X), _ptr(Wq), _ld(Wq), _ptr(col_scale), _ptr(W), 0 if W is None else _ld(W), N, float(tau),
         int(outlier_cap), _ptr(Y), _ld(Y), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
         "llmint8_mixed_matmul")
 
@@ -226,12 +227,14 @@ def llmint8_mixed_gemm(Xq, row_scale, outlier_idx, n_outlier, Xo, Wq, col_scale,
     _rowmajor(Xo, "Xo", torch.float16)
     _rowmajor(Wq, "Wq", torch.int8)
     _rowmajor(col_scale, "col_scale", torch.float32, 1)
-    _rowmajor(W, "W", torch.float16)
+    if W is not None:  # None: no fp16 weight kept, the outlier rows come from Wq
+        _rowmajor(W, "W", torch.float16)
     _rowmajor(Y, "Y", torch.float16)
     M, N = Xq.size(0), Wq.size(0)
     _check(lib().llmint8_mixed_gemm(
         _ptr(Xq), _ld(Xq), _ptr(row_scale), _ptr(outlier_idx), _ptr(n_outlier), outlier_idx.numel(), _ptr(Xo),
-        _ld(Xo), _ptr(Wq), _ld(Wq), _ptr(col_scale), _ptr(W), _ld(W), M, N, K, _ptr(Y), _ld(Y), _ptr(ws),
+        _ld(Xo), _ptr(Wq), _ld(Wq), _ptr(col_scale), _ptr(W), 0 if W is None else _ld(W), M, N, K, _ptr(Y), _ld(Y),
+        _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)), "llmint8_mixed_gemm")
 
 

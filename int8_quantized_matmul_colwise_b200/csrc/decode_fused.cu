@@ -406,13 +406,24 @@ __global__ void __launch_bounds__(kThreadsF, MINB)
     const int tx = min(n_use, kOList);
     const unsigned short* Wb = reinterpret_cast<const unsigned short*>(W);
     const unsigned short* Xb = reinterpret_cast<const unsigned short*>(X);
+    // (no fp16 weight kept: the code Wq[n, O[t]] and cs[n] instead, turned
+    // into the recovered fp16 value when stored)
     unsigned short pf_w[kPW], pf_x[kPX];
+    float pf_c[kPW];
 #pragma unroll
     for (int u = 0; u < kPW; ++u) {
       const int k = at + u * kActThreads;
       const int t = k >> (7 - log2s), i = k & (RO - 1);
       const int n = n0 + static_cast<int>(rank) * RO + i;
-      pf_w[u] = (t < tw && n < p.N) ? Wb[static_cast<int64_t>(s_ol[t]) * p.ldw + n] : static_cast<unsigned short>(0);
+      const bool use = t < tw && n < p.N;
+      if (W != nullptr) {
+        pf_w[u] = use ? Wb[static_cast<int64_t>(s_ol[t]) * p.ldw + n] : static_cast<unsigned short>(0);
+        pf_c[u] = 0.0f;
+      } else {
+        pf_w[u] = use ? static_cast<unsigned short>(static_cast<uint8_t>(p.Wq[int64_t(n) * p.ldk + s_ol[t]]))
+                      : static_cast<unsigned short>(0);
+        pf_c[u] = use ? __ldg(p.cs + n) : 0.0f;
+      }
     }
 #pragma unroll
     for (int u = 0; u < kPX; ++u) {
@@ -480,7 +491,9 @@ __global__ void __launch_bounds__(kThreadsF, MINB)
         *reinterpret_cast<uint2*>(p.Xq + static_cast<int64_t>(m) * p.ldq + c) = make_uint2(0u, 0u);
     }
 #pragma unroll
-    for (int u = 0; u < kPW; ++u) s_w[at + u * kActThreads] = __ushort_as_half(pf_w[u]);
+    for (int u = 0; u < kPW; ++u)
+      s_w[at + u * kActThreads] = __ushort_as_half(
+          W != nullptr ? pf_w[u] : dequant_weight_bits(static_cast<int8_t>(pf_w[u] & 0xFFu), pf_c[u]));
 #pragma unroll
     for (int u = 0; u < kPX; ++u) s_xo[at + u * kActThreads] = __ushort_as_half(pf_x[u]);
     fence_proxy_async_smem();  // the operand was written by the generic proxy
@@ -526,7 +539,8 @@ __global__ void __launch_bounds__(kThreadsF, MINB)
       const int i = et & (RO - 1);                        // row of this CTA's share it finishes
       const int cg = et >> (7 - log2s);                   // and its columns m = cg, cg + S, ...
       const int n = n0 + static_cast<int>(rank) * RO + i;
-      const float csn = n < p.N ? __ldg(p.cs + n) * (1.0f / 16129.0f) : 0.0f;
+      const float csw = n < p.N ? __ldg(p.cs + n) : 0.0f;
+      const float csn = csw * (1.0f / 16129.0f);
       uint32_t v[32];
 #pragma unroll
       for (int m = 0; m < 32; ++m) v[m] = 0u;
@@ -583,7 +597,10 @@ __global__ void __launch_bounds__(kThreadsF, MINB)
 #pragma unroll 1
         for (int t = kWS; t < n_use; ++t) {  // outliers past the staged ones
           const int col = t < kOList ? s_ol[t] : outlier_at(t, s_mask, s_pre, nwords);
-          const float w = n < p.N ? __half2float(W[static_cast<int64_t>(col) * p.ldw + n]) : 0.0f;
+          const float w = n >= p.N ? 0.0f
+                          : W != nullptr
+                              ? __half2float(W[static_cast<int64_t>(col) * p.ldw + n])
+                              : __half2float(__ushort_as_half(dequant_weight_bits(p.Wq[int64_t(n) * p.ldk + col], csw)));
           const float xv =
               t < kOList ? __half2float(s_xo[m * kOList + t]) : __half2float(X[static_cast<int64_t>(m) * p.ldx + col]);
           y = fmaf(xv, w, y);

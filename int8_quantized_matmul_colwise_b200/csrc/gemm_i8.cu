@@ -39,6 +39,7 @@
 
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace llmint8 {
 
@@ -284,7 +285,19 @@ __device__ __forceinline__ void stage_outlier_rows(const GemmArgs& p, const Shar
     const int cc = 8 * (pc % (BN / 8));
     const int c = n0 + cc;
     uint4 u = make_uint4(0u, 0u, 0u, 0u);
-    if (t < tn) {
+    if (t < tn && W == nullptr) {  // no fp16 weight kept: the rows recovered from Wq
+      const int64_t k = __ldg(p.O + t0 + t);
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int n = c + 2 * e;
+        const uint32_t lo = n < p.N ? dequant_weight_bits(p.Wq[int64_t(n) * p.ldk + k], __ldg(p.cs + n)) : 0u;
+        const uint32_t hi =
+            n + 1 < p.N ? dequant_weight_bits(p.Wq[int64_t(n + 1) * p.ldk + k], __ldg(p.cs + n + 1)) : 0u;
+        w[e] = lo | (hi << 16);
+      }
+      u = make_uint4(w[0], w[1], w[2], w[3]);
+    } else if (t < tn) {
       const __half* wr = W + static_cast<int64_t>(__ldg(p.O + t0 + t)) * p.ldw + c;
       if (w_vec && c + 8 <= p.N) {
         u = __ldg(reinterpret_cast<const uint4*>(wr));

@@ -25,6 +25,7 @@
 
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace llmint8 {
 
@@ -97,7 +98,11 @@ __device__ void finish_row(const DecodeArgs& p, const float* s_rs, float* s_xo, 
       }
       named_bar_sync(1, 128);
       for (int t = 0; t < tn; ++t) {
-        const float w = n < p.N ? __half2float(W[static_cast<int64_t>(__ldg(p.O + t0 + t)) * p.ldw + n]) : 0.0f;
+        const int64_t k = __ldg(p.O + t0 + t);
+        const float w = n >= p.N ? 0.0f
+                        : W != nullptr ? __half2float(W[k * p.ldw + n])
+                                       : __half2float(__ushort_as_half(dequant_weight_bits(p.Wq[int64_t(n) * p.ldk + k],
+                                                                                           __ldg(p.cs + n))));
 #pragma unroll
         for (int m = 0; m < NP; ++m) y[m] = fmaf(s_xo[m * kXoCols + t], w, y[m]);
       }
@@ -250,9 +255,18 @@ __global__ void __launch_bounds__(kThreadsD, 1)
       int orow[kWReg];
 #pragma unroll
       for (int t = 0; t < kWReg; ++t) orow[t] = t < n_use ? __ldg(p.O + t) : 0;
+      if (W != nullptr) {
 #pragma unroll
-      for (int t = 0; t < kWReg; ++t)
-        wreg[t] = (t < n_use && n < p.N) ? __half2float(W[static_cast<int64_t>(orow[t]) * p.ldw + n]) : 0.0f;
+        for (int t = 0; t < kWReg; ++t)
+          wreg[t] = (t < n_use && n < p.N) ? __half2float(W[static_cast<int64_t>(orow[t]) * p.ldw + n]) : 0.0f;
+      } else {  // no fp16 weight kept: the outlier rows recovered from Wq
+        const float csw = n < p.N ? __ldg(p.cs + n) : 0.0f;
+#pragma unroll
+        for (int t = 0; t < kWReg; ++t)
+          wreg[t] = (t < n_use && n < p.N)
+                        ? __half2float(__ushort_as_half(dequant_weight_bits(p.Wq[int64_t(n) * p.ldk + orow[t]], csw)))
+                        : 0.0f;
+      }
     } else {
 #pragma unroll
       for (int t = 0; t < kWReg; ++t) wreg[t] = 0.0f;

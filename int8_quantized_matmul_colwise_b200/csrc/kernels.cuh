@@ -44,8 +44,10 @@ struct GemmArgs {
   const int32_t* O;   // [cap] outlier columns (rows of W)
   const int32_t* n_o; // device count
   int cap;
-  const void* W;      // fp16 [K, ldw]
+  const void* W;      // fp16 [K, ldw]; nullptr: the outlier rows come from Wq
   int64_t ldw;
+  const int8_t* Wq;   // int8 [N, ldk] (read for the outlier rows when W is nullptr)
+  int64_t ldk;
   void* Y;            // fp16 [M, ldy]
   int64_t ldy;
   int32_t* C;         // int32 [M, ldc] (raw accumulator output mode)
@@ -87,8 +89,10 @@ struct DecodeArgs {
   const int32_t* O;
   const int32_t* n_o;
   int cap;
-  const void* W;
+  const void* W;       // nullptr: the outlier rows come from Wq
   int64_t ldw;
+  const int8_t* Wq;    // int8 [N, ldk]
+  int64_t ldk;
   void* Y;
   int64_t ldy;
   int32_t* C;  // raw int32 output mode
@@ -124,8 +128,10 @@ struct FusedArgs {
   int M, N, K;
   float tau;
   const float* cs;
-  const void* W;  // fp16 [K, ldw]: outlier rows
+  const void* W;  // fp16 [K, ldw]: outlier rows; nullptr: recovered from Wq
   int64_t ldw;
+  const int8_t* Wq;  // int8 [N, ldk]
+  int64_t ldk;
   void* Y;
   int64_t ldy;
   int8_t* Xq;  // workspace outputs, written by the first cluster

@@ -31,6 +31,18 @@ __device__ __forceinline__ int quantize_exact(float x, float s, float inv_s) {
   return x < 0.0f ? -qi : qi;
 }
 
+// A weight value recovered from its int8 code, for callers that keep no fp16
+// weight: fp16_RNE(q * cs / 127), as the bits of the fp16.  q * cs is exact in
+// binary32 (7- and 11-bit significands, a = |q| * significand(cs) < 2^18) and
+// the quotient is correctly rounded.  Unless the exact quotient is itself an
+// fp16 rounding boundary, it lies at least 2^-19 (relative) from one, since
+// a * 2^j / 127 is at least 1/127 from every odd integer; the binary32
+// rounding moves it by at most 2^-24, so rounding the binary32 quotient to
+// fp16 gives the fp16 rounding of the exact value.
+__device__ __forceinline__ unsigned short dequant_weight_bits(int q, float cs) {
+  return __half_as_ushort(__float2half_rn(__fdiv_rn(__fmul_rn(static_cast<float>(q), cs), 127.0f)));
+}
+
 // Pack four codes (low byte first) into a 32-bit word.
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
   return (uint32_t(a) & 0xFFu) | ((uint32_t(b) & 0xFFu) << 8) | ((uint32_t(c) & 0xFFu) << 16) |

@@ -403,3 +403,71 @@ def test_mixed_matmul_full_size_175b(L):
     X, W = wl.make_inputs(w)
     rows = wl.sample_rows(w.M, n=16)
     check_path(L, X, W, w.tau, rows=rows)
+
+
+# ------------------------------------------------------------------ int8-only weight (W = NULL)
+# No fp16 copy of the weight: the outlier rows are recovered from Wq
+# (fp16_RNE(Wq * cs / 127)); the oracle's int8_weight reading.
+
+def check_int8_weight(L, X, W, tau, rows=None, split=False, Xd=None):
+    M, K = X.shape
+    N = W.shape[1]
+    Wq, cs = L.quantize_weight_colwise(dev(W))
+    Wq_ref, cs_ref = oracle.quantize_weight(W)
+    Xd = dev(X) if Xd is None else Xd
+    if split:
+        act = L.quantize_act_rowwise_outliers(Xd, tau)
+        ws = L.empty_workspace(M, N, K, K)
+        Y = host(L.mixed_gemm(act, Wq, cs, None, ws=ws))
+    else:
+        ws = L.empty_workspace(M, N, K, K)
+        Y = host(L.mixed_matmul(Xd, Wq, cs, None, tau, ws=ws))
+    assert_status_ok(L, ws)
+    r = oracle.mixed_matmul(X, W, tau, rows=rows, weight=(Wq_ref, cs_ref), int8_weight=True)
+    y_close(Y if rows is None else Y[rows], r["Y"])
+    return Y, r
+
+
+INT8W_SHAPES = ["tiny", "decode_m1", "decode_m8", "decode_m32", "ragged_1000x1000x1000", "ragged_129x257x520",
+                "ragged_1x1001x1000", "ragged_2047x4095x4100", "ragged_3x33x24"]
+
+
+@pytest.mark.parametrize("name", INT8W_SHAPES)
+def test_int8_only_weight_path(L, name):
+    w = wl.get(name)
+    X, W = wl.make_inputs(w)
+    check_int8_weight(L, X, W, w.tau)
+
+
+@pytest.mark.parametrize("name", ["ragged_129x257x520", "decode_m8", "tiny"])
+def test_int8_only_weight_split_entry_points(L, name):
+    """mixed_gemm with W = NULL: the prefill GEMM's staged rows (M > 32) and
+    the split-K decode GEMM's register rows (M <= 32)."""
+    w = wl.get(name)
+    X, W = wl.make_inputs(w)
+    check_int8_weight(L, X, W, w.tau, split=True)
+
+
+@pytest.mark.parametrize("M,N,K", [(129, 257, 520), (4, 256, 512), (40, 300, 264)])
+def test_int8_only_weight_every_column_an_outlier(L, M, N, K):
+    """tau = 0: every column is an outlier, so every recovered row is used
+    (several staging passes in the prefill GEMM, the epilogue's reload path in
+    the decode kernels)."""
+    rng = np.random.default_rng(M + N + K)
+    X, W, _ = wl.random_small(rng, M, K, N, 2)
+    check_int8_weight(L, X, W, 0.0)
+
+
+def test_int8_only_weight_three_kernel_decode(L):
+    """X rows not 16-byte aligned (the scan / quantize / split-K path)."""
+    M, N, K = 8, 1000, 1000
+    X, W, _ = wl.random_small(np.random.default_rng(9), M, K, N, 3)
+    wide = np.zeros((M, K + 1), np.float16)
+    wide[:, :K] = X
+    check_int8_weight(L, X, W, 6.0, Xd=dev(wide)[:, :K])
+
+
+def test_int8_only_weight_full_size_ffn(L):
+    w = wl.get("ffn_6p7b_prefill")
+    X, W = wl.make_inputs(w)
+    check_int8_weight(L, X, W, w.tau, rows=wl.sample_rows(w.M))
