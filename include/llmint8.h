@@ -155,6 +155,9 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
  *              rows are then recovered from Wq, W~[k, j] = fp16_RNE(Wq[j, k]
  *              * cs[j] / 127), so the weight lives in memory as int8 only
  *              ("LLM.int8()" arXiv abstract: inference memory halved).
+ *   bias       optional fp16 [N] (NULL for none), 2-byte aligned: the linear
+ *              layer's bias, added to every row after the outlier product and
+ *              before the fp16 rounding (Y = X W + b).
  *   tau        threshold (>= 0 or +inf).
  *   outlier_cap  bound on n_o the workspace is sized for; outlier_cap = K is
  *              always enough.  If n_o > outlier_cap, Y is filled with NaN and
@@ -172,8 +175,8 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
  * synchronisation. */
 llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
                                     int64_t ldk, const float* col_scale, const void* W, int64_t ldw,
-                                    int64_t N, float tau, int64_t outlier_cap, void* Y, int64_t ldy,
-                                    void* ws, size_t ws_bytes, void* stream);
+                                    const void* bias, int64_t N, float tau, int64_t outlier_cap, void* Y,
+                                    int64_t ldy, void* ws, size_t ws_bytes, void* stream);
 
 /* Number of kernels llmint8_mixed_matmul launches on the current device for
  * these arguments (1 on the one-kernel decode path, else 3; 0 for invalid
@@ -188,7 +191,7 @@ int llmint8_mixed_matmul_kernels(int64_t M, int64_t N, int64_t K, int64_t ldx, c
  *   row_scale        fp32 [M]
  *   outlier_idx      int32 [outlier_cap], n_outlier int32 [1] (device)
  *   Xo, ldo          fp16 [M, ldo], ldo >= outlier_cap
- *   Wq, ldk, col_scale, W, ldw, Y, ldy  as for llmint8_mixed_matmul
+ *   Wq, ldk, col_scale, W, ldw, bias, Y, ldy  as for llmint8_mixed_matmul
  *   ws               at least 256 bytes (status word).  For M <= 32 the GEMM
  *                    splits K across CTAs when ws also holds its reduction
  *                    scratch (a workspace of llmint8_workspace_size(M, N, K,
@@ -199,8 +202,9 @@ int llmint8_mixed_matmul_kernels(int64_t M, int64_t N, int64_t K, int64_t ldx, c
 llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* row_scale,
                                   const int32_t* outlier_idx, const int32_t* n_outlier, int64_t outlier_cap,
                                   const void* Xo, int64_t ldo, const int8_t* Wq, int64_t ldk,
-                                  const float* col_scale, const void* W, int64_t ldw, int64_t M, int64_t N,
-                                  int64_t K, void* Y, int64_t ldy, void* ws, size_t ws_bytes, void* stream);
+                                  const float* col_scale, const void* W, int64_t ldw, const void* bias,
+                                  int64_t M, int64_t N, int64_t K, void* Y, int64_t ldy, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /* Allocation-free variant of llmint8_quantize_act_rowwise_outliers (the
  * pages have no counterpart: this serves callers of this library that cannot

@@ -66,9 +66,9 @@ def quantize_act_rowwise_outliers(X, tau: float = 6.0, outlier_cap: Optional[int
 
 
 def mixed_matmul(X, Wq, col_scale, W, tau: float = 6.0, outlier_cap: Optional[int] = None, Y=None, ws=None,
-                 stream=None):
-    """Y = X . W by the LLM.int8() decomposition (fp16 [M, N]).  W = None:
-    no fp16 weight kept, the outlier rows are recovered from Wq."""
+                 stream=None, bias=None):
+    """Y = X . W (+ bias) by the LLM.int8() decomposition (fp16 [M, N]).
+    W = None: no fp16 weight kept, the outlier rows are recovered from Wq."""
     import torch
     M, K = X.shape
     N = Wq.size(0)
@@ -77,11 +77,11 @@ def mixed_matmul(X, Wq, col_scale, W, tau: float = 6.0, outlier_cap: Optional[in
         Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
     if ws is None:
         ws = empty_workspace(M, N, K, cap, device=X.device)
-    llmint8_mixed_matmul(X, Wq, col_scale, W, tau, cap, Y, ws, stream)
+    llmint8_mixed_matmul(X, Wq, col_scale, W, tau, cap, Y, ws, stream, bias)
     return Y
 
 
-def mixed_gemm(act: Dict[str, object], Wq, col_scale, W, Y=None, ws=None, stream=None):
+def mixed_gemm(act: Dict[str, object], Wq, col_scale, W, Y=None, ws=None, stream=None, bias=None):
     """Steps a5-a7 on the output of quantize_act_rowwise_outliers."""
     import torch
     Xq = act["Xq"]
@@ -92,7 +92,7 @@ def mixed_gemm(act: Dict[str, object], Wq, col_scale, W, Y=None, ws=None, stream
     if ws is None:
         ws = act["ws"]
     llmint8_mixed_gemm(Xq, act["row_scale"], act["outlier_idx"], act["n_outlier"], act["Xo"], Wq, col_scale, W,
-                       K, Y, ws, stream)
+                       K, Y, ws, stream, bias)
     return Y
 
 
@@ -125,3 +125,11 @@ class Int8Weight:
 
     def matmul(self, X, tau: float = 6.0, outlier_cap: Optional[int] = None, Y=None, ws=None, stream=None):
         return mixed_matmul(X, self.Wq, self.col_scale, self.W, tau, outlier_cap, Y, ws, stream)
+
+
+def __getattr__(name):
+    # the torch module wrapper is imported on first use
+    if name == "Int8Linear":
+        from .linear import Int8Linear
+        return Int8Linear
+    raise AttributeError(name)

@@ -65,9 +65,9 @@ SIGNATURES = {
     "llmint8_quantize_weight_colwise": (_ST, [_P, _I64, _I64, _I64, _P, _I64, _P, _P]),
     "llmint8_quantize_act_rowwise_outliers": (_ST, [_P, _I64, _I64, _I64, _F, _P, _I64, _P, _P, _I64, _P, _P,
                                                     _I64, _P, _SZ, _P]),
-    "llmint8_mixed_matmul": (_ST, [_P, _I64, _I64, _I64, _P, _I64, _P, _P, _I64, _I64, _F, _I64, _P, _I64, _P,
-                                   _SZ, _P]),
-    "llmint8_mixed_gemm": (_ST, [_P, _I64, _P, _P, _P, _I64, _P, _I64, _P, _I64, _P, _P, _I64, _I64, _I64,
+    "llmint8_mixed_matmul": (_ST, [_P, _I64, _I64, _I64, _P, _I64, _P, _P, _I64, _P, _I64, _F, _I64, _P, _I64,
+                                   _P, _SZ, _P]),
+    "llmint8_mixed_gemm": (_ST, [_P, _I64, _P, _P, _P, _I64, _P, _I64, _P, _I64, _P, _P, _I64, _P, _I64, _I64,
                                  _I64, _P, _I64, _P, _SZ, _P]),
     "llmint8_quantize_act_rowwise_outliers_noalloc": (_ST, [_P, _I64, _I64, _I64, _F, _P, _I64, _P, _P, _I64, _P,
                                                             _P, _I64, _P]),
@@ -141,6 +141,17 @@ def _rowmajor(t, name: str, dtype, ndim=2):
     return t
 
 
+def _vector(t, name: str, n: int):
+    """An optional fp16 [n] device vector (the linear layer's bias)."""
+    if t is None:
+        return None
+    torch = _torch()
+    _rowmajor(t, name, torch.float16, 1)
+    if t.numel() != n:
+        raise ValueError(f"{name}: expected {n} elements, got {t.numel()}")
+    return t
+
+
 def _ld(t) -> int:
     return t.stride(0) if t.size(0) > 1 else max(t.stride(0), t.size(1))
 
@@ -201,7 +212,7 @@ def llmint8_quantize_act_rowwise_outliers(X, tau: float, Xq, row_scale, outlier_
         _stream(stream)), "llmint8_quantize_act_rowwise_outliers")
 
 
-def llmint8_mixed_matmul(X, Wq, col_scale, W, tau: float, outlier_cap: int, Y, ws, stream=None):
+def llmint8_mixed_matmul(X, Wq, col_scale, W, tau: float, outlier_cap: int, Y, ws, stream=None, bias=None):
     torch = _torch()
     _rowmajor(X, "X", torch.float16)
     _rowmajor(Wq, "Wq", torch.int8)
@@ -212,13 +223,14 @@ def llmint8_mixed_matmul(X, Wq, col_scale, W, tau: float, outlier_cap: int, Y, w
     M, K = X.shape
     N = Wq.size(0)
     _check(lib().llmint8_mixed_matmul(
-        _ptr(X), M, K, _ld(X), _ptr(Wq), _ld(Wq), _ptr(col_scale), _ptr(W), 0 if W is None else _ld(W), N, float(tau),
+        _ptr(X), M, K, _ld(X), _ptr(Wq), _ld(Wq), _ptr(col_scale), _ptr(W), 0 if W is None else _ld(W),
+        _ptr(_vector(bias, "bias", N)), N, float(tau),
         int(outlier_cap), _ptr(Y), _ld(Y), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
         "llmint8_mixed_matmul")
 
 
 def llmint8_mixed_gemm(Xq, row_scale, outlier_idx, n_outlier, Xo, Wq, col_scale, W, K: int, Y, ws,
-                       stream=None):
+                       stream=None, bias=None):
     torch = _torch()
     _rowmajor(Xq, "Xq", torch.int8)
     _rowmajor(row_scale, "row_scale", torch.float32, 1)
@@ -233,7 +245,8 @@ def llmint8_mixed_gemm(Xq, row_scale, outlier_idx, n_outlier, Xo, Wq, col_scale,
     M, N = Xq.size(0), Wq.size(0)
     _check(lib().llmint8_mixed_gemm(
         _ptr(Xq), _ld(Xq), _ptr(row_scale), _ptr(outlier_idx), _ptr(n_outlier), outlier_idx.numel(), _ptr(Xo),
-        _ld(Xo), _ptr(Wq), _ld(Wq), _ptr(col_scale), _ptr(W), 0 if W is None else _ld(W), M, N, K, _ptr(Y), _ld(Y),
+        _ld(Xo), _ptr(Wq), _ld(Wq), _ptr(col_scale), _ptr(W), 0 if W is None else _ld(W),
+        _ptr(_vector(bias, "bias", Wq.size(0))), M, N, K, _ptr(Y), _ld(Y),
         _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)), "llmint8_mixed_gemm")
 

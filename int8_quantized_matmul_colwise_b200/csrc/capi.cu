@@ -256,16 +256,17 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
 }
 
 llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
-                                    int64_t ldk, const float* col_scale, const void* W, int64_t ldw, int64_t N,
-                                    float tau, int64_t outlier_cap, void* Y, int64_t ldy, void* ws,
-                                    size_t ws_bytes, void* stream) {
+                                    int64_t ldk, const float* col_scale, const void* W, int64_t ldw,
+                                    const void* bias, int64_t N, float tau, int64_t outlier_cap, void* Y,
+                                    int64_t ldy, void* ws, size_t ws_bytes, void* stream) {
   if (!X || !Wq || !col_scale || !Y) return LLMINT8_ERR_INVALID_ARG;  // W may be NULL: int8-only weight
   if (M < 1 || N < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1)
     return LLMINT8_ERR_INVALID_ARG;
   if (ldx < K || (W && ldw < N) || ldy < N || ldk < K || ldk % 16 != 0 || !valid_tau(tau))
     return LLMINT8_ERR_INVALID_ARG;
   if (outlier_cap < 1 || outlier_cap > K) return LLMINT8_ERR_INVALID_ARG;
-  if (!aligned(Wq, 16) || !aligned(X, 2) || (W && !aligned(W, 2)) || !aligned(Y, 2) || !aligned(col_scale, 4))
+  if (!aligned(Wq, 16) || !aligned(X, 2) || (W && !aligned(W, 2)) || !aligned(Y, 2) || !aligned(col_scale, 4) ||
+      !aligned(bias, 2))
     return LLMINT8_ERR_INVALID_ARG;
   llmint8_ws_layout L;
   size_t colmax_off, bitmask_off, decode_off;
@@ -301,6 +302,7 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
     f.ldw = ldw;
     f.Wq = Wq;
     f.ldk = ldk;
+    f.bias = bias;
     f.Y = Y;
     f.ldy = ldy;
     f.Xq = xq;
@@ -347,6 +349,7 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
     d.ldw = ldw;
     d.Wq = Wq;
     d.ldk = ldk;
+    d.bias = bias;
     d.Y = Y;
     d.ldy = ldy;
     d.partial = reinterpret_cast<int32_t*>(b + decode_off);
@@ -371,6 +374,7 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
   a.ldw = ldw;
   a.Wq = Wq;
   a.ldk = ldk;
+  a.bias = bias;
   a.Y = Y;
   a.ldy = ldy;
   a.C = nullptr;
@@ -384,8 +388,9 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
 llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* row_scale,
                                   const int32_t* outlier_idx, const int32_t* n_outlier, int64_t outlier_cap,
                                   const void* Xo, int64_t ldo, const int8_t* Wq, int64_t ldk,
-                                  const float* col_scale, const void* W, int64_t ldw, int64_t M, int64_t N,
-                                  int64_t K, void* Y, int64_t ldy, void* ws, size_t ws_bytes, void* stream) {
+                                  const float* col_scale, const void* W, int64_t ldw, const void* bias,
+                                  int64_t M, int64_t N, int64_t K, void* Y, int64_t ldy, void* ws,
+                                  size_t ws_bytes, void* stream) {
   if (!Xq || !row_scale || !outlier_idx || !n_outlier || !Xo || !Wq || !col_scale || !Y)
     return LLMINT8_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1)
@@ -394,6 +399,7 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
   if (ldq < K || ldk < K || ldq % 16 != 0 || ldk % 16 != 0 || (W && ldw < N) || ldy < N)
     return LLMINT8_ERR_INVALID_ARG;
   if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Xo, 2) || (W && !aligned(W, 2)) || !aligned(Y, 2) ||
+      !aligned(bias, 2) ||
       !aligned(row_scale, 4) || !aligned(col_scale, 4))
     return LLMINT8_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256) || ws_bytes < 256) return LLMINT8_ERR_WORKSPACE;
@@ -421,6 +427,7 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
     d.ldw = ldw;
     d.Wq = Wq;
     d.ldk = ldk;
+    d.bias = bias;
     d.Y = Y;
     d.ldy = ldy;
     // the split-K scratch is the last decode_scratch_bytes of the workspace
@@ -448,6 +455,7 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
   a.ldw = ldw;
   a.Wq = Wq;
   a.ldk = ldk;
+  a.bias = bias;
   a.Y = Y;
   a.ldy = ldy;
   a.status = static_cast<uint32_t*>(ws);

@@ -541,6 +541,7 @@ __global__ void __launch_bounds__(kThreadsF, MINB)
       const int n = n0 + static_cast<int>(rank) * RO + i;
       const float csw = n < p.N ? __ldg(p.cs + n) : 0.0f;
       const float csn = csw * (1.0f / 16129.0f);
+      const float bn = (p.bias != nullptr && n < p.N) ? __half2float(static_cast<const __half*>(p.bias)[n]) : 0.0f;
       uint32_t v[32];
 #pragma unroll
       for (int m = 0; m < 32; ++m) v[m] = 0u;
@@ -605,6 +606,7 @@ __global__ void __launch_bounds__(kThreadsF, MINB)
               t < kOList ? __half2float(s_xo[m * kOList + t]) : __half2float(X[static_cast<int64_t>(m) * p.ldx + col]);
           y = fmaf(xv, w, y);
         }
+        if (p.bias != nullptr) y += bn;  // the linear layer's bias, added last
         if (n < p.N) Y[static_cast<int64_t>(m) * p.ldy + n] = __float2half_rn(overflow ? __int_as_float(0x7fc00000) : y);
       }
     } else {

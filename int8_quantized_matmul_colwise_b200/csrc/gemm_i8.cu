@@ -68,8 +68,9 @@ struct Geo {
   static constexpr uint32_t kOffB = kOffA + kStages * kBytesA;
   static constexpr uint32_t kOffWo = kOffB + kStages * kBytesB;     // fp16 [kSG][kWoStride]
   static constexpr uint32_t kOffCs = kOffWo + kSG * kWoStride * 2;  // fp32 [BN]
+  static constexpr uint32_t kOffBias = kOffCs + BN * 4;              // fp32 [BN]
   // per epilogue warp, 16 rows x 64 fp16 columns of Y in the 128-byte swizzle
-  static constexpr uint32_t kOffY = (kOffCs + BN * 4 + 1023) & ~1023u;
+  static constexpr uint32_t kOffY = (kOffBias + BN * 4 + 1023) & ~1023u;
   static constexpr uint32_t kYBytes = 16 * 128;
   static constexpr uint32_t kOffBars = kOffY + kEpiWarps * kYBytes;
   static constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;  // full, empty, tmem full/empty, drain
@@ -86,6 +87,7 @@ struct Shared {
   uint8_t* b;
   __half* wo;  // outlier rows of W over the tile's columns
   float* cs;  // column scales of the tile
+  float* bias;  // bias of the tile's columns (zero without a bias)
   uint8_t* ystage;  // Y staging tiles for the TMA store, one per epilogue warp
   uint64_t* full;
   uint64_t* empty;
@@ -105,6 +107,7 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
   s.b = base + G::kOffB;
   s.wo = reinterpret_cast<__half*>(base + G::kOffWo);
   s.cs = reinterpret_cast<float*>(base + G::kOffCs);
+  s.bias = reinterpret_cast<float*>(base + G::kOffBias);
   s.ystage = base + G::kOffY;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + G::kOffBars);
   s.full = bars;
@@ -268,6 +271,16 @@ __device__ __forceinline__ void stage_scales(const GemmArgs& p, const Shared& s,
       v.w = c + 3 < p.N ? __ldg(p.cs + c + 3) : 0.0f;
     }
     *reinterpret_cast<float4*>(s.cs + 4 * et) = v;
+    // the linear layer's bias (fp16), zero without one
+    const __half* bias = static_cast<const __half*>(p.bias);
+    float4 bv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (bias != nullptr) {
+      bv.x = c < p.N ? __half2float(bias[c]) : 0.0f;
+      bv.y = c + 1 < p.N ? __half2float(bias[c + 1]) : 0.0f;
+      bv.z = c + 2 < p.N ? __half2float(bias[c + 2]) : 0.0f;
+      bv.w = c + 3 < p.N ? __half2float(bias[c + 3]) : 0.0f;
+    }
+    *reinterpret_cast<float4*>(s.bias + 4 * et) = bv;
   }
 }
 
@@ -468,6 +481,16 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
                 ldmatrix_x4_trans(wo_lane + 2u * static_cast<uint32_t>(c * 64 + 16 * np), b0, b1, b2, b3);
                 mma_m16n8k16_f16f32(d[2 * np], afr, b0, b1);
                 mma_m16n8k16_f16f32(d[2 * np + 1], afr, b2, b3);
+              }
+            }
+            if (last && p.bias != nullptr) {  // the linear layer's bias, added last
+#pragma unroll
+              for (int n = 0; n < 8; ++n) {
+                const float2 b2 = *reinterpret_cast<const float2*>(s.bias + c * 64 + 8 * n + 2 * t4);
+                d[n][0] += b2.x;
+                d[n][1] += b2.y;
+                d[n][2] += b2.x;
+                d[n][3] += b2.y;
               }
             }
             if (last && p.y_tma) {

@@ -108,6 +108,11 @@ __device__ void finish_row(const DecodeArgs& p, const float* s_rs, float* s_xo, 
       }
     }
     if (n < p.N) {
+      if (p.bias != nullptr) {  // the linear layer's bias, added last
+        const float bn = __half2float(static_cast<const __half*>(p.bias)[n]);
+#pragma unroll
+        for (int m = 0; m < NP; ++m) y[m] += bn;
+      }
       __half* Y = static_cast<__half*>(p.Y);
 #pragma unroll
       for (int m = 0; m < NP; ++m)

@@ -48,6 +48,7 @@ struct GemmArgs {
   int64_t ldw;
   const int8_t* Wq;   // int8 [N, ldk] (read for the outlier rows when W is nullptr)
   int64_t ldk;
+  const void* bias;   // fp16 [N] added to every row, or nullptr
   void* Y;            // fp16 [M, ldy]
   int64_t ldy;
   int32_t* C;         // int32 [M, ldc] (raw accumulator output mode)
@@ -93,6 +94,7 @@ struct DecodeArgs {
   int64_t ldw;
   const int8_t* Wq;    // int8 [N, ldk]
   int64_t ldk;
+  const void* bias;    // fp16 [N] or nullptr
   void* Y;
   int64_t ldy;
   int32_t* C;  // raw int32 output mode
@@ -132,6 +134,7 @@ struct FusedArgs {
   int64_t ldw;
   const int8_t* Wq;  // int8 [N, ldk]
   int64_t ldk;
+  const void* bias;  // fp16 [N] or nullptr
   void* Y;
   int64_t ldy;
   int8_t* Xq;  // workspace outputs, written by the first cluster

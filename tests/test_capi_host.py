@@ -49,11 +49,11 @@ def test_workspace_size_rejects_bad_sizes(lib, M, N, K, cap):
 
 
 def _mm(lib, **kw):
-    a = dict(X=0x1000, M=4, K=32, ldx=32, Wq=0x2000, ldk=32, cs=0x3000, W=0x4000, ldw=16, N=16, tau=6.0,
-             cap=32, Y=0x5000, ldy=16, ws=0x10000, ws_bytes=1 << 20, stream=None)
+    a = dict(X=0x1000, M=4, K=32, ldx=32, Wq=0x2000, ldk=32, cs=0x3000, W=0x4000, ldw=16, bias=None, N=16,
+             tau=6.0, cap=32, Y=0x5000, ldy=16, ws=0x10000, ws_bytes=1 << 20, stream=None)
     a.update(kw)
     return lib.llmint8_mixed_matmul(a["X"], a["M"], a["K"], a["ldx"], a["Wq"], a["ldk"], a["cs"], a["W"],
-                                    a["ldw"], a["N"], a["tau"], a["cap"], a["Y"], a["ldy"], a["ws"],
+                                    a["ldw"], a["bias"], a["N"], a["tau"], a["cap"], a["Y"], a["ldy"], a["ws"],
                                     a["ws_bytes"], a["stream"])
 
 
@@ -73,6 +73,8 @@ def _mm(lib, **kw):
     (dict(ws=None), capi.ERR_WORKSPACE),
     (dict(ws=0x10010), capi.ERR_WORKSPACE),      # not 256-byte aligned
     (dict(ws_bytes=1024), capi.ERR_WORKSPACE),
+    (dict(bias=0x6001), capi.ERR_INVALID_ARG),   # bias not 2-byte aligned
+    (dict(W=None, ldw=0, ws_bytes=1024), capi.ERR_WORKSPACE),  # W = NULL is accepted (int8-only weight)
 ])
 def test_mixed_matmul_rejects_invalid_arguments_on_the_host(lib, kw, expect):
     # these fail validation before any CUDA call, so no device is needed

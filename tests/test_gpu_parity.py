@@ -471,3 +471,66 @@ def test_int8_only_weight_full_size_ffn(L):
     w = wl.get("ffn_6p7b_prefill")
     X, W = wl.make_inputs(w)
     check_int8_weight(L, X, W, w.tau, rows=wl.sample_rows(w.M))
+
+
+# ------------------------------------------------------------------ linear layer: bias fused in the epilogue
+
+def _bias_case(M, N, K, seed):
+    rng = np.random.default_rng(seed)
+    X, W, _ = wl.random_small(rng, M, K, N, 3)
+    b = (rng.standard_normal(N) * 0.5).astype(np.float16)
+    return X, W, b
+
+
+@pytest.mark.parametrize("M,N,K,how", [
+    (129, 257, 520, "matmul"),      # prefill GEMM epilogue
+    (8, 1000, 1000, "matmul"),      # one-kernel decode
+    (8, 1000, 1000, "unaligned"),   # three-kernel decode
+    (129, 257, 520, "split"),       # mixed_gemm, prefill GEMM
+    (8, 1000, 1000, "split"),       # mixed_gemm, split-K decode GEMM
+])
+def test_bias_every_kernel(L, M, N, K, how):
+    X, W, b = _bias_case(M, N, K, M + N + K)
+    Wd = dev(W)
+    Wq, cs = L.quantize_weight_colwise(Wd)
+    bd = dev(b)
+    if how == "split":
+        act = L.quantize_act_rowwise_outliers(dev(X), 6.0)
+        Y = host(L.mixed_gemm(act, Wq, cs, Wd, ws=L.empty_workspace(M, N, K, K), bias=bd))
+        assert_status_ok(L, act["ws"])
+    else:
+        if how == "unaligned":
+            wide = np.zeros((M, K + 1), np.float16)
+            wide[:, :K] = X
+            Xd = dev(wide)[:, :K]
+        else:
+            Xd = dev(X)
+        ws = L.empty_workspace(M, N, K, K)
+        Y = host(L.mixed_matmul(Xd, Wq, cs, Wd, 6.0, ws=ws, bias=bd))
+        assert_status_ok(L, ws)
+    r = oracle.mixed_matmul(X, W, 6.0, bias=b)
+    y_close(Y, r["Y"])
+
+
+@pytest.mark.parametrize("keep", [False, True])
+@pytest.mark.parametrize("lead,K,N", [((2, 3), 520, 300), ((4, 50), 1032, 257), ((1,), 4096, 4096)])
+def test_int8_linear_module(L, keep, lead, K, N):
+    """Int8Linear.from_linear on a randomly initialised fp16 nn.Linear:
+    y = x W^T + b through the C ABI, against the oracle (fp16 or int8-only
+    weight reading), for decode- and prefill-shaped inputs with planted
+    outlier features."""
+    torch.manual_seed(K + N)
+    lin = torch.nn.Linear(K, N, bias=True).cuda().half()
+    m = L.Int8Linear.from_linear(lin, 6.0, keep_fp16_weight=keep)
+    M = int(np.prod(lead))
+    rng = np.random.default_rng(M + K)
+    X, _, _ = wl.random_small(rng, M, K, 1, max(1, K // 500))
+    x = dev(X).reshape(*lead, K)
+    y = m(x)
+    assert y.shape == (*lead, N) and y.dtype == torch.float16
+    W = lin.weight.detach().cpu().numpy().T.copy()
+    b = lin.bias.detach().cpu().numpy()
+    r = oracle.mixed_matmul(X, W, 6.0, bias=b, int8_weight=not keep)
+    y_close(host(y).reshape(M, N), r["Y"])
+    fp16_bytes = 2 * K * N
+    assert m.weight_bytes() < (fp16_bytes * 0.55 if not keep else fp16_bytes * 1.6)
