@@ -62,6 +62,7 @@ def _load():
             "oracle_int8_matmul": (None, [P, P, I64, I64, P, I64, P]),
             "oracle_mixed_output": (None, [P, P, P, P, I64, P, I64, P, I64, P, P, I64, P, P]),
             "oracle_dequantize_weight": (None, [P, I64, I64, P, P]),
+            "oracle_outlier_stats": (None, [P, I64, I64, I64, ctypes.c_float, P]),
             "oracle_num_threads": (ctypes.c_int, []),
         }
         for name, (res, args) in sig.items():
@@ -204,6 +205,15 @@ def mixed_output(acc: np.ndarray, rs: np.ndarray, cs: np.ndarray, X: np.ndarray,
     _load().oracle_mixed_output(_p(acc), _p(_c(rs, np.float32)), _p(_c(cs, np.float32)), _p(Xb), K,
                                 _p(Wb), N, _p(O), O.size, _p(bb), _p(rr), n, _p(Yd), _p(Y))
     return Y.view(np.float16), Yd
+
+
+def outlier_stats(X: np.ndarray, tau: float) -> Dict[str, int]:
+    """Outlier values (|x| >= tau), their feature columns and their rows."""
+    Xb = _bits16(X)
+    M, K = Xb.shape
+    out = np.zeros(3, np.int64)
+    _load().oracle_outlier_stats(_p(Xb), M, K, K, ctypes.c_float(tau), _p(out))
+    return {"values": int(out[0]), "columns": int(out[1]), "rows": int(out[2])}
 
 
 def dequantize_weight(Wq: np.ndarray, cs: np.ndarray) -> np.ndarray:

@@ -312,6 +312,40 @@ void oracle_mixed_output(const int64_t* acc, const float* rs, const float* cs, c
 }
 
 /* ------------------------------------------------------------------ */
+/* Outlier statistics of an activation: how many values reach the         */
+/* threshold, in how many feature dimensions (columns) and in how many    */
+/* rows -- the quantities the pages report ("8-bit Matrix Multiplication  */
+/* for Large Language Models", Summary & Methodology Analysis: at 6.7B,   */
+/* 150,000 outliers per sequence, in 6 feature dimensions).               */
+/* ------------------------------------------------------------------ */
+
+/* out[0] = #{(i,k) : |X[i,k]| >= tau}, out[1] = #{k : some |X[i,k]| >= tau},
+ * out[2] = #{i : some |X[i,k]| >= tau}; NaN never counts. */
+void oracle_outlier_stats(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, float tau, int64_t* out)
+{
+    unsigned char* col = (unsigned char*)calloc((size_t)(K > 0 ? K : 1), 1);
+    int64_t values = 0, rows = 0, cols = 0;
+    for (int64_t i = 0; i < M; ++i) {
+        int any = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            double a = fabs(oracle_half_to_double(X[i * ldx + k]));
+            if ((double)tau <= a) {  /* false for NaN */
+                ++values;
+                any = 1;
+                col[k] = 1;
+            }
+        }
+        rows += any;
+    }
+    for (int64_t k = 0; k < K; ++k)
+        cols += col[k];
+    free(col);
+    out[0] = values;
+    out[1] = cols;
+    out[2] = rows;
+}
+
+/* ------------------------------------------------------------------ */
 /* The 16-bit weight rows recovered from the int8 weight, for callers     */
 /* that keep only the int8 form: the point of the method is halving the   */
 /* weight memory ("LLM.int8()" arXiv abstract: inference memory cut by    */

@@ -29,6 +29,7 @@ MUTANTS = {
     "dequantized_weight_scale_128": ("(double)Wq[k * N + j] * (double)cs[j] / 127.0",
                                      "(double)Wq[k * N + j] * (double)cs[j] / 128.0"),
     "bias_indexed_by_row": ("yd[j] += oracle_half_to_double(bias[j]);", "yd[j] += oracle_half_to_double(bias[i % N]);"),
+    "stats_threshold_strict": ("if ((double)tau <= a) {", "if ((double)tau < a) {"),
     "weight_scale_first_rows_only": ("for (int64_t k = 0; k < K; ++k) {\n            float a = fabsf(half_to_float(W[k * N + j]));",
                                      "for (int64_t k = 0; k < (K + 1) / 2; ++k) {\n            float a = fabsf(half_to_float(W[k * N + j]));"),
 }

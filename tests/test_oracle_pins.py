@@ -437,3 +437,38 @@ def test_bias_on_the_fp16_matmul(name, X, W):
     r = oracle.mixed_matmul(X, W, 0.0, bias=b)
     exact = X.astype(np.float64) @ W.astype(np.float64) + b.astype(np.float64)[None, :]
     assert np.allclose(r["Yd"], exact, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ outlier statistics
+
+def test_outlier_stats_on_constructed_placements():
+    """Known placements: 7.0 at listed (row, column) pairs, exactly tau once
+    (counts: the threshold is inclusive), -inf once, a NaN and a value just
+    below tau (neither counts)."""
+    X = np.zeros((10, 50), np.float16)
+    pairs = [(0, 3), (0, 17), (4, 3), (9, 49), (4, 20), (7, 3)]
+    for i, k in pairs:
+        X[i, k] = 7.0
+    X[2, 30] = -np.inf
+    X[5, 5] = np.nan
+    X[6, 8] = np.nextafter(np.float16(6.0), np.float16(0))
+    X[3, 40] = 6.0
+    st = oracle.outlier_stats(X, 6.0)
+    assert st == {"values": 8, "columns": 6, "rows": 6}
+    assert st["columns"] == oracle.outlier_columns(X, 6.0).size
+
+
+def test_outlier_stats_at_tau_limits():
+    X = wl.make_x(wl.get("tiny"))
+    M, K = X.shape
+    assert oracle.outlier_stats(X, 0.0) == {"values": M * K, "columns": K, "rows": M}
+    assert oracle.outlier_stats(X, np.inf) == {"values": 0, "columns": 0, "rows": 0}
+
+
+@pytest.mark.parametrize("name,X,W", _problems())
+def test_outlier_stats_columns_agree_with_the_outlier_set(name, X, W):
+    st = oracle.outlier_stats(X, 6.0)
+    O = oracle.outlier_columns(X, 6.0)
+    assert st["columns"] == O.size
+    assert st["values"] >= st["columns"] and st["values"] >= st["rows"]
+    assert st["values"] <= st["rows"] * max(1, O.size)
