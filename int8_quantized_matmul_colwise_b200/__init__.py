@@ -16,7 +16,7 @@ from typing import Dict, Optional, Tuple
 
 from . import capi
 from .capi import (LLMInt8Error, empty_workspace, llmint8_check_status, llmint8_debug_int8_gemm_i32,
-                   llmint8_mixed_gemm, llmint8_mixed_matmul, llmint8_mixed_matmul_kernels,
+                   llmint8_mixed_gemm, llmint8_mixed_matmul, llmint8_mixed_matmul_kernels, llmint8_outlier_stats,
                    llmint8_quantize_act_rowwise_outliers, llmint8_quantize_weight_colwise,
                    llmint8_status_string, llmint8_workspace_init, llmint8_workspace_layout,
                    llmint8_workspace_size, round_up, workspace_views)
@@ -28,6 +28,7 @@ __all__ = [
     "llmint8_mixed_gemm", "mixed_gemm",
     "llmint8_check_status", "llmint8_debug_int8_gemm_i32", "llmint8_status_string", "llmint8_workspace_size",
     "llmint8_workspace_init", "llmint8_workspace_layout", "llmint8_mixed_matmul_kernels",
+    "llmint8_outlier_stats", "outlier_stats", "Int8Linear",
 ]
 
 
@@ -94,6 +95,19 @@ def mixed_gemm(act: Dict[str, object], Wq, col_scale, W, Y=None, ws=None, stream
     llmint8_mixed_gemm(Xq, act["row_scale"], act["outlier_idx"], act["n_outlier"], act["Xo"], Wq, col_scale, W,
                        K, Y, ws, stream, bias)
     return Y
+
+
+def outlier_stats(X, tau: float = 6.0, ws=None, stream=None) -> Dict[str, int]:
+    """Values with |x| >= tau in X, the feature columns and the rows holding
+    them (reads the three counts back to the host)."""
+    import torch
+    M, K = X.shape
+    if ws is None:
+        ws = empty_workspace(1, 1, K, K, device=X.device)
+    stats = torch.empty(3, dtype=torch.int64, device=X.device)
+    llmint8_outlier_stats(X, tau, stats, ws, stream)
+    v = stats.tolist()
+    return {"values": int(v[0]), "columns": int(v[1]), "rows": int(v[2])}
 
 
 def check_status(ws, stream=None) -> int:

@@ -73,6 +73,7 @@ SIGNATURES = {
                                                             _P, _I64, _P]),
     "llmint8_check_status": (_ST, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "llmint8_mixed_matmul_kernels": (ctypes.c_int, [_I64, _I64, _I64, _I64, _P]),
+    "llmint8_outlier_stats": (_ST, [_P, _I64, _I64, _I64, _F, _P, _P, _SZ, _P]),
     "llmint8_debug_int8_gemm_i32": (_ST, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64, _P, _SZ, _P]),
 }
 
@@ -256,6 +257,18 @@ def llmint8_check_status(ws, stream=None) -> Tuple[int, int]:
     flags = ctypes.c_uint32(0)
     st = lib().llmint8_check_status(_ptr(ws), _stream(stream), ctypes.byref(flags))
     return int(st), int(flags.value)
+
+
+def llmint8_outlier_stats(X, tau: float, stats, ws, stream=None):
+    """stats int64 [3] (device) <- values with |x| >= tau, their columns, their rows."""
+    torch = _torch()
+    _rowmajor(X, "X", torch.float16)
+    _rowmajor(stats, "stats", torch.int64, 1)
+    if stats.numel() != 3:
+        raise ValueError("stats: expected 3 elements")
+    M, K = X.shape
+    _check(lib().llmint8_outlier_stats(_ptr(X), M, K, _ld(X), float(tau), _ptr(stats), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)), "llmint8_outlier_stats")
 
 
 def llmint8_mixed_matmul_kernels(X, N: int) -> int:

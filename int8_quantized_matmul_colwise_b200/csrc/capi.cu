@@ -124,7 +124,8 @@ bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t
   off = align_up(off + 4 * size_t((K + 255) / 256), 256);  // block counters follow colmax
   *bitmask = off;
   off = align_up(off + 4 * size_t((K + 31) / 32), 256);
-  off += act_fused_bytes(K);  // the one-kernel activation step's counters and bitmasks
+  off += act_fused_bytes(K);      // the one-kernel activation step's counters and bitmasks
+  off += stats_scratch_bytes(K);  // the outlier statistics' bitmask and counters
   L->status = 0;
   L->n_outlier = 8;
   L->outlier_idx = off;
@@ -198,6 +199,24 @@ llmint8_status llmint8_workspace_layout(int64_t M, int64_t N, int64_t K, int64_t
   size_t c, b, d;
   if (!make_layout(M, K, outlier_cap, out, &c, &b, N, &d)) return LLMINT8_ERR_INVALID_ARG;
   return LLMINT8_OK;
+}
+
+llmint8_status llmint8_outlier_stats(const void* X, int64_t M, int64_t K, int64_t ldx, float tau, int64_t* stats,
+                                     void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !stats) return LLMINT8_ERR_INVALID_ARG;
+  if (M < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || ldx < K || !valid_tau(tau))
+    return LLMINT8_ERR_INVALID_ARG;
+  if (!aligned(X, 2) || !aligned(stats, 8)) return LLMINT8_ERR_INVALID_ARG;
+  llmint8_ws_layout L;
+  size_t colmax, bitmask;
+  if (!make_layout(1, K, 1, &L, &colmax, &bitmask)) return LLMINT8_ERR_INVALID_ARG;
+  const size_t scratch_off = align_up(bitmask + 4 * size_t((K + 31) / 32), 256) + act_fused_bytes(K);
+  if (!ws || !aligned(ws, 256) || ws_bytes < scratch_off + stats_scratch_bytes(K)) return LLMINT8_ERR_WORKSPACE;
+  int num_sms = 0;
+  llmint8_status st = current_device(&num_sms);
+  if (st != LLMINT8_OK) return st;
+  uint32_t* scratch = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + scratch_off);
+  return cuda_status(launch_outlier_stats(X, M, K, ldx, tau, scratch, stats, num_sms, static_cast<cudaStream_t>(stream)));
 }
 
 int llmint8_mixed_matmul_kernels(int64_t M, int64_t N, int64_t K, int64_t ldx, const void* X) {

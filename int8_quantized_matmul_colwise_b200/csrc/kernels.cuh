@@ -24,6 +24,15 @@ struct ActWs {
 // Bytes of ActWs::fused for K columns (256-byte multiple).
 inline size_t act_fused_bytes(int64_t K) { return (16 + 8 * size_t((K + 31) / 32) + 255) / 256 * 256; }
 
+// Outlier statistics scratch (zero between calls): a column bitmask of
+// ceil(K/32) words, then three 64-bit counters (values, rows, CTAs done).
+inline size_t stats_scratch_bytes(int64_t K) {
+  return (8 * size_t(((K + 31) / 32 + 1) / 2) + 24 + 255) / 256 * 256;
+}
+// stats: int64 [3] (device) <- values with |x| >= tau, their columns, their rows.
+cudaError_t launch_outlier_stats(const void* X, int64_t M, int64_t K, int64_t ldx, float tau, uint32_t* scratch,
+                                 int64_t* stats, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_quantize_weight_colwise(const void* W, int64_t K, int64_t N, int64_t ldw, int8_t* Wq,
                                            int64_t ldk, float* col_scale, cudaStream_t stream);
 

@@ -551,6 +551,90 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
   }
 }
 
+// ----------------------------------------------------------------- outlier statistics
+// Values with |x| >= tau, the feature columns they fall in, and the rows that
+// hold one -- the quantities the pages report ("8-bit Matrix Multiplication
+// for Large Language Models", Summary & Methodology Analysis: 150,000 outliers
+// per sequence in 6 feature dimensions at 6.7B).  Rows are split over the
+// CTAs; the column bitmask and the counters live in a workspace scratch that
+// is zero between calls, and the last CTA counts the bitmask, writes the three
+// numbers and returns the scratch to zero.
+template <bool kVec>
+__global__ void __launch_bounds__(256) outlier_stats_kernel(const __half* __restrict__ X, int64_t M, int64_t K,
+                                                            int64_t ldx, float tau, int rows_per,
+                                                            uint32_t* __restrict__ scratch,
+                                                            int64_t* __restrict__ stats) {
+  __shared__ unsigned long long s_val[8];
+  __shared__ int s_last;
+  const int nwords = static_cast<int>((K + 31) / 32);
+  uint32_t* mask = scratch;
+  unsigned long long* cnt = reinterpret_cast<unsigned long long*>(scratch + ((nwords + 1) & ~1));
+  griddep_wait();
+  griddep_launch_dependents();
+
+  unsigned long long my_values = 0;
+  unsigned long long my_rows = 0;
+  const int64_t r0 = int64_t(blockIdx.x) * rows_per;
+  const int64_t r1 = min(M, r0 + rows_per);
+  for (int64_t r = r0; r < r1; ++r) {
+    const __half* xr = X + r * ldx;
+    int any = 0;
+    for (int64_t c = 8 * int64_t(threadIdx.x); c < K; c += 8 * 256) {
+      const uint4 u = load8_packed<kVec>(xr, K, c);
+      uint32_t fl = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float a = fabsf(__half2float(__ushort_as_half(half_bits_at(u, e))));
+        if (c + e < K && a >= tau) fl |= 1u << e;  // false for NaN
+      }
+      if (fl != 0u) {
+        my_values += __popc(fl);
+        any = 1;
+        atomicOr(mask + (c >> 5), fl << (c & 31));
+      }
+    }
+    if (__syncthreads_or(any) && threadIdx.x == 0) ++my_rows;
+  }
+  // this CTA's value count
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) my_values += __shfl_down_sync(0xffffffffu, my_values, o);
+  if ((threadIdx.x & 31) == 0) s_val[threadIdx.x >> 5] = my_values;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long v = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += s_val[w];
+    if (v) atomicAdd(cnt + 0, v);
+    if (my_rows) atomicAdd(cnt + 1, my_rows);
+    __threadfence();
+    s_last = atomicAdd(cnt + 2, 1ull) == static_cast<unsigned long long>(gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  int cols = 0;
+  for (int w = threadIdx.x; w < nwords; w += 256) {
+    cols += __popc(__ldcg(mask + w));
+    mask[w] = 0u;  // zero for the next call
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cols += __shfl_down_sync(0xffffffffu, cols, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) s_val[threadIdx.x >> 5] = static_cast<unsigned long long>(cols);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long c = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) c += s_val[w];
+    stats[0] = static_cast<int64_t>(__ldcg(cnt + 0));
+    stats[1] = static_cast<int64_t>(c);
+    stats[2] = static_cast<int64_t>(__ldcg(cnt + 1));
+    cnt[0] = 0ull;
+    cnt[1] = 0ull;
+    cnt[2] = 0ull;
+  }
+}
+
 // Rows too long for the register-resident kernel (K > 16384): one CTA per row,
 // two passes over the row.
 __global__ void __launch_bounds__(256) quantize_rows_long_kernel(const __half* __restrict__ X, int64_t M,
@@ -716,6 +800,27 @@ cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx
   cfg.gridDim = dim3(static_cast<unsigned>(M));
   return cudaLaunchKernelEx(&cfg, quantize_rows_long_kernel, x, M, K, ldx, tau, ws, O, n_out, cap, Xq, ldq, rs, xo,
                             ldo);
+}
+
+cudaError_t launch_outlier_stats(const void* X, int64_t M, int64_t K, int64_t ldx, float tau, uint32_t* scratch,
+                                 int64_t* stats, int num_sms, cudaStream_t stream) {
+  const __half* x = static_cast<const __half*>(X);
+  const bool vec_ok = (ldx % 8 == 0) && (K % 8 == 0) && (reinterpret_cast<uintptr_t>(X) % 16 == 0);
+  const int64_t target = int64_t(num_sms > 0 ? num_sms : 148) * 4;  // CTAs
+  const int64_t rows_per = (M + target - 1) / target;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((M + rows_per - 1) / rows_per));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return vec_ok ? cudaLaunchKernelEx(&cfg, outlier_stats_kernel<true>, x, M, K, ldx, tau, static_cast<int>(rows_per),
+                                     scratch, stats)
+                : cudaLaunchKernelEx(&cfg, outlier_stats_kernel<false>, x, M, K, ldx, tau,
+                                     static_cast<int>(rows_per), scratch, stats);
 }
 
 }  // namespace llmint8

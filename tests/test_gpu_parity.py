@@ -534,3 +534,27 @@ def test_int8_linear_module(L, keep, lead, K, N):
     y_close(host(y).reshape(M, N), r["Y"])
     fp16_bytes = 2 * K * N
     assert m.weight_bytes() < (fp16_bytes * 0.55 if not keep else fp16_bytes * 1.6)
+
+
+# ------------------------------------------------------------------ outlier statistics
+
+@pytest.mark.parametrize("name", ["tiny", "decode_m8", "ffn_6p7b_prefill", "ragged_2047x4095x4100", "ragged_3x33x24",
+                                  "sweep8k_o1"])
+def test_outlier_stats_exact(L, name):
+    """The three counts equal the oracle's (integers: exact), for tau 6, 0
+    (every value), +inf (none), and twice through one workspace (the scratch
+    is returned to zero)."""
+    w = wl.get(name)
+    X = wl.make_x(w)
+    Xd = dev(X)
+    ws = L.empty_workspace(1, 1, w.K, w.K)
+    for tau in (w.tau, 0.0, np.inf, w.tau):
+        assert L.outlier_stats(Xd, tau, ws=ws) == oracle.outlier_stats(X, tau), tau
+
+
+def test_outlier_stats_strided_rows(L):
+    X = wl.make_x(wl.get("ragged_129x257x520"))
+    wide = np.zeros((X.shape[0], X.shape[1] + 3), np.float16)
+    wide[:, 1:1 + X.shape[1]] = X
+    t = dev(wide)[:, 1:1 + X.shape[1]]
+    assert L.outlier_stats(t, 6.0) == oracle.outlier_stats(X, 6.0)
