@@ -139,22 +139,33 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ distributed plumbing
 class Dist:
-    def __init__(self):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE): NCCL
+    on GPUs; gloo when no GPU is present (the host-side logic under CPU
+    tests).  Only used for the barrier around the timed region and the
+    max-over-ranks of the timings: the path itself needs no exchange."""
+
+    def __init__(self, backend=None):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
         self.pg = None
 
     def init(self, torch):
+        backend = self.backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        self.backend = backend
         if self.world > 1:
             import datetime
 
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                    device_id=torch.device("cuda", self.local))
+            timeout = datetime.timedelta(seconds=120)  # ranks that wait on a lost peer end with an error
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", self.local))
+            else:
+                dist.init_process_group(backend, timeout=timeout)
             self.pg = dist
-        else:
+        elif backend == "nccl":
             torch.cuda.set_device(0)
 
     def barrier(self, torch):
@@ -164,7 +175,7 @@ class Dist:
     def max(self, torch, v: float) -> float:
         if not self.pg:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device="cuda" if self.backend == "nccl" else "cpu")
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
