@@ -534,7 +534,7 @@ def run_ours(args, wl_, dist):
                   f"> 3x L2; consecutive steps touch different buffers",
             "weight_quant_ms_offline": wq_ms, "workspace_bytes": ws_bytes,
             "launch": ("llmint8_mixed_matmul: 1 kernel (a1-a7 fused)" if n_kern == 1 else
-                       "llmint8_mixed_matmul: 3 kernels chained with programmatic dependent launch") +
+                       f"llmint8_mixed_matmul: {n_kern} kernels chained with programmatic dependent launch") +
                       ("; the K steps replayed from one CUDA graph" if args.graph else "")}),
         "roofline": roofline, "path_roofline": path, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": n_kern * args.steps, "clocks": clk,

@@ -225,7 +225,8 @@ int llmint8_mixed_matmul_kernels(int64_t M, int64_t N, int64_t K, int64_t ldx, c
     return 0;
   int num_sms = 0, s = 0, kb = 0, stages = 0;
   if (current_device(&num_sms) != LLMINT8_OK) return 0;
-  return use_fused_decode(M, N, K, ldx, X, num_sms, &s, &kb, &stages) ? 1 : 3;
+  if (use_fused_decode(M, N, K, ldx, X, num_sms, &s, &kb, &stages)) return 1;
+  return act_fused_plan(M, K, ldx, X, num_sms) ? 2 : 3;  // activation step in one or two kernels, then the GEMM
 }
 
 size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K, int64_t outlier_cap) {

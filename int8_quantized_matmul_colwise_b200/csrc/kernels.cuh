@@ -36,6 +36,10 @@ cudaError_t launch_outlier_stats(const void* X, int64_t M, int64_t K, int64_t ld
 cudaError_t launch_quantize_weight_colwise(const void* W, int64_t K, int64_t N, int64_t ldw, int8_t* Wq,
                                            int64_t ldk, float* col_scale, cudaStream_t stream);
 
+// Whether the activation step for these arguments runs as one kernel (X fits
+// in shared memory spread over num_sms CTAs and its rows allow 16-byte loads).
+bool act_fused_plan(int64_t M, int64_t K, int64_t ldx, const void* X, int num_sms);
+
 // num_sms > 0 and ws.fused set: shapes whose X fits in shared memory across
 // the SMs run as one persistent kernel (grid barrier between the column scan
 // and the row quantization); otherwise two kernels.

@@ -721,6 +721,19 @@ cudaError_t launch_rows(cudaLaunchConfig_t& cfg, int64_t M, const __half* x, int
 
 }  // namespace
 
+bool act_fused_plan(int64_t M, int64_t K, int64_t ldx, const void* X, int num_sms) {
+  if (num_sms <= 0 || ldx % 8 != 0 || K % 8 != 0 || reinterpret_cast<uintptr_t>(X) % 16 != 0) return false;
+  const int64_t rows_per = (M + num_sms - 1) / num_sms;
+  const int64_t cpad = ((K / 8) + 31) / 32 * 32;  // chunks padded to whole warps
+  if (cpad > kActFusedThreads) return false;
+  const int64_t groups = kActFusedThreads / cpad;
+  const int64_t r = (rows_per + groups - 1) / groups;
+  const size_t mask_bytes = static_cast<size_t>((K + 31) / 32) * sizeof(uint32_t);
+  const size_t smem = size_t(rows_per) * size_t(K) * 2 + 2 * ((mask_bytes + 15) / 16 * 16) +
+                      size_t(kActFusedThreads) * 16;
+  return r <= 8 && rows_per <= kActFusedMaxRows && smem <= kActFusedSmemMax;
+}
+
 cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx, float tau, int8_t* Xq,
                                 int64_t ldq, float* rs, int32_t* O, int64_t cap, int32_t* n_out, void* Xo,
                                 int64_t ldo, ActWs ws, cudaStream_t stream, bool pdl, int num_sms) {
@@ -739,34 +752,30 @@ cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx
   cfg.numAttrs = pdl ? 1 : 0;
 
   // One kernel when X fits in shared memory over at most num_sms CTAs.
-  if (ws.fused != nullptr && num_sms > 0 && vec_ok) {
+  if (ws.fused != nullptr && act_fused_plan(M, K, ldx, X, num_sms)) {
     const int64_t rows_per = (M + num_sms - 1) / num_sms;
     const int64_t cpad = ((K / 8) + 31) / 32 * 32;  // chunks padded to whole warps
-    const int64_t groups = cpad <= kActFusedThreads ? kActFusedThreads / cpad : 0;
-    const int64_t r = groups > 0 ? (rows_per + groups - 1) / groups : 0;
+    const int64_t r = (rows_per + kActFusedThreads / cpad - 1) / (kActFusedThreads / cpad);  // rows per thread
     const size_t smem = size_t(rows_per) * size_t(K) * 2 + 2 * ((mask_bytes + 15) / 16 * 16) +
                         size_t(kActFusedThreads) * 16;
-    if (groups > 0 && r <= 8 && rows_per <= kActFusedMaxRows && smem <= kActFusedSmemMax) {
-      const int rt = r <= 1 ? 1 : r <= 2 ? 2 : r <= 4 ? 4 : 8;
-      auto kern = rt == 1 ? act_fused_kernel<1> : rt == 2 ? act_fused_kernel<2> : rt == 4 ? act_fused_kernel<4>
-                                                                                            : act_fused_kernel<8>;
-      static bool attr_set[4][64] = {};
-      const int ri = rt == 1 ? 0 : rt == 2 ? 1 : rt == 4 ? 2 : 3;
-      int dev = 0;
-      cudaError_t e = cudaGetDevice(&dev);
+    const int ri = r <= 1 ? 0 : r <= 2 ? 1 : r <= 4 ? 2 : 3;
+    auto kern = ri == 0 ? act_fused_kernel<1> : ri == 1 ? act_fused_kernel<2> : ri == 2 ? act_fused_kernel<4>
+                                                                                        : act_fused_kernel<8>;
+    static bool attr_set[4][64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[ri][dev]) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kActFusedSmemMax));
       if (e != cudaSuccess) return e;
-      if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-      if (!attr_set[ri][dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kActFusedSmemMax));
-        if (e != cudaSuccess) return e;
-        attr_set[ri][dev] = true;
-      }
-      cfg.blockDim = dim3(kActFusedThreads);
-      cfg.gridDim = dim3(static_cast<unsigned>((M + rows_per - 1) / rows_per));
-      cfg.dynamicSmemBytes = smem;
-      return cudaLaunchKernelEx(&cfg, kern, x, M, K, ldx, tau, ws, O, n_out, cap, Xq, ldq, rs,
-                                static_cast<__half*>(Xo), ldo, static_cast<int>(rows_per), static_cast<int>(cpad));
+      attr_set[ri][dev] = true;
     }
+    cfg.blockDim = dim3(kActFusedThreads);
+    cfg.gridDim = dim3(static_cast<unsigned>((M + rows_per - 1) / rows_per));
+    cfg.dynamicSmemBytes = smem;
+    return cudaLaunchKernelEx(&cfg, kern, x, M, K, ldx, tau, ws, O, n_out, cap, Xq, ldq, rs, static_cast<__half*>(Xo),
+                              ldo, static_cast<int>(rows_per), static_cast<int>(cpad));
   }
 
   cfg.gridDim = dim3(static_cast<unsigned>((K + kScanCols - 1) / kScanCols),

@@ -558,3 +558,16 @@ def test_outlier_stats_strided_rows(L):
     wide[:, 1:1 + X.shape[1]] = X
     t = dev(wide)[:, 1:1 + X.shape[1]]
     assert L.outlier_stats(t, 6.0) == oracle.outlier_stats(X, 6.0)
+
+
+def test_kernel_count_query(L):
+    """llmint8_mixed_matmul_kernels: 1 on the one-kernel decode path, 2 when
+    the activation step is one kernel, 3 otherwise."""
+    def count(M, N, K, ldx=None):
+        ldx = K if ldx is None else ldx
+        X = torch.empty((M, ldx), dtype=torch.float16, device="cuda")[:, :K]
+        return L.llmint8_mixed_matmul_kernels(X, N)
+    assert count(8, 4096, 4096) == 1
+    assert count(2048, 16384, 4096) == 2
+    assert count(8192, 8192, 8192) == 3        # X too large for shared memory
+    assert count(100, 300, 1000, ldx=1001) == 3  # rows not 16-byte aligned
