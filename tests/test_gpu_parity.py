@@ -571,3 +571,26 @@ def test_kernel_count_query(L):
     assert count(2048, 16384, 4096) == 2
     assert count(8192, 8192, 8192) == 3        # X too large for shared memory
     assert count(100, 300, 1000, ldx=1001) == 3  # rows not 16-byte aligned
+
+
+@pytest.mark.parametrize("name", ["ragged_1000x1000x1000", "ffn_6p7b_prefill"])
+def test_outlier_overflow_on_the_prefill_path(L, name):
+    """A cap below n_o through the one-kernel activation step and the tcgen05
+    GEMM: the status bit, the true count and a NaN-filled Y."""
+    w = wl.get(name)
+    X, W = wl.make_inputs(w)
+    n_true = oracle.outlier_columns(X, w.tau).size
+    assert n_true >= 2
+    Y, ws, v, _, (st, flags) = run_path(L, X, W, w.tau, cap=1)
+    assert st == 5 and flags & 1
+    assert int(host(v["n_outlier"])[0]) == n_true
+    assert np.isnan(host(Y).astype(np.float32)).all()
+
+
+@pytest.mark.parametrize("M,N,K", [(40, 72, 20000), (5, 130, 20000)])
+def test_rows_longer_than_16384(L, M, N, K):
+    """K > 16384: the long-row activation kernel (prefill) and the three-kernel
+    decode path (the one-kernel plan stops at K = 16384)."""
+    rng = np.random.default_rng(K + M)
+    X, W, _ = wl.random_small(rng, M, K, N, 20)
+    check_path(L, X, W, 6.0)
