@@ -164,6 +164,37 @@ struct FusedArgs {
   int stages;  // Wq ring depth: 4 (two CTAs per SM) or 8
 };
 
+// ------------------------------------------------------------------ decode as a matrix-vector product (M <= 8)
+struct GemvArgs {
+  const void* X;  // fp16 [M, ldx], rows 16-byte aligned
+  int64_t ldx;
+  int M, N;
+  int64_t K;      // K % 512 == 0, K <= 4096
+  float tau;
+  const float* cs;
+  const void* W;  // fp16 [K, ldw] outlier rows, or nullptr (recovered from Wq)
+  int64_t ldw;
+  const int8_t* Wq;  // int8 [N, ldk]
+  int64_t ldk;
+  const void* bias;  // fp16 [N] or nullptr
+  void* Y;
+  int64_t ldy;
+  int8_t* Xq;  // workspace outputs, written by the first CTA
+  int64_t ldq;
+  float* rs;
+  int32_t* O;
+  int32_t* n_out;
+  void* Xo;
+  int64_t ldo;
+  int cap;
+  uint32_t* status;
+  int rows_per;  // Wq rows per CTA
+  int tiles;     // 16-row MMA tiles covering rows_per (at most 4)
+};
+// Rows per CTA and tiles for a call; false if this kernel does not take the shape.
+bool decode_gemv_plan(int M, int N, int K, int64_t ldk, int num_sms, int* rows_per, int* tiles);
+cudaError_t launch_decode_gemv(const GemvArgs& a, cudaStream_t stream, bool pdl);
+
 // Cluster size and K blocks per CTA for a decode call; false if the fused
 // kernel does not take this shape (the caller then runs the three-kernel path).
 bool decode_fused_plan(int M, int N, int K, int num_sms, int* splits, int* kb_per, int* stages);

@@ -149,6 +149,12 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu_u32(const uint32_t* p) {
 }
 
 // Prefetch a 2D tile of a tensor into L2 (no shared memory, no completion).
+// Hint: bring the line holding p into L1 (no register written, no fault on
+// the hint itself for a valid global address).
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
 __device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int32_t x, int32_t y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
                    reinterpret_cast<uint64_t>(tmap)),
@@ -412,6 +418,18 @@ __device__ __forceinline__ void mma_m16n8k16_f16f32(float (&d)[4], const uint32_
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Warp-level int8 MMA, 16 x 8 x 32, int32 accumulate.  Lane l (g = l / 4,
+// t = l % 4) holds A rows g and g + 8 at K bytes 4t..4t+3 (a0, a1) and
+// 16+4t.. (a2, a3); B column g at K bytes 4t.. (b0) and 16+4t.. (b1); D rows g
+// and g + 8 at columns 2t, 2t + 1 (d0, d1 / d2, d3).
+__device__ __forceinline__ void mma_m16n8k32_s8s32(int32_t (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                   uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 // Four transposed 8x8 fp16 tiles from shared memory (lane l gives the row
