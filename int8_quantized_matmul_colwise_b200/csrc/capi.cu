@@ -168,10 +168,10 @@ llmint8_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK
 bool valid_tau(float tau) { return !std::isnan(tau) && tau >= 0.0f; }
 
 // Whether llmint8_mixed_matmul runs the matrix-vector decode kernel (M <= 8).
-// Rows of X up to which the matrix-vector kernel beats the cluster kernel on
-// the 4096 x 4096 decode shape (5.7 us at one row, 11.9 us at eight, against
-// 10.4-11.2 us for the cluster kernel at any row count up to eight).
-constexpr int64_t kGemvMaxM = 4;
+// Rows of X the matrix-vector kernel takes.  It needs K a multiple of 512 up
+// to 4096 and at most 64 Wq rows per SM; other decode calls take the cluster
+// kernel, which costs about the same at any row count up to 32.
+constexpr int64_t kGemvMaxM = 8;
 
 bool use_gemv_decode(int64_t M, int64_t N, int64_t K, int64_t ldx, int64_t ldk, const void* X, int num_sms,
                      int* rows_per, int* tiles) {

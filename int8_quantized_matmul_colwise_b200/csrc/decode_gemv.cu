@@ -19,13 +19,16 @@
 // The activation step runs in registers.  Warp w owns the columns
 // [K/8 w, K/8 (w+1)); lane L of it holds 16 consecutive columns for all M rows,
 // flags the columns with |x| >= tau in some row, and takes the row maxima over
-// the rest; one barrier combines the warps' maxima into the row scales.  The
-// lane then quantizes its columns and hands the codes to the lanes that use
-// them as the B operand of the warp-level int8 MMA (m16n8k32, the X rows as
-// the N side).  The MMA fragments are loaded 16 bytes at a time: inside each
-// 64-column chunk, lane quarter t supplies columns 16t..16t+15, for both
-// operands alike, so the products pair the same columns of Wq and Xq and the
-// int32 sums are exact.  The warps' partial sums are added in shared memory
+// the rest; one barrier combines the warps' maxima into the row scales, and
+// the lane quantizes its columns.  With at most four rows of X the lane then
+// takes the dot products of its own columns with every Wq row on the CUDA
+// cores (dp4a) and the warp adds them across its lanes.  With more rows the
+// codes go to the lanes that use them as the B operand of the warp-level int8
+// MMA (m16n8k32, the X rows as the N side), whose fragments are loaded 16
+// bytes at a time: inside each 64-column chunk, lane quarter t supplies
+// columns 16t..16t+15, for both operands alike, so the products pair the same
+// columns of Wq and Xq.  The int32 sums are exact either way.  The warps'
+// partial sums are added in shared memory
 // (the weight's space, once it has been used), and one thread per output
 // dequantizes, adds the 16-bit outlier product in ascending outlier order and
 // the bias, and stores Y.  The first CTA also writes Xq, rs, O, n_o and Xo to
@@ -46,7 +49,7 @@ constexpr int kRowsV = 8;       // rows of X: the MMA's N
 constexpr int kChunksV = 8;     // 64-column chunks per warp at most: K <= 4096
 constexpr int kTilesV = 4;      // 16-row tiles of Wq per CTA at most
 constexpr int kListV = 32;      // outlier columns listed in shared memory
-constexpr int kPreV = 8;        // outlier terms whose 16-bit weights are prefetched, per output
+constexpr int kPreV = 8;        // outlier terms whose operands are loaded ahead of the MMA, per output
 
 // Byte offsets in the dynamic shared memory.
 struct LayoutV {
@@ -90,11 +93,36 @@ __device__ __noinline__ int outlier_col_at(int t, const uint32_t* s_mask, int nw
   return 0;
 }
 
+// Sum of R per-lane values over the 32 lanes, halving the vector at each
+// step: afterwards the lane holds the total of value `row` (lanes that agree
+// on the bits above 32 / R hold the same value).
+template <int R>
+__device__ __forceinline__ int32_t rows_sum_transposed(int32_t (&v)[R], int lane, int& row) {
+  int o = 16;
+  row = 0;
+#pragma unroll
+  for (int half = R >> 1; half > 0; half >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < half; ++j) {
+      const int32_t mine = up ? v[j + half] : v[j];
+      const int32_t other = up ? v[j] : v[j + half];
+      v[j] = mine + __shfl_xor_sync(0xffffffffu, other, o);
+    }
+    row += up ? half : 0;
+    o >>= 1;
+  }
+  int32_t x = v[0];
+  for (; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
 // MR: rows of X (1..8), a template parameter so that every per-row loop is
 // straight code of the right length.
 template <int MR>
 __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArgs p) {
   constexpr int RP = MR <= 1 ? 1 : MR <= 2 ? 2 : MR <= 4 ? 4 : 8;  // rows rounded up to a power of two
+  constexpr bool kDp4a = MR <= 4;  // products by dp4a on the CUDA cores, else warp-level MMAs
   extern __shared__ __align__(128) uint8_t smem_v[];
   const int64_t K = p.K;
   const int64_t ldk = p.ldk;
@@ -288,59 +316,135 @@ __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArg
   __syncthreads();  // the outlier list
 
   // output (row r of this CTA, X row m) of this thread: warp w takes X row
-  // w % MR and the Wq rows lane + 32 (w / MR) + 32 G i
+  // w % MR and the Wq rows lane + 32 (w / MR) + 32 G i, i = 0, 1
   constexpr int G = kWarpsV / MR;  // warps per X row
   const int em = warp % MR;
   const int eg = warp / MR;
   const bool eact = eg < G;
   const int n_use = overflow ? 0 : n_o;
   const __half* W = static_cast<const __half*>(p.W);
-  // the operands of the first outlier terms into L1 while the MMAs run
-  if (eact && W != nullptr) {
-#pragma unroll 1
-    for (int r = lane + 32 * eg; r < rb; r += 32 * G) {
-#pragma unroll 1
-      for (int t = 0; t < min(n_use, kPreV); ++t) prefetch_l1(W + int64_t(s_list[t]) * p.ldw + n0 + r);
+  const __half* bias = static_cast<const __half*>(p.bias);
+  // the epilogue's operands from global memory, loaded while the MMAs run:
+  // column scales, bias, and the first outlier terms' x and 16-bit w
+  const int npre = W != nullptr ? min(n_use, kPreV) : 0;
+  float csw[2] = {0.0f, 0.0f}, bv[2] = {0.0f, 0.0f};
+  __half px[kPreV], pw[2][kPreV];
+#pragma unroll
+  for (int t = 0; t < kPreV; ++t) px[t] = pw[0][t] = pw[1][t] = __ushort_as_half(0);
+  if (eact) {
+#pragma unroll
+    for (int t = 0; t < kPreV; ++t)
+      if (t < npre) px[t] = X[int64_t(em) * p.ldx + s_list[t]];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int r = lane + 32 * (eg + G * i);
+      if (r < rb) {
+        const int n = n0 + r;
+        csw[i] = __ldg(p.cs + n);
+        if (bias != nullptr) bv[i] = __half2float(bias[n]);
+#pragma unroll
+        for (int t = 0; t < kPreV; ++t)
+          if (t < npre) pw[i][t] = W[int64_t(s_list[t]) * p.ldw + n];
+      }
     }
   }
 
-  // a5: int8 products of this warp's chunks for every tile of the CTA's rows;
-  // the B fragment of chunk c (row g, columns 64 ch + 16 t4 .. + 15) comes
-  // from lane 4c + t4, which quantized those columns
+  // a5: int8 products
   const bool wok = mbar_wait(wbar, 0, p.status);
   int32_t d[kTilesV][4];
 #pragma unroll
   for (int tl = 0; tl < kTilesV; ++tl) d[tl][0] = d[tl][1] = d[tl][2] = d[tl][3] = 0;
-  int ra[kTilesV], rc[kTilesV];  // rows past this CTA's read row rb - 1 (in bounds; their sums are not used)
+  // few rows of X: each lane takes the dot products of its own 16 columns
+  // with every Wq row (dp4a), then the warp sums them over its lanes, in
+  // groups of RG Wq rows (lane L ends with row RG gi + (L >> (5 - log2 RG)))
+  constexpr int RG = MR <= 2 ? 32 : 16;       // Wq rows per group
+  constexpr int NG = 64 / RG;                 // groups at most (rows_per <= 64)
+  constexpr int SH = RG == 32 ? 0 : 1;        // lane bits below the row index
+  int32_t rsum[NG][MR];
 #pragma unroll
-  for (int tl = 0; tl < kTilesV; ++tl) {
-    ra[tl] = min(tl * 16 + g, rb - 1);
-    rc[tl] = min(tl * 16 + g + 8, rb - 1);
-  }
+  for (int gi = 0; gi < NG; ++gi)
+#pragma unroll
+    for (int j = 0; j < MR; ++j) rsum[gi][j] = 0;
+  if constexpr (kDp4a) {
 #pragma unroll 1
-  for (int c = 0; c < S; ++c) {
-    uint32_t bq[4];
+    for (int gi = 0; gi < (rb + RG - 1) / RG; ++gi) {
+      int32_t acc[MR][RG];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      uint32_t v = 0u;
+      for (int rr = 0; rr < RG; ++rr) {
+        const int r = min(RG * gi + rr, rb - 1);  // rows past rb read row rb - 1, unused
+        const uint4 wv = *reinterpret_cast<const uint4*>(sW + int64_t(r) * ldk + (act ? c0 : 0));
+#pragma unroll
+        for (int j = 0; j < MR; ++j) {
+          int32_t a = __dp4a(static_cast<int>(wv.x), static_cast<int>(q[j][0]), 0);
+          a = __dp4a(static_cast<int>(wv.y), static_cast<int>(q[j][1]), a);
+          a = __dp4a(static_cast<int>(wv.z), static_cast<int>(q[j][2]), a);
+          acc[j][rr] = __dp4a(static_cast<int>(wv.w), static_cast<int>(q[j][3]), a);
+        }
+      }
 #pragma unroll
       for (int j = 0; j < MR; ++j) {
-        const uint32_t u = __shfl_sync(0xffffffffu, q[j][r], 4 * c + t4);
-        v = g == j ? u : v;
+        int row = 0;
+        const int32_t tot = rows_sum_transposed<RG>(acc[j], lane, row);
+#pragma unroll
+        for (int k = 0; k < NG; ++k) rsum[k][j] = gi == k ? tot : rsum[k][j];
       }
-      bq[r] = v;
     }
-    const int64_t kof = 64 * int64_t(S * warp + c) + 16 * t4;
+  } else {
+    // the B fragment of chunk c (row g, columns 64 ch + 16 t4 .. + 15) comes
+    // from lane 4c + t4, which quantized those columns; even and odd chunks
+    // accumulate apart (two independent MMA chains per tile)
+    int32_t e[kTilesV][4];
+#pragma unroll
+    for (int tl = 0; tl < kTilesV; ++tl) e[tl][0] = e[tl][1] = e[tl][2] = e[tl][3] = 0;
+    int ra[kTilesV], rc[kTilesV];  // rows past this CTA's read row rb - 1 (in bounds; their sums are not used)
 #pragma unroll
     for (int tl = 0; tl < kTilesV; ++tl) {
-      if (tl < T) {
-        const uint4 ua = *reinterpret_cast<const uint4*>(sW + int64_t(ra[tl]) * ldk + kof);
-        const uint4 uc = *reinterpret_cast<const uint4*>(sW + int64_t(rc[tl]) * ldk + kof);
-        const uint32_t a0[4] = {ua.x, uc.x, ua.y, uc.y};
-        const uint32_t a1[4] = {ua.z, uc.z, ua.w, uc.w};
-        mma_m16n8k32_s8s32(d[tl], a0, bq[0], bq[1]);
-        mma_m16n8k32_s8s32(d[tl], a1, bq[2], bq[3]);
+      ra[tl] = min(tl * 16 + g, rb - 1);
+      rc[tl] = min(tl * 16 + g + 8, rb - 1);
+    }
+#pragma unroll 1
+    for (int c = 0; c < S; c += 2) {
+#pragma unroll
+      for (int hc = 0; hc < 2; ++hc) {
+        const int cc = c + hc;
+        if (cc < S) {
+          uint32_t bq[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            uint32_t v = 0u;
+#pragma unroll
+            for (int j = 0; j < MR; ++j) {
+              const uint32_t u = __shfl_sync(0xffffffffu, q[j][r], 4 * cc + t4);
+              v = g == j ? u : v;
+            }
+            bq[r] = v;
+          }
+          const int64_t kof = 64 * int64_t(S * warp + cc) + 16 * t4;
+#pragma unroll
+          for (int tl = 0; tl < kTilesV; ++tl) {
+            if (tl < T) {
+              const uint4 ua = *reinterpret_cast<const uint4*>(sW + int64_t(ra[tl]) * ldk + kof);
+              const uint4 uc = *reinterpret_cast<const uint4*>(sW + int64_t(rc[tl]) * ldk + kof);
+              const uint32_t a0[4] = {ua.x, uc.x, ua.y, uc.y};
+              const uint32_t a1[4] = {ua.z, uc.z, ua.w, uc.w};
+              if (hc == 0) {
+                mma_m16n8k32_s8s32(d[tl], a0, bq[0], bq[1]);
+                mma_m16n8k32_s8s32(d[tl], a1, bq[2], bq[3]);
+              } else {
+                mma_m16n8k32_s8s32(e[tl], a0, bq[0], bq[1]);
+                mma_m16n8k32_s8s32(e[tl], a1, bq[2], bq[3]);
+              }
+            }
+          }
+        }
       }
+    }
+#pragma unroll
+    for (int tl = 0; tl < kTilesV; ++tl) {
+      d[tl][0] += e[tl][0];
+      d[tl][1] += e[tl][1];
+      d[tl][2] += e[tl][2];
+      d[tl][3] += e[tl][3];
     }
   }
   if (!__syncthreads_and(wok)) {  // the weight never landed: status has the timeout bit
@@ -348,21 +452,33 @@ __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArg
     return;
   }
   // a6: the warps' partial sums, [warp][tile][16][8], in the weight's space
+  if constexpr (kDp4a) {
+    if ((lane & ((1 << SH) - 1)) == 0) {
 #pragma unroll
-  for (int tl = 0; tl < kTilesV; ++tl) {
-    if (tl < T) {
-      int32_t* pp = s_part + (warp * T + tl) * 128;
-      pp[g * 8 + 2 * t4] = d[tl][0];
-      pp[g * 8 + 2 * t4 + 1] = d[tl][1];
-      pp[(g + 8) * 8 + 2 * t4] = d[tl][2];
-      pp[(g + 8) * 8 + 2 * t4 + 1] = d[tl][3];
+      for (int gi = 0; gi < NG; ++gi) {
+        const int r = RG * gi + (lane >> SH);
+        if (r < rb) {
+#pragma unroll
+          for (int j = 0; j < MR; ++j) s_part[(warp * T + (r >> 4)) * 128 + (r & 15) * 8 + j] = rsum[gi][j];
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int tl = 0; tl < kTilesV; ++tl) {
+      if (tl < T) {
+        int32_t* pp = s_part + (warp * T + tl) * 128;
+        pp[g * 8 + 2 * t4] = d[tl][0];
+        pp[g * 8 + 2 * t4 + 1] = d[tl][1];
+        pp[(g + 8) * 8 + 2 * t4] = d[tl][2];
+        pp[(g + 8) * 8 + 2 * t4 + 1] = d[tl][3];
+      }
     }
   }
   __syncthreads();
 
   // a6-a7: dequantize, add the 16-bit outlier product (ascending) and the bias
   if (!eact) return;
-  const __half* bias = static_cast<const __half*>(p.bias);
   __half* Y = static_cast<__half*>(p.Y);
   const int nwords = static_cast<int>(K / 32);
   const float rsm = s_rs[em];
@@ -375,18 +491,20 @@ __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArg
       int32_t acc = 0;
 #pragma unroll
       for (int v = 0; v < kWarpsV; ++v) acc += s_part[(v * T + tl) * 128 + rr * 8 + em];
-      const float csw = __ldg(p.cs + n);
-      float y = static_cast<float>(acc) * rsm * (csw * (1.0f / 16129.0f));
-#pragma unroll 4
-      for (int t = 0; t < n_use; ++t) {
+      float y = static_cast<float>(acc) * rsm * (csw[i] * (1.0f / 16129.0f));
+#pragma unroll
+      for (int t = 0; t < kPreV; ++t)
+        if (t < npre) y = fmaf(__half2float(px[t]), __half2float(pw[i][t]), y);
+#pragma unroll 1
+      for (int t = npre; t < n_use; ++t) {  // many outliers, or no 16-bit weight: fetched one by one
         const int col = t < kListV ? s_list[t] : outlier_col_at(t, s_mask, nwords);
         // without the 16-bit weight, the outlier rows come from the int8 codes
         const float w = W != nullptr ? __half2float(W[int64_t(col) * p.ldw + n])
                                      : __half2float(__ushort_as_half(dequant_weight_bits(
-                                           static_cast<int8_t>(p.Wq[int64_t(n) * ldk + col]), csw)));
+                                           static_cast<int8_t>(p.Wq[int64_t(n) * ldk + col]), csw[i])));
         y = fmaf(__half2float(X[int64_t(em) * p.ldx + col]), w, y);
       }
-      if (bias != nullptr) y += __half2float(bias[n]);  // the linear layer's bias, added last
+      y += bv[i];  // the linear layer's bias, added last (0 without one)
       Y[int64_t(em) * p.ldy + n] = __float2half_rn(overflow ? __int_as_float(0x7fc00000) : y);
     }
   }

@@ -341,11 +341,12 @@ def test_decode_repeat_calls_leave_split_k_scratch_at_zero(L):
 # for the one-kernel path (three kernels); a 2-row call at the decode size.
 DECODE_SHAPES = [(1, 128, 128), (5, 300, 1032), (17, 520, 2056), (24, 129, 264), (9, 2048, 16384),
                  (32, 1024, 8192), (16, 16384, 4096), (2, 4096, 4096),
-                 # matrix-vector kernel (M <= 4, K a multiple of 512 up to 4096, at most 64 Wq rows per CTA):
-                 # one Wq row per CTA, 61 rows per CTA (two outputs per thread), one 64-column chunk per warp;
-                 # the others take the cluster kernel (more rows of X, too many Wq rows per CTA, K not a
-                 # multiple of 512, K too large)
-                 (1, 100, 512), (4, 9000, 512), (2, 2000, 1024), (3, 4096, 2048), (6, 1500, 4096),
+                 # matrix-vector kernel (M <= 8, K a multiple of 512 up to 4096, at most 64 Wq rows per CTA;
+                 # dp4a products up to 4 rows of X, warp MMAs above): one Wq row per CTA, 61 rows per CTA
+                 # (two outputs per thread), one 64-column chunk per warp; the others take the cluster
+                 # kernel (too many Wq rows per CTA, K not a multiple of 512, K too large)
+                 (1, 100, 512), (4, 9000, 512), (5, 9000, 512), (2, 2000, 1024), (8, 2000, 1024),
+                 (3, 4096, 2048), (6, 1500, 4096), (7, 4096, 4096),
                  (8, 16384, 1024), (7, 129, 96), (3, 1000, 16384)]
 
 
