@@ -198,6 +198,17 @@ llmint8_status llmint8_outlier_stats(const void* X, int64_t M, int64_t K, int64_
  * Host-only query. */
 int llmint8_mixed_matmul_kernels(int64_t M, int64_t N, int64_t K, int64_t ldx, const void* X);
 
+/* The kernels llmint8_mixed_matmul launches for these arguments, by name, in
+ * launch order and comma-separated: "decode_gemv_kernel" (M <= 8, whole Wq
+ * rows per CTA), "decode_fused_kernel" (M <= 32, cluster split-K), or the
+ * activation step ("act_fused_kernel", or "scan_columns_kernel" then
+ * "quantize_rows_kernel" / "quantize_rows_long_kernel") followed by the GEMM
+ * ("gemm_i8_decode_kernel" for M <= 32, else "gemm_i8_kernel").  ldk is the
+ * leading dimension of the Wq the call will get.  The string is static (do
+ * not free it).  NULL for arguments the call rejects as invalid, or when no
+ * CUDA device is current.  Launches nothing. */
+const char* llmint8_mixed_matmul_path(int64_t M, int64_t N, int64_t K, int64_t ldx, int64_t ldk, const void* X);
+
 /* Steps a5-a7 alone, on an activation already quantized by
  * llmint8_quantize_act_rowwise_outliers (so that one quantized X can feed
  * several weights, e.g. projections that share their input):

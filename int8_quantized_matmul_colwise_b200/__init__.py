@@ -16,7 +16,8 @@ from typing import Dict, Optional, Tuple
 
 from . import capi
 from .capi import (LLMInt8Error, empty_workspace, llmint8_check_status, llmint8_debug_int8_gemm_i32,
-                   llmint8_mixed_gemm, llmint8_mixed_matmul, llmint8_mixed_matmul_kernels, llmint8_outlier_stats,
+                   llmint8_mixed_gemm, llmint8_mixed_matmul, llmint8_mixed_matmul_kernels, llmint8_mixed_matmul_path,
+                   llmint8_outlier_stats,
                    llmint8_quantize_act_rowwise_outliers, llmint8_quantize_weight_colwise,
                    llmint8_status_string, llmint8_workspace_init, llmint8_workspace_layout,
                    llmint8_workspace_size, round_up, workspace_views)
@@ -28,6 +29,7 @@ __all__ = [
     "llmint8_mixed_gemm", "mixed_gemm",
     "llmint8_check_status", "llmint8_debug_int8_gemm_i32", "llmint8_status_string", "llmint8_workspace_size",
     "llmint8_workspace_init", "llmint8_workspace_layout", "llmint8_mixed_matmul_kernels",
+    "llmint8_mixed_matmul_path",
     "llmint8_outlier_stats", "outlier_stats", "Int8Linear",
 ]
 

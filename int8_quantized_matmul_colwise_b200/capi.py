@@ -73,6 +73,7 @@ SIGNATURES = {
                                                             _P, _I64, _P]),
     "llmint8_check_status": (_ST, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "llmint8_mixed_matmul_kernels": (ctypes.c_int, [_I64, _I64, _I64, _I64, _P]),
+    "llmint8_mixed_matmul_path": (ctypes.c_char_p, [_I64, _I64, _I64, _I64, _I64, _P]),
     "llmint8_outlier_stats": (_ST, [_P, _I64, _I64, _I64, _F, _P, _P, _SZ, _P]),
     "llmint8_debug_int8_gemm_i32": (_ST, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64, _P, _SZ, _P]),
 }
@@ -272,9 +273,18 @@ def llmint8_outlier_stats(X, tau: float, stats, ws, stream=None):
 
 
 def llmint8_mixed_matmul_kernels(X, N: int) -> int:
-    """Kernels llmint8_mixed_matmul launches for this X and N (1 or 3)."""
+    """Kernels llmint8_mixed_matmul launches for this X and N (1, 2 or 3)."""
     M, K = X.shape
     return int(lib().llmint8_mixed_matmul_kernels(M, N, K, _ld(X), _ptr(X)))
+
+
+def llmint8_mixed_matmul_path(X, Wq, K: int):
+    """Names of the kernels llmint8_mixed_matmul launches for this X and Wq
+    ([N, ldk] int8), in launch order; None if the call would be rejected."""
+    M = X.shape[0]
+    N = Wq.shape[0]
+    r = lib().llmint8_mixed_matmul_path(M, N, K, _ld(X), _ld(Wq), _ptr(X))
+    return None if r is None else r.decode().split(",")
 
 
 def llmint8_debug_int8_gemm_i32(Xq, Wq, K: int, C, ws, stream=None):

@@ -243,6 +243,25 @@ int llmint8_mixed_matmul_kernels(int64_t M, int64_t N, int64_t K, int64_t ldx, c
   return act_fused_plan(M, K, ldx, X, num_sms) ? 2 : 3;  // activation step in one or two kernels, then the GEMM
 }
 
+const char* llmint8_mixed_matmul_path(int64_t M, int64_t N, int64_t K, int64_t ldx, int64_t ldk, const void* X) {
+  if (!X || M < 1 || N < 1 || K < 1 || K > kMaxK || ldx < K || ldk < K || ldk % 16 != 0 ||
+      M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1)
+    return nullptr;
+  int num_sms = 0, s = 0, kb = 0, stages = 0;
+  if (current_device(&num_sms) != LLMINT8_OK) return nullptr;
+  if (use_gemv_decode(M, N, K, ldx, ldk, X, num_sms, &s, &kb)) return "decode_gemv_kernel";
+  if (use_fused_decode(M, N, K, ldx, X, num_sms, &s, &kb, &stages)) return "decode_fused_kernel";
+  const bool decode = M <= kDecodeMaxM;
+  if (act_fused_plan(M, K, ldx, X, num_sms))
+    return decode ? "act_fused_kernel,gemm_i8_decode_kernel" : "act_fused_kernel,gemm_i8_kernel";
+  // the row kernel takes rows of up to 2048 chunks of 8 columns; longer rows the long-row kernel
+  if ((K + 7) / 8 > 2048)
+    return decode ? "scan_columns_kernel,quantize_rows_long_kernel,gemm_i8_decode_kernel"
+                  : "scan_columns_kernel,quantize_rows_long_kernel,gemm_i8_kernel";
+  return decode ? "scan_columns_kernel,quantize_rows_kernel,gemm_i8_decode_kernel"
+                : "scan_columns_kernel,quantize_rows_kernel,gemm_i8_kernel";
+}
+
 size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K, int64_t outlier_cap) {
   llmint8_ws_layout L;
   if (llmint8_workspace_layout(M, N, K, outlier_cap, &L) != LLMINT8_OK) return 0;

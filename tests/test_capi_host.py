@@ -103,6 +103,16 @@ def test_binding_refuses_host_tensors():
         L.llmint8_quantize_weight_colwise(W, torch.zeros(8, 16, dtype=torch.int8), torch.zeros(8))
 
 
+def test_kernel_path_query_rejects_invalid_sizes(lib):
+    f = lib.llmint8_mixed_matmul_path
+    assert f(0, 16, 16, 16, 16, 0x1000) is None        # M < 1
+    assert f(4, 16, 16, 8, 16, 0x1000) is None         # ldx < K
+    assert f(4, 16, 16, 16, 8, 0x1000) is None         # ldk < K
+    assert f(4, 16, 24, 24, 40, 0x1000) is None        # ldk not a multiple of 16
+    assert f(4, 16, 16, 16, 16, None) is None          # no X
+    assert f(4, 16, 200000, 200000, 200000, 0x1000) is None  # K beyond the int32 accumulator bound
+
+
 def test_kernel_count_query_rejects_invalid_sizes(lib):
     f = lib.llmint8_mixed_matmul_kernels
     assert f(0, 16, 16, 16, 0x1000) == 0        # M < 1

@@ -581,6 +581,27 @@ def test_kernel_count_query(L):
     assert count(100, 300, 1000, ldx=1001) == 3  # rows not 16-byte aligned
 
 
+def test_kernel_path_query(L):
+    """llmint8_mixed_matmul_path names the kernels of each path, as many as
+    llmint8_mixed_matmul_kernels counts."""
+    def path(M, N, K, ldx=None, ldk=None):
+        ldx = K if ldx is None else ldx
+        ldk = L.round_up(K, 16) if ldk is None else ldk
+        X = torch.empty((M, ldx), dtype=torch.float16, device="cuda")[:, :K]
+        Wq = torch.empty((N, ldk), dtype=torch.int8, device="cuda")
+        p = L.llmint8_mixed_matmul_path(X, Wq, K)
+        assert len(p) == L.llmint8_mixed_matmul_kernels(X, N)
+        return p
+    assert path(1, 4096, 4096) == ["decode_gemv_kernel"]
+    assert path(8, 4096, 4096) == ["decode_gemv_kernel"]
+    assert path(8, 16384, 1024) == ["decode_fused_kernel"]         # more Wq rows per SM than the kernel holds
+    assert path(32, 4096, 4096) == ["decode_fused_kernel"]         # more rows of X
+    assert path(2048, 16384, 4096) == ["act_fused_kernel", "gemm_i8_kernel"]
+    assert path(8192, 8192, 8192) == ["scan_columns_kernel", "quantize_rows_kernel", "gemm_i8_kernel"]
+    assert path(100, 300, 1000, ldx=1001) == ["scan_columns_kernel", "quantize_rows_kernel", "gemm_i8_kernel"]
+    assert path(5, 130, 20000) == ["scan_columns_kernel", "quantize_rows_long_kernel", "gemm_i8_decode_kernel"]
+
+
 @pytest.mark.parametrize("name", ["ragged_1000x1000x1000", "ffn_6p7b_prefill"])
 def test_outlier_overflow_on_the_prefill_path(L, name):
     """A cap below n_o through the one-kernel activation step and the tcgen05
