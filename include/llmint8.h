@@ -193,9 +193,10 @@ llmint8_status llmint8_outlier_stats(const void* X, int64_t M, int64_t K, int64_
                                      void* ws, size_t ws_bytes, void* stream);
 
 /* Number of kernels llmint8_mixed_matmul launches on the current device for
- * these arguments: 1 on the one-kernel decode path, 2 when the activation step
+ * these arguments, for a Wq with the packed leading dimension ldk =
+ * round_up(K, 16): 1 on a one-kernel decode path, 2 when the activation step
  * is one kernel, else 3 (0 for invalid sizes or no supported device).
- * Host-only query. */
+ * llmint8_mixed_matmul_path takes ldk.  Host-only query. */
 int llmint8_mixed_matmul_kernels(int64_t M, int64_t N, int64_t K, int64_t ldx, const void* X);
 
 /* The kernels llmint8_mixed_matmul launches for these arguments, by name, in
