@@ -169,14 +169,15 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
  * that streams Wq on all SMs), or two when the activation step fits one
  * kernel.  Decode-shaped calls (ldx % 8 == 0, X 16-byte aligned) take one
  * kernel for all of it: for M <= 8 with K a multiple of 512 up to 4096 and at
- * most 64 Wq rows per SM, each CTA owns whole Wq rows (the weight is read
- * before the preceding kernel has finished, under programmatic dependent
- * launch: it must not be written by a kernel that triggers its dependents
- * early); otherwise for M <= 32 with K % 8 == 0 and K <= 16384 (and N, K small
- * enough that each CTA's share of Xq fits in 32 KB of shared memory) CTA
- * clusters split K, exchange outlier flags and row maxima through distributed
- * shared memory and reduce their int32 partial sums there.  The workspace
- * then receives the same Xq, row scales, O, n_o and Xo.
+ * most 64 Wq rows per SM, each CTA owns whole Wq rows; otherwise for M <= 32
+ * with K % 8 == 0 and K <= 16384 (and N, K small enough that each CTA's share
+ * of Xq fits in 32 KB of shared memory) CTA clusters split K, exchange outlier
+ * flags and row maxima through distributed shared memory and reduce their
+ * int32 partial sums there.  Both start reading Wq before the preceding
+ * kernel on the stream has finished (programmatic dependent launch), so Wq
+ * must not be written by a kernel that lets its dependents start early (no
+ * kernel of this library does).  The workspace then receives the same Xq,
+ * row scales, O, n_o and Xo.
  * llmint8_mixed_matmul_path names the kernels of a call.  No host
  * synchronisation. */
 llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
