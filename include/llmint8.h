@@ -175,9 +175,9 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
  * flags and row maxima through distributed shared memory and reduce their
  * int32 partial sums there.  Both start reading Wq before the preceding
  * kernel on the stream has finished (programmatic dependent launch), so Wq
- * must not be written by a kernel that lets its dependents start early (no
- * kernel of this library does).  The workspace then receives the same Xq,
- * row scales, O, n_o and Xo.
+ * must not be written by a kernel that lets its dependents start early
+ * (llmint8_quantize_weight_colwise's kernel does not).  The workspace then
+ * receives the same Xq, row scales, O, n_o and Xo.
  * llmint8_mixed_matmul_path names the kernels of a call.  No host
  * synchronisation. */
 llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
