@@ -94,8 +94,9 @@ __device__ __noinline__ int outlier_col_at(int t, const uint32_t* s_mask, int nw
 }
 
 // Sum of R per-lane values over the 32 lanes, halving the vector at each
-// step: afterwards the lane holds the total of value `row` (lanes that agree
-// on the bits above 32 / R hold the same value).
+// step: afterwards the lane holds the total of value `row`, which is the
+// lane's top log2(R) bits (lanes that differ only in the lower 5 - log2(R)
+// bits hold the same total).
 template <int R>
 __device__ __forceinline__ int32_t rows_sum_transposed(int32_t (&v)[R], int lane, int& row) {
   int o = 16;
