@@ -328,24 +328,30 @@ __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArg
   // the epilogue's operands from global memory, loaded while the MMAs run:
   // column scales, bias, and the first outlier terms' x and 16-bit w
   const int npre = W != nullptr ? min(n_use, kPreV) : 0;
-  float csw[2] = {0.0f, 0.0f}, bv[2] = {0.0f, 0.0f};
-  __half px[kPreV], pw[2][kPreV];
+  // (16-bit values stay one per 32-bit register, unconverted, so that no
+  // instruction waits on these loads before the epilogue)
+  const unsigned short* Xb = static_cast<const unsigned short*>(p.X);
+  const unsigned short* Wb = static_cast<const unsigned short*>(p.W);
+  const unsigned short* Bb = static_cast<const unsigned short*>(p.bias);
+  float csw[2] = {0.0f, 0.0f};
+  uint32_t bv[2] = {0u, 0u};
+  uint32_t px[kPreV], pw[2][kPreV];
 #pragma unroll
-  for (int t = 0; t < kPreV; ++t) px[t] = pw[0][t] = pw[1][t] = __ushort_as_half(0);
+  for (int t = 0; t < kPreV; ++t) px[t] = pw[0][t] = pw[1][t] = 0u;
   if (eact) {
 #pragma unroll
     for (int t = 0; t < kPreV; ++t)
-      if (t < npre) px[t] = X[int64_t(em) * p.ldx + s_list[t]];
+      if (t < npre) px[t] = Xb[int64_t(em) * p.ldx + s_list[t]];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int r = lane + 32 * (eg + G * i);
       if (r < rb) {
         const int n = n0 + r;
         csw[i] = __ldg(p.cs + n);
-        if (bias != nullptr) bv[i] = __half2float(bias[n]);
+        if (bias != nullptr) bv[i] = Bb[n];
 #pragma unroll
         for (int t = 0; t < kPreV; ++t)
-          if (t < npre) pw[i][t] = W[int64_t(s_list[t]) * p.ldw + n];
+          if (t < npre) pw[i][t] = Wb[int64_t(s_list[t]) * p.ldw + n];
       }
     }
   }
@@ -495,7 +501,9 @@ __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArg
       float y = static_cast<float>(acc) * rsm * (csw[i] * (1.0f / 16129.0f));
 #pragma unroll
       for (int t = 0; t < kPreV; ++t)
-        if (t < npre) y = fmaf(__half2float(px[t]), __half2float(pw[i][t]), y);
+        if (t < npre)
+          y = fmaf(__half2float(__ushort_as_half(static_cast<unsigned short>(px[t]))),
+                   __half2float(__ushort_as_half(static_cast<unsigned short>(pw[i][t]))), y);
 #pragma unroll 1
       for (int t = npre; t < n_use; ++t) {  // many outliers, or no 16-bit weight: fetched one by one
         const int col = t < kListV ? s_list[t] : outlier_col_at(t, s_mask, nwords);
@@ -505,7 +513,7 @@ __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArg
                                            static_cast<int8_t>(p.Wq[int64_t(n) * ldk + col]), csw[i])));
         y = fmaf(__half2float(X[int64_t(em) * p.ldx + col]), w, y);
       }
-      y += bv[i];  // the linear layer's bias, added last (0 without one)
+      y += __half2float(__ushort_as_half(static_cast<unsigned short>(bv[i])));  // the bias, added last (0 without one)
       Y[int64_t(em) * p.ldy + n] = __float2half_rn(overflow ? __int_as_float(0x7fc00000) : y);
     }
   }
