@@ -22,6 +22,43 @@ def test_every_declared_function_is_exported(lib):
     assert set(names) == set(capi.SIGNATURES), set(names) ^ set(capi.SIGNATURES)
 
 
+def _c_kind(decl: str):
+    """ctypes type a C parameter or return declaration maps to."""
+    d = " ".join(decl.replace("const", " ").split())
+    if d.startswith("char*") or d.endswith("char*"):
+        return ctypes.c_char_p
+    if "*" in d:
+        return "pointer"
+    for c, t in (("int64_t", ctypes.c_int64), ("size_t", ctypes.c_size_t), ("float", ctypes.c_float),
+                 ("llmint8_status", ctypes.c_int), ("int", ctypes.c_int)):
+        if d.split()[0] == c:
+            return t
+    raise AssertionError(f"unmapped C type: {decl}")
+
+
+def test_binding_signatures_match_the_header():
+    """Every prototype in include/llmint8.h against the binding's ctypes
+    signature: same number of parameters, same kind for each, same return."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", open(capi.HEADER).read(), flags=re.S)
+    text = re.sub(r"#[^\n]*", "", text)
+    protos = re.findall(r"([A-Za-z_][\w\s\*]*?)\b(llmint8_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", text)
+    assert {n for _, n, _ in protos} == set(capi.SIGNATURES)
+    for ret, name, args in protos:
+        want_ret, want_args = capi.SIGNATURES[name]
+        ret_words = ret.split()
+        ret_decl = " ".join(ret_words[-2:]) if ret_words[-1] == "char*" else ret_words[-1]
+        assert _c_kind(ret_decl) == want_ret, (name, ret_decl)
+        params = [a.strip() for a in args.split(",") if a.strip()]
+        assert len(params) == len(want_args), (name, len(params), len(want_args))
+        for i, (prm, t) in enumerate(zip(params, want_args)):
+            k = _c_kind(prm if "*" in prm else prm.rsplit(" ", 1)[0])
+            if k == "pointer":
+                assert t is ctypes.c_void_p or issubclass(t, ctypes._Pointer), (name, i, prm)
+            else:
+                assert k == t, (name, i, prm, t)
+
+
 def test_status_strings(lib):
     for code, name in capi.STATUS_NAMES.items():
         assert capi.llmint8_status_string(code) == name
