@@ -48,23 +48,25 @@ ScratchLayout scratch_layout(int64_t K) {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void* g_ptr[kMaxDevices] = {};  // device address of g_scratch, per device
+void* g_zeroed[kMaxDevices] = {};  // per device: the array address last zero-filled
 
-// Once per device, with that device current: the array's device address (the
-// host-side name g_scratch is only a stand-in) and a zero fill, since the
-// column maxima and counters must start at zero (the kernels return them to
-// zero after every call).
+// With the device current: the array's device address (the host-side name
+// g_scratch is only a stand-in), looked up on every call, since a device
+// reset or a new primary context loads the module again and may place the
+// array elsewhere.  The first call that sees an address zero-fills the array,
+// since the column maxima and counters must start at zero (the kernels return
+// them to zero after every call).
 llmint8_status scratch_for_current_device(void** out, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LLMINT8_ERR_CUDA;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return LLMINT8_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (g_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return LLMINT8_ERR_CUDA;
+  if (g_zeroed[dev] != p) {
     if (cudaMemsetAsync(p, 0, kScratchBytes, stream) != cudaSuccess) return LLMINT8_ERR_CUDA;
-    g_ptr[dev] = p;
+    g_zeroed[dev] = p;
   }
-  *out = g_ptr[dev];
+  *out = p;
   return LLMINT8_OK;
 }
 

@@ -71,6 +71,45 @@ def test_noalloc_matches_workspace_entry_on_two_calls(L, names):
         _same(got, ref_out, n)
 
 
+@pytest.mark.parametrize("M,K", [(3, 20000), (2, 61440)])
+def test_noalloc_long_rows_and_the_largest_k(L, M, K):
+    """Rows longer than 16384 columns (the long-row kernel) and K at the
+    array's limit, where the per-block counters and the outlier bitmask sit
+    at the end of the array; a few planted outlier columns; two calls."""
+    rng = np.random.default_rng(K + M)
+    for call in range(2):
+        X = (rng.standard_normal((M, K), dtype=np.float32)).astype(np.float16)
+        cols = np.sort(rng.choice(K, size=5, replace=False))
+        cols[-1] = K - 1  # the last column, in the last bitmask word
+        X[:, cols] = (X[:, cols].astype(np.float32) * 20.0).astype(np.float16)
+        X[0, cols] = 7.5  # with two rows a x20 column can stay below the threshold; make each one an outlier
+        Xd = torch.from_numpy(X).cuda()
+        ref = L.quantize_act_rowwise_outliers(Xd, 6.0, K)
+        got = _outputs(M, K, K)
+        _noalloc(L, Xd, 6.0, got)
+        torch.cuda.synchronize()
+        n = int(ref["n_outlier"].item())
+        assert set(cols.tolist()) <= set(ref["outlier_idx"][:n].tolist())
+        _same(got, {k: ref[k] for k in ("Xq", "row_scale", "outlier_idx", "n_outlier", "Xo")}, n)
+
+
+def test_noalloc_allocates_nothing_at_call_time(L):
+    """After one warm-up call, further calls leave both torch's allocator and
+    the device's free memory unchanged."""
+    w = wl.get("ragged_129x257x520")
+    X = torch.from_numpy(wl.make_x(w)).cuda()
+    out = _outputs(w.M, w.K, w.K)
+    _noalloc(L, X, w.tau, out)
+    torch.cuda.synchronize()
+    before_torch = torch.cuda.memory_allocated()
+    before_free = torch.cuda.mem_get_info()[0]
+    for _ in range(5):
+        _noalloc(L, X, w.tau, out)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == before_torch
+    assert torch.cuda.mem_get_info()[0] == before_free
+
+
 def test_noalloc_rejects_k_beyond_its_array(L):
     M, K = 2, 61441
     X = torch.zeros((M, K), dtype=torch.float16, device="cuda")
