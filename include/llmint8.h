@@ -249,13 +249,19 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
  * per-block counters, outlier bitmask) lives in a 256 KiB device array inside
  * the library, which every GPU it is used on keeps until the process exits.
  *   K <= LLMINT8_NOALLOC_MAX_K, otherwise LLMINT8_ERR_WORKSPACE and nothing
- *   runs.  Nothing is allocated: no cudaMalloc, cudaFree or allocating library
- *   call.  The first call on a device looks up the array's device address and
- *   zero-fills it on `stream`; make that first call before any stream capture.
- *   All calls share the array: calls that overlap on the GPU (different
- *   streams or host threads) race and must be ordered by the caller.  The
- *   status word is not reported; an outlier overflow shows as
- *   *n_outlier > outlier_cap. */
+ *   runs.  This entry point calls no cudaMalloc, cudaFree or allocating
+ *   library routine.  With lazy module loading (the CUDA 12 default) the
+ *   first call on a device loads the library's device code, and the driver
+ *   places the array in device memory at that moment: a caller that must not
+ *   see any allocation at call time makes one call during its initialisation.
+ *   Every call looks up the array's device address on the current device (so
+ *   a device reset or a new primary context is picked up); the first call
+ *   that sees a new address zero-fills the array on `stream`, so make that
+ *   first call before any stream capture.  All calls share the array and it
+ *   keeps the last call's contents (the kernels return the parts that must
+ *   start at zero to zero): calls that overlap on the GPU (different streams
+ *   or host threads) race and must be ordered by the caller.  The status word
+ *   is not reported; an outlier overflow shows as *n_outlier > outlier_cap. */
 #define LLMINT8_NOALLOC_MAX_K 61440
 llmint8_status llmint8_quantize_act_rowwise_outliers_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
                                                              float tau, int8_t* Xq, int64_t ldq, float* row_scale,
@@ -279,6 +285,35 @@ llmint8_status llmint8_check_status(void* ws, void* stream, uint32_t* flags_out)
 llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const int8_t* Wq, int64_t ldk,
                                            int64_t M, int64_t N, int64_t K, int32_t* C, int64_t ldc,
                                            void* ws, size_t ws_bytes, void* stream);
+
+/* Test hook for the whole path's step a5: runs exactly what
+ * llmint8_mixed_matmul runs for these arguments (the same kernels, launch
+ * plan and workspace outputs Xq, rs, O, n_o, Xo), except that every path's
+ * epilogue stores the raw int32 accumulator
+ *   C[i,j] = sum_k Xq[i,k] * Wq[j,k]      ("Compress your LLMs", Vector-wise
+ * quantization: the int8 product before the outer-product dequantization)
+ * into C int32 [M, ldc] (ldc >= N, 4-byte aligned) instead of Y, so that the
+ * one-kernel decode paths' int32 sums can be compared exactly.  No fp16
+ * weight or bias is read.  Same errors as llmint8_mixed_matmul. */
+llmint8_status llmint8_debug_mixed_matmul_i32(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
+                                              int64_t ldk, const float* col_scale, int64_t N, float tau,
+                                              int64_t outlier_cap, int32_t* C, int64_t ldc, void* ws,
+                                              size_t ws_bytes, void* stream);
+
+/* Test hook for failure detection (the pages have no counterpart).  Sets, on
+ * the current device, the bound after which every bounded wait inside the
+ * kernels gives up (default 2 s) and a mask of waits that are made to wait
+ * for an event that never comes, so that a test can watch a wait run out and
+ * the kernel return with LLMINT8_STATUS_TIMEOUT set instead of hanging:
+ *   0x1  the one-kernel activation step's grid barrier,
+ *   0x2  the matrix-vector decode kernel's wait for its weight copy,
+ *   0x4  the tcgen05 GEMM's MMA issuer, before its first operand stage.
+ * The kernels still let every copy they issued land before they exit.  After
+ * a stalled activation step the workspace must be zero-filled again.
+ * limit_ns == 0 is rejected (INVALID_ARG).  Synchronous; call it with no work
+ * of this library in flight, and call llmint8_debug_set_waits(2000000000, 0)
+ * to restore the defaults. */
+llmint8_status llmint8_debug_set_waits(uint64_t limit_ns, uint32_t stall_mask);
 
 #ifdef __cplusplus
 }

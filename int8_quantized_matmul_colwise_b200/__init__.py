@@ -16,6 +16,7 @@ from typing import Dict, Optional, Tuple
 
 from . import capi
 from .capi import (LLMInt8Error, empty_workspace, llmint8_check_status, llmint8_debug_int8_gemm_i32,
+                   llmint8_debug_mixed_matmul_i32, llmint8_debug_set_waits,
                    llmint8_mixed_gemm, llmint8_mixed_matmul, llmint8_mixed_matmul_kernels, llmint8_mixed_matmul_path,
                    llmint8_outlier_stats,
                    llmint8_quantize_act_rowwise_outliers, llmint8_quantize_weight_colwise,
@@ -30,7 +31,8 @@ __all__ = [
     "llmint8_check_status", "llmint8_debug_int8_gemm_i32", "llmint8_status_string", "llmint8_workspace_size",
     "llmint8_workspace_init", "llmint8_workspace_layout", "llmint8_mixed_matmul_kernels",
     "llmint8_mixed_matmul_path",
-    "llmint8_outlier_stats", "outlier_stats", "Int8Linear",
+    "llmint8_outlier_stats", "outlier_stats", "Int8Linear", "llmint8_debug_mixed_matmul_i32",
+    "llmint8_debug_set_waits", "debug_mixed_matmul_i32",
 ]
 
 
@@ -128,6 +130,21 @@ def debug_int8_gemm_i32(Xq, Wq, K: int, stream=None):
     ws = empty_workspace(M, N, K, 1, device=Xq.device)  # status word + decode split-K scratch
     llmint8_debug_int8_gemm_i32(Xq, Wq, K, C, ws, stream)
     return C
+
+
+def debug_mixed_matmul_i32(X, Wq, col_scale, tau: float = 6.0, outlier_cap: Optional[int] = None, ws=None,
+                           stream=None):
+    """int32 [M, N]: the accumulator the whole path computes for X (same
+    kernels as mixed_matmul), and the workspace holding its Xq, rs, O, Xo."""
+    import torch
+    M, K = X.shape
+    N = Wq.size(0)
+    cap = K if outlier_cap is None else outlier_cap
+    C = torch.empty((M, N), dtype=torch.int32, device=X.device)
+    if ws is None:
+        ws = empty_workspace(M, N, K, cap, device=X.device)
+    llmint8_debug_mixed_matmul_i32(X, Wq, col_scale, tau, cap, C, ws, stream)
+    return C, ws
 
 
 class Int8Weight:

@@ -76,6 +76,9 @@ SIGNATURES = {
     "llmint8_mixed_matmul_path": (ctypes.c_char_p, [_I64, _I64, _I64, _I64, _I64, _P]),
     "llmint8_outlier_stats": (_ST, [_P, _I64, _I64, _I64, _F, _P, _P, _SZ, _P]),
     "llmint8_debug_int8_gemm_i32": (_ST, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64, _P, _SZ, _P]),
+    "llmint8_debug_mixed_matmul_i32": (_ST, [_P, _I64, _I64, _I64, _P, _I64, _P, _I64, _F, _I64, _P, _I64, _P,
+                                             _SZ, _P]),
+    "llmint8_debug_set_waits": (_ST, [ctypes.c_uint64, ctypes.c_uint32]),
 }
 
 _lock = threading.Lock()
@@ -296,6 +299,33 @@ def llmint8_debug_int8_gemm_i32(Xq, Wq, K: int, C, ws, stream=None):
     _check(lib().llmint8_debug_int8_gemm_i32(_ptr(Xq), _ld(Xq), _ptr(Wq), _ld(Wq), M, N, K, _ptr(C), _ld(C),
                                              _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "llmint8_debug_int8_gemm_i32")
+
+
+def llmint8_debug_mixed_matmul_i32(X, Wq, col_scale, tau: float, outlier_cap: int, C, ws, stream=None):
+    """Test hook: the path of llmint8_mixed_matmul with the raw int32
+    accumulator stored in C [M, >= N] instead of Y."""
+    torch = _torch()
+    _rowmajor(X, "X", torch.float16)
+    _rowmajor(Wq, "Wq", torch.int8)
+    _rowmajor(col_scale, "col_scale", torch.float32, 1)
+    _rowmajor(C, "C", torch.int32)
+    M, K = X.shape
+    N = Wq.size(0)
+    _check(lib().llmint8_debug_mixed_matmul_i32(
+        _ptr(X), M, K, _ld(X), _ptr(Wq), _ld(Wq), _ptr(col_scale), N, float(tau), int(outlier_cap), _ptr(C), _ld(C),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "llmint8_debug_mixed_matmul_i32")
+
+
+DEFAULT_WAIT_LIMIT_NS = 2_000_000_000
+STALL_ACT_GRID_BARRIER = 0x1
+STALL_GEMV_WEIGHT = 0x2
+STALL_GEMM_OPERANDS = 0x4
+
+
+def llmint8_debug_set_waits(limit_ns: int = DEFAULT_WAIT_LIMIT_NS, stall_mask: int = 0):
+    """Test hook: the bound of the kernels' bounded waits and the mask of
+    waits held back (see include/llmint8.h).  Defaults restore normal use."""
+    _check(lib().llmint8_debug_set_waits(int(limit_ns), int(stall_mask)), "llmint8_debug_set_waits")
 
 
 # ------------------------------------------------------------------ allocation helpers (torch memory)

@@ -308,15 +308,23 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
                                          static_cast<cudaStream_t>(stream), true, num_sms));
 }
 
-llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
-                                    int64_t ldk, const float* col_scale, const void* W, int64_t ldw,
-                                    const void* bias, int64_t N, float tau, int64_t outlier_cap, void* Y,
-                                    int64_t ldy, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// llmint8_mixed_matmul, and its test hook: with C non-null every path stores
+// the raw int32 accumulator [M, ldc] in place of Y (Y, W and bias unused),
+// through the same kernels and launch plan.
+llmint8_status mixed_matmul_impl(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq, int64_t ldk,
+                                 const float* col_scale, const void* W, int64_t ldw, const void* bias, int64_t N,
+                                 float tau, int64_t outlier_cap, void* Y, int64_t ldy, void* ws, size_t ws_bytes,
+                                 void* stream, int32_t* C, int64_t ldc) {
   if (!X || !Wq || !col_scale || !Y) return LLMINT8_ERR_INVALID_ARG;  // W may be NULL: int8-only weight
   if (M < 1 || N < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1)
     return LLMINT8_ERR_INVALID_ARG;
   if (ldx < K || (W && ldw < N) || ldy < N || ldk < K || ldk % 16 != 0 || !valid_tau(tau))
     return LLMINT8_ERR_INVALID_ARG;
+  if (C && (ldc < N || !aligned(C, 4))) return LLMINT8_ERR_INVALID_ARG;
   if (outlier_cap < 1 || outlier_cap > K) return LLMINT8_ERR_INVALID_ARG;
   if (!aligned(Wq, 16) || !aligned(X, 2) || (W && !aligned(W, 2)) || !aligned(Y, 2) || !aligned(col_scale, 4) ||
       !aligned(bias, 2))
@@ -368,6 +376,8 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
     g.status = reinterpret_cast<uint32_t*>(b + L.status);
     g.rows_per = g_rows;
     g.tiles = g_tiles;
+    g.C = C;
+    g.ldc = ldc;
     return cuda_status(launch_decode_gemv(g, s, true));
   }
 
@@ -403,6 +413,8 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
     f.splits = f_splits;
     f.kb_per = f_kb;
     f.stages = f_stages;
+    f.C = C;
+    f.ldc = ldc;
     return cuda_status(launch_decode_fused(tmW, f, s, true));
   }
 
@@ -442,7 +454,9 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
     d.tile_counter = reinterpret_cast<uint32_t*>(
         b + decode_off + align_up(size_t(N) * size_t(decode_rows_padded(d.M)) * 4, 256));
     d.status = reinterpret_cast<uint32_t*>(b + L.status);
-    return cuda_status(launch_gemm_i8_decode(tmA, tmB, d, false, s, true));
+    d.C = C;
+    d.ldc = ldc;
+    return cuda_status(launch_gemm_i8_decode(tmA, tmB, d, C != nullptr, s, true));
   }
 
   GemmArgs a = {};
@@ -463,12 +477,50 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
   a.bias = bias;
   a.Y = Y;
   a.ldy = ldy;
-  a.C = nullptr;
-  a.ldc = 0;
+  a.C = C;
+  a.ldc = ldc;
   a.status = reinterpret_cast<uint32_t*>(b + L.status);
   CUtensorMap tmY;
-  a.y_tma = prepare_output(&tmY, Y, M, N, ldy);
-  return cuda_status(launch_gemm_i8(tmA, tmB, tmY, a, false, num_sms, s, true));
+  if (C) {
+    std::memset(&tmY, 0, sizeof(tmY));
+    a.y_tma = false;
+  } else {
+    a.y_tma = prepare_output(&tmY, Y, M, N, ldy);
+  }
+  return cuda_status(launch_gemm_i8(tmA, tmB, tmY, a, C != nullptr, num_sms, s, true));
+}
+
+}  // namespace
+
+extern "C" {
+
+llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
+                                    int64_t ldk, const float* col_scale, const void* W, int64_t ldw,
+                                    const void* bias, int64_t N, float tau, int64_t outlier_cap, void* Y,
+                                    int64_t ldy, void* ws, size_t ws_bytes, void* stream) {
+  return mixed_matmul_impl(X, M, K, ldx, Wq, ldk, col_scale, W, ldw, bias, N, tau, outlier_cap, Y, ldy, ws, ws_bytes,
+                           stream, nullptr, 0);
+}
+
+llmint8_status llmint8_debug_mixed_matmul_i32(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
+                                              int64_t ldk, const float* col_scale, int64_t N, float tau,
+                                              int64_t outlier_cap, int32_t* C, int64_t ldc, void* ws,
+                                              size_t ws_bytes, void* stream) {
+  if (!C) return LLMINT8_ERR_INVALID_ARG;
+  // Y is not written on this path; C stands in for the pointer check only
+  return mixed_matmul_impl(X, M, K, ldx, Wq, ldk, col_scale, nullptr, 0, nullptr, N, tau, outlier_cap, C, ldc, ws,
+                           ws_bytes, stream, C, ldc);
+}
+
+llmint8_status llmint8_debug_set_waits(uint64_t limit_ns, uint32_t stall_mask) {
+  if (limit_ns == 0) return LLMINT8_ERR_INVALID_ARG;
+  if (current_device(nullptr) != LLMINT8_OK) return LLMINT8_ERR_CUDA;
+  cudaError_t (*const setters[])(uint64_t, uint32_t) = {set_debug_waits_decode_fused, set_debug_waits_decode_gemv,
+                                                       set_debug_waits_gemm_i8, set_debug_waits_gemm_i8_decode,
+                                                       set_debug_waits_quant_act};
+  for (auto fn : setters)
+    if (fn(limit_ns, stall_mask) != cudaSuccess) return LLMINT8_ERR_CUDA;
+  return LLMINT8_OK;
 }
 
 llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* row_scale,

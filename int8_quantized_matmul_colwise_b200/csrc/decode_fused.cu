@@ -592,6 +592,10 @@ __global__ void __launch_bounds__(kThreadsF, MINB)
 #pragma unroll
         for (int src = 0; src < 8; ++src) part[src] = src < S ? s_red[(src * NP + m) * RO + i] : 0;
         const int32_t acc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+        if (p.C != nullptr) {  // test hook: the raw accumulator instead of Y
+          if (n < p.N) p.C[static_cast<int64_t>(m) * p.ldc + n] = acc;
+          continue;
+        }
         float y = static_cast<float>(acc) * s_rs[m] * csn;
 #pragma unroll 4
         for (int t = 0; t < tw; ++t) y = fmaf(__half2float(s_xo[m * kOList + t]), __half2float(s_w[t * RO + i]), y);
@@ -751,6 +755,11 @@ cudaError_t launch_decode_fused(const CUtensorMap& tmA, const FusedArgs& a, cuda
                          : launch_fused_variant<32, 16, 1>(tmA, a, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// Test hook: this file's wait bound and stall mask (see ptx.cuh).
+cudaError_t set_debug_waits_decode_fused(uint64_t limit_ns, uint32_t stall_mask) {
+  return set_debug_waits_in_this_file(limit_ns, stall_mask);
 }
 
 }  // namespace llmint8

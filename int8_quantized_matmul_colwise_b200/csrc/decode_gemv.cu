@@ -71,7 +71,7 @@ struct LayoutV {
     o += kListV * 4;
     rs = o;    // float [8] row scales
     o += kRowsV * 4;
-    bar = o;   // mbarrier: Wq landed
+    bar = o;   // mbarriers: Wq landed; a second one nothing arrives on (stall test hook)
     o += 16;
     total = o;
   }
@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArg
   int* s_list = reinterpret_cast<int*>(smem_v + lo.list);
   float* s_rs = reinterpret_cast<float*>(smem_v + lo.rs);
   uint64_t* wbar = reinterpret_cast<uint64_t*>(smem_v + lo.bar);
+  uint64_t* never = wbar + 1;
 
   const int tid = static_cast<int>(threadIdx.x);
   const int lane = tid & 31;
@@ -151,6 +152,7 @@ __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArg
   // The CTA's Wq rows are contiguous in memory: one bulk copy.
   if (tid == 0) {
     mbar_init(wbar, 1);
+    mbar_init(never, 1);
     fence_mbar_init();
     fence_proxy_async_smem();
     const uint32_t bytes = static_cast<uint32_t>(rb) * static_cast<uint32_t>(ldk);
@@ -357,7 +359,9 @@ __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArg
   }
 
   // a5: int8 products
-  const bool wok = mbar_wait(wbar, 0, p.status);
+  // (the stall test hook waits on a barrier that nothing arrives on instead:
+  // the wait runs out, the copy itself still lands and is waited for below)
+  const bool wok = mbar_wait(stalled(kStallGemvWeight) ? never : wbar, 0, p.status);
   int32_t d[kTilesV][4];
 #pragma unroll
   for (int tl = 0; tl < kTilesV; ++tl) d[tl][0] = d[tl][1] = d[tl][2] = d[tl][3] = 0;
@@ -498,6 +502,10 @@ __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArg
       int32_t acc = 0;
 #pragma unroll
       for (int v = 0; v < kWarpsV; ++v) acc += s_part[(v * T + tl) * 128 + rr * 8 + em];
+      if (p.C != nullptr) {  // test hook: the raw accumulator instead of Y
+        p.C[int64_t(em) * p.ldc + n] = acc;
+        continue;
+      }
       float y = static_cast<float>(acc) * rsm * (csw[i] * (1.0f / 16129.0f));
 #pragma unroll
       for (int t = 0; t < kPreV; ++t)
@@ -576,6 +584,11 @@ cudaError_t launch_decode_gemv(const GemvArgs& a, cudaStream_t stream, bool pdl)
     case 8: return cudaLaunchKernelEx(&cfg, decode_gemv_kernel<8>, a);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// Test hook: this file's wait bound and stall mask (see ptx.cuh).
+cudaError_t set_debug_waits_decode_gemv(uint64_t limit_ns, uint32_t stall_mask) {
+  return set_debug_waits_in_this_file(limit_ns, stall_mask);
 }
 
 }  // namespace llmint8

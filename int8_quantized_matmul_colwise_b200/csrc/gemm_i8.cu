@@ -131,7 +131,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, ui
     if (mbar_try_wait(a, parity)) return true;
     if ((++n & 63u) == 0u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > wait_limit_ns()) {
         atomicOr(status, kStatusTimeout);
         *abort = 1;
         return false;
@@ -203,6 +203,10 @@ __device__ void run_mma(const Shared& s, uint32_t tmem_base, const Sched& sc, ui
   uint32_t stage = 0, phase = 0, it = 0;
   bool ok = true;
   bool any = false;
+  // (the stall test hook first waits on the drain barrier, which nothing has
+  // arrived on yet: the wait runs out before any MMA is issued and the CTA
+  // takes the abort path)
+  if (stalled(kStallGemmOperands) && !wait_or_abort(s.drain, 0, status, s.abort)) ok = false;
   for (int tile = sc.first; tile < sc.num_tiles && ok; tile += sc.stride, ++it) {
     const uint32_t b = it & 1u;
     const uint32_t use = (it >> 1) & 1u;
@@ -721,6 +725,11 @@ cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const
   }
   return pair ? launch_variant<false, true>(tmA, tmB, tmY, a, num_sms, stream, pdl)
               : launch_variant<false, false>(tmA, tmB, tmY, a, num_sms, stream, pdl);
+}
+
+// Test hook: this file's wait bound and stall mask (see ptx.cuh).
+cudaError_t set_debug_waits_gemm_i8(uint64_t limit_ns, uint32_t stall_mask) {
+  return set_debug_waits_in_this_file(limit_ns, stall_mask);
 }
 
 }  // namespace llmint8

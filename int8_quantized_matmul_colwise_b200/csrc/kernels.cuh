@@ -162,6 +162,8 @@ struct FusedArgs {
   int splits;  // CTAs per tile (cluster size): 1, 2, 4 or 8
   int kb_per;  // 128-column K blocks per CTA (a power of two)
   int stages;  // Wq ring depth: 4 (two CTAs per SM) or 8
+  int32_t* C;  // test hook: non-null stores the int32 accumulator [M, ldc] instead of Y
+  int64_t ldc;
 };
 
 // ------------------------------------------------------------------ decode as a matrix-vector product (M <= 8)
@@ -190,6 +192,8 @@ struct GemvArgs {
   uint32_t* status;
   int rows_per;  // Wq rows per CTA
   int tiles;     // 16-row MMA tiles covering rows_per (at most 4)
+  int32_t* C;    // test hook: non-null stores the int32 accumulator [M, ldc] instead of Y
+  int64_t ldc;
 };
 // Rows per CTA and tiles for a call; false if this kernel does not take the shape.
 bool decode_gemv_plan(int M, int N, int K, int64_t ldk, int num_sms, int* rows_per, int* tiles);
@@ -200,5 +204,14 @@ cudaError_t launch_decode_gemv(const GemvArgs& a, cudaStream_t stream, bool pdl)
 bool decode_fused_plan(int M, int N, int K, int num_sms, int* splits, int* kb_per, int* stages);
 // tmA: Wq [N rows, K cols] int8, boxes of 128 rows x 128 bytes, 128-byte swizzle.
 cudaError_t launch_decode_fused(const CUtensorMap& tmA, const FusedArgs& a, cudaStream_t stream, bool pdl);
+
+// ------------------------------------------------------------------ test hooks
+// Each compiled file keeps its own copy of the wait bound and the stall mask
+// (ptx.cuh); these set them, one per file.
+cudaError_t set_debug_waits_decode_fused(uint64_t limit_ns, uint32_t stall_mask);
+cudaError_t set_debug_waits_decode_gemv(uint64_t limit_ns, uint32_t stall_mask);
+cudaError_t set_debug_waits_gemm_i8(uint64_t limit_ns, uint32_t stall_mask);
+cudaError_t set_debug_waits_gemm_i8_decode(uint64_t limit_ns, uint32_t stall_mask);
+cudaError_t set_debug_waits_quant_act(uint64_t limit_ns, uint32_t stall_mask);
 
 }  // namespace llmint8

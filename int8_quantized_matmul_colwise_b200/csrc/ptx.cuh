@@ -15,7 +15,30 @@ constexpr uint32_t kStatusTimeout = 0x2u;
 // A bounded wait gives up after this many nanoseconds of %globaltimer.  Real
 // waits in these kernels last microseconds; the bound only turns a hang into
 // an error status.
-constexpr uint64_t kWaitLimitNs = 2000ull * 1000ull * 1000ull;
+constexpr uint64_t kDefaultWaitLimitNs = 2000ull * 1000ull * 1000ull;
+
+// Test hooks, one copy per compiled file (set together for every file by
+// llmint8_debug_set_waits): the bound of the bounded waits, and a mask of
+// waits that are made to wait for an event that never comes, so that a test
+// can watch the bound run out and the kernel report it through the status
+// word instead of hanging.  Both stay at their defaults in normal use.
+static __device__ uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
+static __device__ uint32_t g_stall_mask = 0u;
+
+// Bits of g_stall_mask (which wait is held back).
+constexpr uint32_t kStallActGridBarrier = 0x1u;  // act_fused_kernel: the grid barrier never completes
+constexpr uint32_t kStallGemvWeight = 0x2u;      // decode_gemv_kernel: the weight copy is never seen to land
+constexpr uint32_t kStallGemmOperands = 0x4u;    // gemm_i8_kernel: the MMA issuer never sees its first stage
+
+__device__ __forceinline__ uint64_t wait_limit_ns() { return *const_cast<volatile uint64_t*>(&g_wait_limit_ns); }
+__device__ __forceinline__ bool stalled(uint32_t bit) { return (g_stall_mask & bit) != 0u; }
+
+// Host side: set this file's copies of the two hooks (synchronous).
+static inline cudaError_t set_debug_waits_in_this_file(uint64_t limit_ns, uint32_t stall_mask) {
+  cudaError_t e = cudaMemcpyToSymbol(g_wait_limit_ns, &limit_ns, sizeof(limit_ns));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_stall_mask, &stall_mask, sizeof(stall_mask));
+  return e;
+}
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -79,7 +102,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   uint32_t n = 0;
   while (true) {
     if (mbar_try_wait(a, parity)) return true;
-    if ((++n & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((++n & 63u) == 0u && globaltimer_ns() - t0 > wait_limit_ns()) {
       if (status) atomicOr(status, kStatusTimeout);
       return false;
     }
@@ -99,7 +122,7 @@ __device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t pari
     if (mbar_try_wait(a, parity)) return true;
     if ((++n & 63u) == 0u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > wait_limit_ns()) {
         atomicOr(status, kStatusTimeout);
         *abort = 1;
         return false;

@@ -407,14 +407,17 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
   __syncthreads();
   if (tid == 0) {
     int ok = 1;
-    if (atom_add_acq_rel_gpu_u32(arrived, 1u) == gridDim.x - 1u) {
+    // (the stall test hook asks for one arrival more than the grid has: the
+    // barrier then never completes and every CTA's wait runs out)
+    const uint32_t last = gridDim.x - 1u + (stalled(kStallActGridBarrier) ? 1u : 0u);
+    if (atom_add_acq_rel_gpu_u32(arrived, 1u) == last) {
       *arrived = 0u;                             // for the next call
       st_release_gpu_u32(generation, gen + 1u);  // releases the others
     } else {
       const uint64_t t0 = globaltimer_ns();
       uint32_t n = 0;
       while (ld_acquire_gpu_u32(generation) == gen) {
-        if ((++n & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+        if ((++n & 255u) == 0u && globaltimer_ns() - t0 > wait_limit_ns()) {
           atomicOr(ws.status, kStatusTimeout);
           ok = 0;
           break;
@@ -830,6 +833,11 @@ cudaError_t launch_outlier_stats(const void* X, int64_t M, int64_t K, int64_t ld
                                      scratch, stats)
                 : cudaLaunchKernelEx(&cfg, outlier_stats_kernel<false>, x, M, K, ldx, tau,
                                      static_cast<int>(rows_per), scratch, stats);
+}
+
+// Test hook: this file's wait bound and stall mask (see ptx.cuh).
+cudaError_t set_debug_waits_quant_act(uint64_t limit_ns, uint32_t stall_mask) {
+  return set_debug_waits_in_this_file(limit_ns, stall_mask);
 }
 
 }  // namespace llmint8

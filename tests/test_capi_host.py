@@ -29,7 +29,8 @@ def _c_kind(decl: str):
         return ctypes.c_char_p
     if "*" in d:
         return "pointer"
-    for c, t in (("int64_t", ctypes.c_int64), ("size_t", ctypes.c_size_t), ("float", ctypes.c_float),
+    for c, t in (("int64_t", ctypes.c_int64), ("uint64_t", ctypes.c_uint64), ("uint32_t", ctypes.c_uint32),
+                 ("size_t", ctypes.c_size_t), ("float", ctypes.c_float),
                  ("llmint8_status", ctypes.c_int), ("int", ctypes.c_int)):
         if d.split()[0] == c:
             return t
@@ -130,6 +131,25 @@ def test_debug_gemm_rejects_invalid_arguments(lib):
     f = lib.llmint8_debug_int8_gemm_i32
     assert f(0x1000, 16, 0x2000, 16, 1, 1, 17, 0x3000, 1, 0x10000, 256, None) == capi.ERR_INVALID_ARG
     assert f(0x1000, 16, 0x2000, 16, 1, 1, 16, 0x3000, 1, 0x10000, 128, None) == capi.ERR_WORKSPACE
+
+
+def test_debug_path_accumulator_rejects_invalid_arguments(lib):
+    f = lib.llmint8_debug_mixed_matmul_i32
+    ok = dict(X=0x1000, M=4, K=32, ldx=32, Wq=0x2000, ldk=32, cs=0x3000, N=16, tau=6.0, cap=32, C=0x5000, ldc=16,
+              ws=0x10000, ws_bytes=1 << 20)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["X"], a["M"], a["K"], a["ldx"], a["Wq"], a["ldk"], a["cs"], a["N"], a["tau"], a["cap"], a["C"],
+                 a["ldc"], a["ws"], a["ws_bytes"], None)
+    assert call(C=None) == capi.ERR_INVALID_ARG
+    assert call(ldc=15) == capi.ERR_INVALID_ARG      # ldc < N
+    assert call(C=0x5002) == capi.ERR_INVALID_ARG    # C not 4-byte aligned
+    assert call(ws_bytes=512) == capi.ERR_WORKSPACE
+
+
+def test_debug_set_waits_rejects_a_zero_bound(lib):
+    assert lib.llmint8_debug_set_waits(0, 0) == capi.ERR_INVALID_ARG
 
 
 def test_binding_refuses_host_tensors():

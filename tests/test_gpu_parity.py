@@ -3,10 +3,11 @@
 Bit-exact: Wq, col scales, outlier set and count, row scales, Xq, the gathered
 outlier columns and the int32 accumulator.  Y (fp16) within
 |Y_gpu - Y_oracle| <= 1e-3 |Y_oracle| + 1e-3 max|Y_oracle|.
-Small and ragged shapes are compared element by element; the full-size
-workloads are compared on every intermediate and on the accumulator and Y of
-64 seeded rows plus the first and last row, in the launch configuration the
-benchmark times.
+Small, ragged, decode, 6.7B FFN and 8192^3 sweep shapes are compared element
+by element over the whole matrices; the 175B shape on every intermediate and
+on Y of 64 seeded rows plus the first and last row, in the launch
+configuration the benchmark times.  (The int32 accumulators of every path and
+the quantizer at every kernel that quantizes are in test_gpu_paths.py.)
 """
 import numpy as np
 import pytest
@@ -247,6 +248,9 @@ def check_path(L, X, W, tau, rows=None, cap=None):
     if n <= (K if cap is None else cap):  # the gathered outlier columns, bit for bit
         assert np.array_equal(host(v["xo"])[:, :n].view(np.uint16), X[:, r["O"]].view(np.uint16))
     assert np.array_equal(host(cs), cs_ref)
+    Wq_g = host(Wq)
+    assert np.array_equal(Wq_g[:, :K], Wq_ref.T)
+    assert not Wq_g[:, K:].any()
     Yg = host(Y)
     Yg = Yg if rows is None else Yg[rows]
     y_close(Yg, r["Y"])
@@ -261,8 +265,7 @@ SMALL_PATH = ["tiny", "decode_m1", "decode_m8", "decode_m32", "ragged_1000x1000x
 def test_mixed_matmul_small_and_ragged(L, name):
     w = wl.get(name)
     X, W = wl.make_inputs(w)
-    rows = wl.sample_rows(w.M) if w.M * w.N * w.K > 4e9 else None
-    check_path(L, X, W, w.tau, rows=rows)
+    check_path(L, X, W, w.tau)
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged_129x257x520", "ragged_3x33x24"])
@@ -393,22 +396,26 @@ def test_decode_unaligned_rows_take_the_three_kernel_path(L):
     assert np.array_equal(Ya.view(np.uint16), Y.view(np.uint16))
 
 
-# ------------------------------------------------------------------ full-size workloads (sampled rows)
+# ------------------------------------------------------------------ full-size workloads
 
 @pytest.mark.parametrize("name", ["ffn_6p7b_prefill", "sweep8k_o0", "sweep8k_o0p1", "sweep8k_o1"])
 def test_mixed_matmul_full_size(L, name):
+    """The whole Y, Xq, O, rs, Xo, cs and Wq of the 6.7B FFN prefill and of
+    the 8192^3 sweeps (tau = 6 and +inf) against the oracle."""
     w = wl.get(name)
     X, W = wl.make_inputs(w)
-    rows = wl.sample_rows(w.M)
-    check_path(L, X, W, w.tau, rows=rows)
+    check_path(L, X, W, w.tau)
     if name.startswith("sweep"):
-        check_path(L, X, W, np.inf, rows=rows)
+        check_path(L, X, W, np.inf)
 
 
 def test_mixed_matmul_full_size_175b(L):
+    """175B hidden shape: every intermediate whole, Y on 64 seeded rows plus
+    the first and last (the oracle's int8 matmul over all 4096 rows would be
+    4.9e12 multiply-adds)."""
     w = wl.get("hidden_175b")
     X, W = wl.make_inputs(w)
-    rows = wl.sample_rows(w.M, n=16)
+    rows = wl.sample_rows(w.M, n=64)
     check_path(L, X, W, w.tau, rows=rows)
 
 
