@@ -269,6 +269,21 @@ llmint8_status llmint8_quantize_act_rowwise_outliers_noalloc(const void* X, int6
                                                              int32_t* n_outlier, void* Xo, int64_t ldo,
                                                              void* stream);
 
+/* Reassembly of an output whose columns were computed on several GPUs
+ * ("Compress your LLMs": the pages serve one model from 8 GPUs; the
+ * column-parallel split needs no exchange before the matmul, since the outlier
+ * set is a function of the replicated X, and one all-gather of Y after it).
+ *   blocks   fp16 [world, M, ld_block] (device): block r holds Y[:, bounds[r]
+ *            .. bounds[r+1]) in its first bounds[r+1] - bounds[r] <= ld_block
+ *            columns (what an all-gather of each GPU's shard leaves behind).
+ *   bounds   int64 [world + 1] (HOST), bounds[0] = 0, non-decreasing,
+ *            bounds[world] = N >= 1.  world <= 64.
+ *   Y, ldy   fp16 [M, N] written, row stride ldy >= N.
+ * One copy kernel on `stream` (16-byte moves when the block starts and both
+ * strides are multiples of 8 halves).  INVALID_ARG for bad sizes or bounds. */
+llmint8_status llmint8_unshard_columns(const void* blocks, int64_t world, int64_t M, int64_t ld_block,
+                                       const int64_t* bounds, void* Y, int64_t ldy, void* stream);
+
 /* Synchronise `stream`, read the status word of `ws`, clear it, and return
  * LLMINT8_OK, LLMINT8_ERR_OUTLIER_OVERFLOW or LLMINT8_ERR_TIMEOUT (timeout
  * wins).  `flags_out` (host, may be NULL) receives the raw bits.  After a

@@ -79,6 +79,7 @@ SIGNATURES = {
     "llmint8_debug_mixed_matmul_i32": (_ST, [_P, _I64, _I64, _I64, _P, _I64, _P, _I64, _F, _I64, _P, _I64, _P,
                                              _SZ, _P]),
     "llmint8_debug_set_waits": (_ST, [ctypes.c_uint64, ctypes.c_uint32]),
+    "llmint8_unshard_columns": (_ST, [_P, _I64, _I64, _I64, _P, _P, _I64, _P]),
 }
 
 _lock = threading.Lock()

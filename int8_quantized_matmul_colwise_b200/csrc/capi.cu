@@ -648,6 +648,25 @@ llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const 
   return cuda_status(launch_gemm_i8(tmA, tmB, tmY, a, true, num_sms, static_cast<cudaStream_t>(stream), false));
 }
 
+llmint8_status llmint8_unshard_columns(const void* blocks, int64_t world, int64_t M, int64_t ld_block,
+                                      const int64_t* bounds, void* Y, int64_t ldy, void* stream) {
+  if (!blocks || !bounds || !Y) return LLMINT8_ERR_INVALID_ARG;
+  if (world < 1 || world > kUnshardMaxWorld || M < 1 || ld_block < 1) return LLMINT8_ERR_INVALID_ARG;
+  if (!aligned(blocks, 2) || !aligned(Y, 2)) return LLMINT8_ERR_INVALID_ARG;
+  UnshardBounds b;
+  if (bounds[0] != 0) return LLMINT8_ERR_INVALID_ARG;
+  for (int64_t r = 0; r <= world; ++r) {
+    b.bounds[r] = bounds[r];
+    if (r > 0 && (bounds[r] < bounds[r - 1] || bounds[r] - bounds[r - 1] > ld_block)) return LLMINT8_ERR_INVALID_ARG;
+  }
+  if (bounds[world] < 1 || ldy < bounds[world]) return LLMINT8_ERR_INVALID_ARG;
+  int num_sms = 0;
+  llmint8_status st = current_device(&num_sms);
+  if (st != LLMINT8_OK) return st;
+  return cuda_status(launch_unshard_columns(blocks, static_cast<int>(world), M, ld_block, b, Y, ldy, num_sms,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 llmint8_status llmint8_check_status(void* ws, void* stream, uint32_t* flags_out) {
   if (!ws || !aligned(ws, 256)) return LLMINT8_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

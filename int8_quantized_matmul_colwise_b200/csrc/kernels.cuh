@@ -205,6 +205,15 @@ bool decode_fused_plan(int M, int N, int K, int num_sms, int* splits, int* kb_pe
 // tmA: Wq [N rows, K cols] int8, boxes of 128 rows x 128 bytes, 128-byte swizzle.
 cudaError_t launch_decode_fused(const CUtensorMap& tmA, const FusedArgs& a, cudaStream_t stream, bool pdl);
 
+// ------------------------------------------------------------------ column-sharded output (several GPUs)
+constexpr int kUnshardMaxWorld = 64;
+struct UnshardBounds {
+  int64_t bounds[kUnshardMaxWorld + 1];  // block r holds columns [bounds[r], bounds[r+1]) of Y
+};
+// blocks: fp16 [world, M, ld_block] -> Y fp16 [M, bounds[world]] (row stride ldy).
+cudaError_t launch_unshard_columns(const void* blocks, int world, int64_t M, int64_t ld_block, const UnshardBounds& b,
+                                   void* Y, int64_t ldy, int num_sms, cudaStream_t stream);
+
 // ------------------------------------------------------------------ test hooks
 // Each compiled file keeps its own copy of the wait bound and the stall mask
 // (ptx.cuh); these set them, one per file.

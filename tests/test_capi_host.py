@@ -148,6 +148,22 @@ def test_debug_path_accumulator_rejects_invalid_arguments(lib):
     assert call(ws_bytes=512) == capi.ERR_WORKSPACE
 
 
+def test_unshard_rejects_invalid_bounds(lib):
+    import ctypes as C
+    f = lib.llmint8_unshard_columns
+
+    def call(bounds, world=None, M=4, ld=8, ldy=64):
+        b = (C.c_int64 * len(bounds))(*bounds)
+        return f(0x1000, len(bounds) - 1 if world is None else world, M, ld, b, 0x2000, ldy, None)
+    assert call([1, 8]) == capi.ERR_INVALID_ARG          # bounds[0] != 0
+    assert call([0, 8, 4]) == capi.ERR_INVALID_ARG       # decreasing
+    assert call([0, 9]) == capi.ERR_INVALID_ARG          # a block wider than ld_block
+    assert call([0, 0]) == capi.ERR_INVALID_ARG          # N = 0
+    assert call([0, 8, 16], ldy=15) == capi.ERR_INVALID_ARG
+    assert call([0, 8], world=0) == capi.ERR_INVALID_ARG
+    assert f(None, 1, 4, 8, (C.c_int64 * 2)(0, 8), 0x2000, 8, None) == capi.ERR_INVALID_ARG
+
+
 def test_debug_set_waits_rejects_a_zero_bound(lib):
     assert lib.llmint8_debug_set_waits(0, 0) == capi.ERR_INVALID_ARG
 
