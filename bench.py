@@ -35,6 +35,11 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 2.0  # nominal dense ratio, 4.5 POPS int8 / 2.25 PFLOP/s bf16
+INT8_DATASHEET_TOPS = 4500.0  # B200 dense int8, datasheet
+# supplementary configurations of the default line: (workload, threshold or None for its own)
+SUPPLEMENTARY = [("hidden_175b", None), ("sweep8k_o0", None), ("sweep8k_o0p1", None), ("sweep8k_o1", None),
+                 ("sweep8k_o1", float("inf")), ("ragged_1000x1000x1000", None), ("ragged_2047x4095x4100", None),
+                 ("ragged_129x257x520", None), ("ragged_1x1001x1000", None), ("ragged_3x33x24", None)]
 
 
 def parse_args():
@@ -48,6 +53,11 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the supplementary decode-shape measurement")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the supplementary 175B / sweep / ragged measurements")
+    ap.add_argument("--leg-seconds", type=float, default=0.25,
+                    help="device time each supplementary leg is replayed for (clock record; long enough that the "
+                         "power cap applies: its fractions are also given against the sustained peak)")
     ap.add_argument("--graph", action="store_true",
                     help="capture the K timed steps in one CUDA graph (small, launch-bound workloads)")
     return ap.parse_args()
@@ -81,7 +91,7 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
 class ClockSampler:
     """Polls SM clock and clock-event reasons through NVML (read only)."""
 
-    def __init__(self, index: int, period_s: float = 0.01):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.samples = []
         self.period = period_s
         self._stop = threading.Event()
@@ -119,6 +129,15 @@ class ClockSampler:
         self._stop.set()
         if self.ok:
             self.t.join(timeout=2)
+
+    def window(self, t0, t1):
+        """Median SM clock, sample count and reasons seen inside [t0, t1]."""
+        if not self.ok:
+            return {"sm_mhz": None, "samples": 0, "reasons": []}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        reasons = sorted({name for _, _, r in win for bit, name in REASON_BITS.items() if r & bit})
+        return {"sm_mhz": statistics.median([s[1] for s in win]) if win else None, "samples": len(win),
+                "reasons": reasons}
 
     def summary(self, t0, t1):
         if not self.ok:
@@ -313,6 +332,149 @@ def measure_decode(L, torch, dev, peaks, names=("decode_m1", "decode_m8", "decod
     return out
 
 
+# ------------------------------------------------------------------ supplementary configurations
+def replay_for(torch, stream, graph, units_per_replay, seconds, clocks):
+    """Replay `graph` back to back for about `seconds` of device time (at
+    least 3 replays), timed by CUDA events on the replaying stream; returns
+    (us per unit, clock record of the window)."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    one = max(e0.elapsed_time(e1) * 1e-3, 1e-6)
+    reps = max(3, int(math.ceil(seconds / one)))
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * units_per_replay)
+    clk = clocks.window(t0, t1)
+    clk["replays"] = reps
+    return us, clk
+
+
+def capture(torch, fn):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn(torch.cuda.current_stream())
+    g.replay()
+    torch.cuda.synchronize()
+    return g
+
+
+def roofline_times(M, N, K, n_o, peaks):
+    """T_roof = max(2MNK / int8 peak, algorithmic bytes / HBM bandwidth) for
+    the measured peaks and for the datasheet ones."""
+    ops = 2.0 * M * N * K
+    byts = algorithmic_bytes(M, N, K, n_o)
+    meas = (peaks["bf16_tflops"] * INT8_PER_BF16 * 1e12, peaks["hbm_gbs"] * 1e9)
+    sust = (peaks["bf16_tflops_sustained"] * INT8_PER_BF16 * 1e12, peaks["hbm_gbs"] * 1e9)
+    ds = (INT8_DATASHEET_TOPS * 1e12, 8000.0 * 1e9)
+    out = {}
+    # "measured": the burst figures (a kernel timed alone); "sustained": the
+    # measured GEMM rate under the power cap (a kernel timed in a long run);
+    # "datasheet": 4.5 POPS int8, 8 TB/s
+    for tag, (p_int8, bw) in (("measured", meas), ("sustained", sust), ("datasheet", ds)):
+        t_t, t_m = ops / p_int8, byts / bw
+        out[tag] = {"t_roof_us": max(t_t, t_m) * 1e6, "bound": "tensor" if t_t >= t_m else "hbm",
+                    "int8_tops": p_int8 / 1e12, "hbm_gbs": bw / 1e9}
+    return out, byts
+
+
+def measure_config(L, torch, dev, peaks, clocks, name, tau, leg_s):
+    """One supplementary configuration: the whole call (one pass of
+    llmint8_mixed_matmul over rotating input sets > 3x L2, as a CUDA graph),
+    and for the multi-kernel paths the activation step and the GEMM alone,
+    each replayed for about leg_s seconds with its own clock record."""
+    import workloads as wl
+    w = wl.get(name)
+    tau = w.tau if tau is None else tau
+    M, N, K = w.M, w.N, w.K
+    X_np, W_np = wl.make_inputs(w)
+    W = torch.from_numpy(W_np).to(dev)
+    X0 = torch.from_numpy(X_np).to(dev)
+    del W_np
+    Wq0, cs0 = L.quantize_weight_colwise(W)
+    ldq = L.round_up(K, 16)
+    per_set = 2 * M * K + Wq0.numel() + 2 * M * N + M * ldq
+    n_sets = max(2, min(16, math.ceil(3 * L2_BYTES / per_set)))
+    sets = [{"X": X0 if i == 0 else X0.clone(), "Wq": Wq0 if i == 0 else Wq0.clone(),
+             "cs": cs0 if i == 0 else cs0.clone(), "Y": torch.empty((M, N), dtype=torch.float16, device=dev),
+             "ws": L.empty_workspace(M, N, K, K, device=dev)} for i in range(n_sets)]
+    stream = torch.cuda.current_stream()
+
+    def path_pass(on):
+        for st in sets:
+            L.llmint8_mixed_matmul(st["X"], st["Wq"], st["cs"], W, tau, K, st["Y"], st["ws"], on)
+
+    for _ in range(2):
+        path_pass(stream)
+    torch.cuda.synchronize()
+    st_, flags = L.llmint8_check_status(sets[0]["ws"])
+    if st_ != 0:
+        raise RuntimeError(f"device status after {name}: {st_} flags={flags}")
+    n_o = int(L.workspace_views(sets[0]["ws"], M, N, K, K)["n_outlier"].item())
+    kernels = L.llmint8_mixed_matmul_path(sets[0]["X"], sets[0]["Wq"], K)
+    g = capture(torch, path_pass)
+    t_path, clk_path = replay_for(torch, stream, g, n_sets, leg_s, clocks)
+    del g
+    roof, byts = roofline_times(M, N, K, n_o, peaks)
+    ops = 2.0 * M * N * K
+    out = {"M": M, "N": N, "K": K, "tau": tau, "n_outlier": n_o, "kernels": kernels, "us_per_step": t_path,
+           "tops": ops / (t_path * 1e-6) / 1e12, "algorithmic_bytes": byts,
+           "path_frac": {k: v["t_roof_us"] / t_path for k, v in roof.items()}, "roofline": roof,
+           "rotating_sets": n_sets, "clocks": {"path": clk_path}}
+    if len(kernels) > 1:
+        acts = [{"Xq": torch.empty((M, ldq), dtype=torch.int8, device=dev),
+                 "row_scale": torch.empty(M, dtype=torch.float32, device=dev),
+                 "outlier_idx": torch.empty(K, dtype=torch.int32, device=dev),
+                 "n_outlier": torch.empty(1, dtype=torch.int32, device=dev),
+                 "Xo": torch.empty((M, K), dtype=torch.float16, device=dev)} for _ in sets]
+
+        def act_pass(on):
+            for st, a in zip(sets, acts):
+                L.llmint8_quantize_act_rowwise_outliers(st["X"], tau, a["Xq"], a["row_scale"], a["outlier_idx"],
+                                                        a["n_outlier"], a["Xo"], st["ws"], on)
+
+        def gemm_pass(on):
+            for st, a in zip(sets, acts):
+                L.llmint8_mixed_gemm(a["Xq"], a["row_scale"], a["outlier_idx"], a["n_outlier"], a["Xo"], st["Wq"],
+                                     st["cs"], W, K, st["Y"], st["ws"], on)
+
+        act_pass(stream)
+        gemm_pass(stream)
+        torch.cuda.synchronize()
+        g = capture(torch, act_pass)
+        t_act, clk_act = replay_for(torch, stream, g, n_sets, leg_s, clocks)
+        del g
+        g = capture(torch, gemm_pass)
+        t_gemm, clk_gemm = replay_for(torch, stream, g, n_sets, leg_s, clocks)
+        del g, acts
+        out.update({"activation_us": t_act, "gemm_us": t_gemm, "gemm_tops": ops / (t_gemm * 1e-6) / 1e12,
+                    "gemm_frac": {k: ops / (t_gemm * 1e-6) / 1e12 / v["int8_tops"] for k, v in roof.items()},
+                    "activation_gbs": 3 * M * K / (t_act * 1e-6) / 1e9})
+        out["clocks"].update({"activation": clk_act, "gemm": clk_gemm})
+    st_, flags = L.llmint8_check_status(sets[0]["ws"])
+    if st_ != 0:
+        raise RuntimeError(f"device status after {name}: {st_} flags={flags}")
+    del sets, W, X0, Wq0, cs0
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_supplementary(L, torch, dev, peaks, clocks, leg_s):
+    out = {}
+    for name, tau in SUPPLEMENTARY:
+        key = name if tau is None else f"{name}_tau_" + ("inf" if math.isinf(tau) else format(tau, "g"))
+        out[key] = measure_config(L, torch, dev, peaks, clocks, name, tau, leg_s)
+    return out
+
+
 # ------------------------------------------------------------------ our arm
 def source_digest(path):
     with open(path, "rb") as f:
@@ -493,37 +655,64 @@ def run_ours(args, wl_, dist):
                     "frac": gemm_tops / int8_peak, "traffic": traffic,
                     "kernel": "gemm_i8_kernel (tcgen05 kind::i8 + dequant/outlier epilogue)",
                     "peak_note": f"int8 dense = {INT8_PER_BF16:g} x bf16 burst {peaks['bf16_tflops']:.1f} TFLOP/s "
-                                 f"({peaks['source']}); algorithmic ops per launch = 2MNK = {ops:.4g}"}
-        t_roof = max(ops / (int8_peak * 1e12), byts / (peaks["hbm_gbs"] * 1e9))
+                                 f"({peaks['source']}); algorithmic ops per launch = 2MNK = {ops:.4g}",
+                    "peak_datasheet": INT8_DATASHEET_TOPS, "frac_datasheet": gemm_tops / INT8_DATASHEET_TOPS}
+        roof2, _ = roofline_times(M, N, K, n_o, peaks)
+        t_roof = roof2["measured"]["t_roof_us"] * 1e-6
         path = {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step * 1e-3),
-                "algorithmic_bytes": byts, "int8_peak_tops": int8_peak, "hbm_gbs": peaks["hbm_gbs"],
-                "scan_quantize_us": t_quant, "gemm_us": t_gemm,
-                "scan_quantize_gbs": (2 * M * K + M * K) / (t_quant * 1e-6) / 1e9}
+                "frac_datasheet": roof2["datasheet"]["t_roof_us"] / (ms_per_step * 1e3),
+                "t_roof_datasheet_us": roof2["datasheet"]["t_roof_us"],
+                "algorithmic_bytes": byts, "int8_peak_tops": int8_peak, "int8_datasheet_tops": INT8_DATASHEET_TOPS,
+                "hbm_gbs": peaks["hbm_gbs"], "scan_quantize_us": t_quant, "gemm_us": t_gemm,
+                "scan_quantize_gbs": (2 * M * K + M * K) / (t_quant * 1e-6) / 1e9,
+                "legs_note": "gemm_us / scan_quantize_us: the split entry points replayed from CUDA graphs"}
 
-    # ---- end to end through the public API with host buffers
-    Xh = torch.from_numpy(X_np).pin_memory()
-    Yh = torch.empty((M, N), dtype=torch.float16).pin_memory()
+    # ---- end to end through the public API with host buffers: every step
+    # copies its X from pinned host memory and its Y back; the copies run on
+    # two copy streams so that step i's compute overlaps the H2D of step i+1
+    # and the D2H of step i-1 (events order each step's three parts)
     n_e = max(5, min(args.steps, 50))
+    Xh = [torch.from_numpy(X_np).pin_memory() for _ in range(2)]
+    Yh = [torch.empty((M, N), dtype=torch.float16).pin_memory() for _ in range(2)]
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    n_buf = min(n_sets, 3)
 
-    def e2e_step(i):
-        s = sets[i % n_sets]
-        s["X"].copy_(Xh, non_blocking=True)
-        L.llmint8_mixed_matmul(s["X"], s["Wq"], s["cs"], W, wl_.tau, cap, s["Y"], s["ws"], stream)
-        Yh.copy_(s["Y"], non_blocking=True)
+    def e2e_run(n):
+        loaded = [torch.cuda.Event() for _ in range(n)]
+        done = [torch.cuda.Event() for _ in range(n)]
+        copied = [torch.cuda.Event() for _ in range(n)]
+        for i in range(n):
+            s = sets[i % n_buf]
+            with torch.cuda.stream(h2d):
+                if i >= n_buf:
+                    h2d.wait_event(done[i - n_buf])  # the compute that read this X buffer has finished
+                s["X"].copy_(Xh[i % 2], non_blocking=True)
+                loaded[i].record(h2d)
+            stream.wait_event(loaded[i])
+            if i >= n_buf:
+                stream.wait_event(copied[i - n_buf])  # the previous D2H of this Y buffer has finished
+            L.llmint8_mixed_matmul(s["X"], s["Wq"], s["cs"], W, wl_.tau, cap, s["Y"], s["ws"], stream)
+            done[i].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(done[i])
+                Yh[i % 2].copy_(s["Y"], non_blocking=True)
+                copied[i].record(d2h)
+        return copied[-1]
 
-    for i in range(3):
-        e2e_step(i)
+    e2e_run(3)
     torch.cuda.synchronize()
     ev_a.record(stream)
-    for i in range(n_e):
-        e2e_step(i)
+    h2d.wait_event(ev_a)
+    last = e2e_run(n_e)
+    stream.wait_event(last)
     ev_b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = dist.max(torch, ev_a.elapsed_time(ev_b)) / n_e
     e2e = {"value": dist.world * ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
-           "h2d_bytes_per_step": Xh.numel() * 2, "d2h_bytes_per_step": Yh.numel() * 2,
-           "ms_per_step": e2e_ms, "steps": n_e}
-    clocks.stop()
+           "h2d_bytes_per_step": Xh[0].numel() * 2, "d2h_bytes_per_step": Yh[0].numel() * 2,
+           "ms_per_step": e2e_ms, "steps": n_e,
+           "note": "X copied in and Y copied out every step on two copy streams, overlapping the neighbouring "
+                   "steps' compute; timed from the first H2D to the last D2H"}
 
     st, flags = L.llmint8_check_status(sets[0]["ws"])
     if st != 0:
@@ -549,6 +738,11 @@ def run_ours(args, wl_, dist):
     }
     if not args.no_decode and M > 32:
         line["decode"] = measure_decode(L, torch, dev, peaks)
+    if not args.no_configs and M > 32 and dist.world == 1:
+        sets.clear()
+        torch.cuda.empty_cache()
+        line["configs"] = measure_supplementary(L, torch, dev, peaks, clocks, args.leg_seconds)
+    clocks.stop()
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()

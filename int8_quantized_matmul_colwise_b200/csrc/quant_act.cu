@@ -777,6 +777,14 @@ cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx
     cfg.blockDim = dim3(kActFusedThreads);
     cfg.gridDim = dim3(static_cast<unsigned>((M + rows_per - 1) / rows_per));
     cfg.dynamicSmemBytes = smem;
+    // The grid barrier needs every CTA resident at once: a cooperative launch
+    // has the driver guarantee it (the grid is at most one CTA per SM).
+    cudaLaunchAttribute fattr[2];
+    fattr[0].id = cudaLaunchAttributeCooperative;
+    fattr[0].val.cooperative = 1;
+    fattr[1] = attr[0];
+    cfg.attrs = fattr;
+    cfg.numAttrs = pdl ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, kern, x, M, K, ldx, tau, ws, O, n_out, cap, Xq, ldq, rs, static_cast<__half*>(Xo),
                               ldo, static_cast<int>(rows_per), static_cast<int>(cpad));
   }
