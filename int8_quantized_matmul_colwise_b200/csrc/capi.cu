@@ -8,12 +8,22 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kernels.cuh"
 #include "llmint8.h"
 
 using namespace llmint8;
 
 namespace {
+
+// An NVTX range around each entry point's host work and launches, so that a
+// profiler timeline shows which library call issued which kernels (the
+// header-only NVTX calls cost nothing when no tool is attached).
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+};
 
 constexpr int64_t kMaxK = 133143;  // 127^2 * K < 2^31: the int32 accumulator cannot overflow
 constexpr int kMaxDevices = 64;
@@ -216,6 +226,7 @@ llmint8_status llmint8_workspace_layout(int64_t M, int64_t N, int64_t K, int64_t
 
 llmint8_status llmint8_outlier_stats(const void* X, int64_t M, int64_t K, int64_t ldx, float tau, int64_t* stats,
                                      void* ws, size_t ws_bytes, void* stream) {
+  const Range range("llmint8_outlier_stats");
   if (!X || !stats) return LLMINT8_ERR_INVALID_ARG;
   if (M < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || ldx < K || !valid_tau(tau))
     return LLMINT8_ERR_INVALID_ARG;
@@ -275,6 +286,7 @@ llmint8_status llmint8_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 
 llmint8_status llmint8_quantize_weight_colwise(const void* W, int64_t K, int64_t N, int64_t ldw, int8_t* Wq,
                                                int64_t ldk, float* col_scale, void* stream) {
+  const Range range("llmint8_quantize_weight_colwise");
   if (!W || !Wq || !col_scale) return LLMINT8_ERR_INVALID_ARG;
   if (K < 1 || N < 1 || K > kMaxK || N > (int64_t(1) << 31) - 1 || ldw < N) return LLMINT8_ERR_INVALID_ARG;
   if (ldk < K || ldk % 16 != 0 || !aligned(Wq, 16) || !aligned(W, 2) || !aligned(col_scale, 4))
@@ -290,6 +302,7 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
                                                      int32_t* outlier_idx, int64_t outlier_cap,
                                                      int32_t* n_outlier, void* Xo, int64_t ldo, void* ws,
                                                      size_t ws_bytes, void* stream) {
+  const Range range("llmint8_quantize_act_rowwise_outliers");
   if (!X || !Xq || !row_scale || !outlier_idx || !n_outlier) return LLMINT8_ERR_INVALID_ARG;
   if (M < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || ldx < K || !valid_tau(tau))
     return LLMINT8_ERR_INVALID_ARG;
@@ -498,6 +511,7 @@ llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t
                                     int64_t ldk, const float* col_scale, const void* W, int64_t ldw,
                                     const void* bias, int64_t N, float tau, int64_t outlier_cap, void* Y,
                                     int64_t ldy, void* ws, size_t ws_bytes, void* stream) {
+  const Range range("llmint8_mixed_matmul");
   return mixed_matmul_impl(X, M, K, ldx, Wq, ldk, col_scale, W, ldw, bias, N, tau, outlier_cap, Y, ldy, ws, ws_bytes,
                            stream, nullptr, 0);
 }
@@ -506,6 +520,7 @@ llmint8_status llmint8_debug_mixed_matmul_i32(const void* X, int64_t M, int64_t 
                                               int64_t ldk, const float* col_scale, int64_t N, float tau,
                                               int64_t outlier_cap, int32_t* C, int64_t ldc, void* ws,
                                               size_t ws_bytes, void* stream) {
+  const Range range("llmint8_debug_mixed_matmul_i32");
   if (!C) return LLMINT8_ERR_INVALID_ARG;
   // Y is not written on this path; C stands in for the pointer check only
   return mixed_matmul_impl(X, M, K, ldx, Wq, ldk, col_scale, nullptr, 0, nullptr, N, tau, outlier_cap, C, ldc, ws,
@@ -529,6 +544,7 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
                                   const float* col_scale, const void* W, int64_t ldw, const void* bias,
                                   int64_t M, int64_t N, int64_t K, void* Y, int64_t ldy, void* ws,
                                   size_t ws_bytes, void* stream) {
+  const Range range("llmint8_mixed_gemm");
   if (!Xq || !row_scale || !outlier_idx || !n_outlier || !Xo || !Wq || !col_scale || !Y)
     return LLMINT8_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1)
@@ -605,6 +621,7 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
 llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const int8_t* Wq, int64_t ldk,
                                            int64_t M, int64_t N, int64_t K, int32_t* C, int64_t ldc, void* ws,
                                            size_t ws_bytes, void* stream) {
+  const Range range("llmint8_debug_int8_gemm_i32");
   if (!Xq || !Wq || !C) return LLMINT8_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 1 || K > kMaxK || M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1)
     return LLMINT8_ERR_INVALID_ARG;
@@ -650,6 +667,7 @@ llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const 
 
 llmint8_status llmint8_unshard_columns(const void* blocks, int64_t world, int64_t M, int64_t ld_block,
                                       const int64_t* bounds, void* Y, int64_t ldy, void* stream) {
+  const Range range("llmint8_unshard_columns");
   if (!blocks || !bounds || !Y) return LLMINT8_ERR_INVALID_ARG;
   if (world < 1 || world > kUnshardMaxWorld || M < 1 || ld_block < 1) return LLMINT8_ERR_INVALID_ARG;
   if (!aligned(blocks, 2) || !aligned(Y, 2)) return LLMINT8_ERR_INVALID_ARG;
