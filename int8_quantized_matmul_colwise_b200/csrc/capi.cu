@@ -6,6 +6,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include <nvtx3/nvToolsExt.h>
@@ -162,6 +163,11 @@ bool encode_decode_maps(CUtensorMap* tmA, CUtensorMap* tmB, const int8_t* Wq, in
          encode_operand_map(tmB, Xq, M, K, ldq, static_cast<uint32_t>(decode_rows_padded(static_cast<int>(M))));
 }
 
+// Test hook: the stall mask of llmint8_debug_set_waits, passed to the kernels
+// in their launch arguments (0 in normal use).
+std::atomic<uint32_t> g_stall_mask{0};
+uint32_t stall_mask() { return g_stall_mask.load(std::memory_order_relaxed); }
+
 ActWs act_ws(void* ws, size_t colmax_off, size_t bitmask_off, int64_t K) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   ActWs a;
@@ -170,10 +176,12 @@ ActWs act_ws(void* ws, size_t colmax_off, size_t bitmask_off, int64_t K) {
   a.blk_counter = reinterpret_cast<uint32_t*>(b + align_up(colmax_off + 4 * size_t(K), 256));
   a.bitmask = reinterpret_cast<uint32_t*>(b + bitmask_off);
   a.fused = reinterpret_cast<uint32_t*>(b + align_up(bitmask_off + 4 * size_t((K + 31) / 32), 256));
+  a.stall = stall_mask();
   return a;
 }
 
 llmint8_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA; }
+
 
 bool valid_tau(float tau) { return !std::isnan(tau) && tau >= 0.0f; }
 
@@ -391,6 +399,7 @@ llmint8_status mixed_matmul_impl(const void* X, int64_t M, int64_t K, int64_t ld
     g.tiles = g_tiles;
     g.C = C;
     g.ldc = ldc;
+    g.stall = stall_mask();
     return cuda_status(launch_decode_gemv(g, s, true));
   }
 
@@ -493,6 +502,7 @@ llmint8_status mixed_matmul_impl(const void* X, int64_t M, int64_t K, int64_t ld
   a.C = C;
   a.ldc = ldc;
   a.status = reinterpret_cast<uint32_t*>(b + L.status);
+  a.stall = stall_mask();
   CUtensorMap tmY;
   if (C) {
     std::memset(&tmY, 0, sizeof(tmY));
@@ -530,11 +540,12 @@ llmint8_status llmint8_debug_mixed_matmul_i32(const void* X, int64_t M, int64_t 
 llmint8_status llmint8_debug_set_waits(uint64_t limit_ns, uint32_t stall_mask) {
   if (limit_ns == 0) return LLMINT8_ERR_INVALID_ARG;
   if (current_device(nullptr) != LLMINT8_OK) return LLMINT8_ERR_CUDA;
-  cudaError_t (*const setters[])(uint64_t, uint32_t) = {set_debug_waits_decode_fused, set_debug_waits_decode_gemv,
-                                                       set_debug_waits_gemm_i8, set_debug_waits_gemm_i8_decode,
-                                                       set_debug_waits_quant_act};
+  cudaError_t (*const setters[])(uint64_t) = {set_debug_waits_decode_fused, set_debug_waits_decode_gemv,
+                                             set_debug_waits_gemm_i8, set_debug_waits_gemm_i8_decode,
+                                             set_debug_waits_quant_act};
   for (auto fn : setters)
-    if (fn(limit_ns, stall_mask) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (fn(limit_ns) != cudaSuccess) return LLMINT8_ERR_CUDA;
+  g_stall_mask.store(stall_mask, std::memory_order_relaxed);
   return LLMINT8_OK;
 }
 
@@ -613,6 +624,7 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
   a.Y = Y;
   a.ldy = ldy;
   a.status = static_cast<uint32_t*>(ws);
+  a.stall = stall_mask();
   CUtensorMap tmY;
   a.y_tma = prepare_output(&tmY, Y, M, N, ldy);
   return cuda_status(launch_gemm_i8(tmA, tmB, tmY, a, false, num_sms, static_cast<cudaStream_t>(stream), true));

@@ -757,9 +757,7 @@ cudaError_t launch_decode_fused(const CUtensorMap& tmA, const FusedArgs& a, cuda
   }
 }
 
-// Test hook: this file's wait bound and stall mask (see ptx.cuh).
-cudaError_t set_debug_waits_decode_fused(uint64_t limit_ns, uint32_t stall_mask) {
-  return set_debug_waits_in_this_file(limit_ns, stall_mask);
-}
+// Test hook: this file's wait bound (see ptx.cuh).
+cudaError_t set_debug_waits_decode_fused(uint64_t limit_ns) { return set_debug_waits_in_this_file(limit_ns); }
 
 }  // namespace llmint8

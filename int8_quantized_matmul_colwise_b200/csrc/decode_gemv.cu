@@ -361,7 +361,7 @@ __global__ void __launch_bounds__(kThreadsV, 2) decode_gemv_kernel(const GemvArg
   // a5: int8 products
   // (the stall test hook waits on a barrier that nothing arrives on instead:
   // the wait runs out, the copy itself still lands and is waited for below)
-  const bool wok = mbar_wait(stalled(kStallGemvWeight) ? never : wbar, 0, p.status);
+  const bool wok = mbar_wait((p.stall & kStallGemvWeight) ? never : wbar, 0, p.status);
   int32_t d[kTilesV][4];
 #pragma unroll
   for (int tl = 0; tl < kTilesV; ++tl) d[tl][0] = d[tl][1] = d[tl][2] = d[tl][3] = 0;
@@ -586,9 +586,7 @@ cudaError_t launch_decode_gemv(const GemvArgs& a, cudaStream_t stream, bool pdl)
   }
 }
 
-// Test hook: this file's wait bound and stall mask (see ptx.cuh).
-cudaError_t set_debug_waits_decode_gemv(uint64_t limit_ns, uint32_t stall_mask) {
-  return set_debug_waits_in_this_file(limit_ns, stall_mask);
-}
+// Test hook: this file's wait bound (see ptx.cuh).
+cudaError_t set_debug_waits_decode_gemv(uint64_t limit_ns) { return set_debug_waits_in_this_file(limit_ns); }
 
 }  // namespace llmint8

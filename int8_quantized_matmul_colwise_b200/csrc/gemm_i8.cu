@@ -197,7 +197,7 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
 }
 
 template <bool kPair>
-__device__ void run_mma(const Shared& s, uint32_t tmem_base, const Sched& sc, uint32_t* status) {
+__device__ void run_mma(const Shared& s, uint32_t tmem_base, const Sched& sc, uint32_t* status, uint32_t stall) {
   using G = Geo<kPair>;
   constexpr uint32_t idesc = idesc_i8(G::kTileM, BN);
   uint32_t stage = 0, phase = 0, it = 0;
@@ -206,7 +206,7 @@ __device__ void run_mma(const Shared& s, uint32_t tmem_base, const Sched& sc, ui
   // (the stall test hook first waits on the drain barrier, which nothing has
   // arrived on yet: the wait runs out before any MMA is issued and the CTA
   // takes the abort path)
-  if (stalled(kStallGemmOperands) && !wait_or_abort(s.drain, 0, status, s.abort)) ok = false;
+  if ((stall & kStallGemmOperands) && !wait_or_abort(s.drain, 0, status, s.abort)) ok = false;
   for (int tile = sc.first; tile < sc.num_tiles && ok; tile += sc.stride, ++it) {
     const uint32_t b = it & 1u;
     const uint32_t use = (it >> 1) & 1u;
@@ -627,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) run_producer<kPair>(&tmA, &tmB, s, sc, rank, p.status);
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) run_mma<kPair>(s, tmem_base, sc, p.status);
+    if (lane == 0 && rank == 0) run_mma<kPair>(s, tmem_base, sc, p.status, p.stall);
   } else {
     run_epilogue<kRaw, kPair>(p, tmY, s, tmem_base, sc, rank, warp, lane);
   }
@@ -727,9 +727,7 @@ cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const
               : launch_variant<false, false>(tmA, tmB, tmY, a, num_sms, stream, pdl);
 }
 
-// Test hook: this file's wait bound and stall mask (see ptx.cuh).
-cudaError_t set_debug_waits_gemm_i8(uint64_t limit_ns, uint32_t stall_mask) {
-  return set_debug_waits_in_this_file(limit_ns, stall_mask);
-}
+// Test hook: this file's wait bound (see ptx.cuh).
+cudaError_t set_debug_waits_gemm_i8(uint64_t limit_ns) { return set_debug_waits_in_this_file(limit_ns); }
 
 }  // namespace llmint8

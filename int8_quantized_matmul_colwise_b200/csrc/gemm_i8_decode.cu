@@ -387,9 +387,7 @@ cudaError_t launch_gemm_i8_decode(const CUtensorMap& tmA, const CUtensorMap& tmB
                  : launch_decode_variant<false, 32>(tmA, tmB, a, stream, pdl);
 }
 
-// Test hook: this file's wait bound and stall mask (see ptx.cuh).
-cudaError_t set_debug_waits_gemm_i8_decode(uint64_t limit_ns, uint32_t stall_mask) {
-  return set_debug_waits_in_this_file(limit_ns, stall_mask);
-}
+// Test hook: this file's wait bound (see ptx.cuh).
+cudaError_t set_debug_waits_gemm_i8_decode(uint64_t limit_ns) { return set_debug_waits_in_this_file(limit_ns); }
 
 }  // namespace llmint8

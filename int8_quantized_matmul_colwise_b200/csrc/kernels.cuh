@@ -19,6 +19,7 @@ struct ActWs {
   // (this call ORs into one, zeroes the other for the next call); zero-filled
   // once with the workspace.
   uint32_t* fused = nullptr;
+  uint32_t stall = 0;  // test hook: stall mask (ptx.cuh), 0 in normal use
 };
 
 // Bytes of ActWs::fused for K columns (256-byte multiple).
@@ -68,6 +69,7 @@ struct GemmArgs {
   int64_t ldc;
   uint32_t* status;
   bool y_tma;         // Y is written through the tmY tensor map (16-byte aligned rows)
+  uint32_t stall;     // test hook: stall mask (ptx.cuh), 0 in normal use
 };
 
 // Whether the GEMM for M rows runs as CTA pairs (256 x 256 tiles, cta_group::2)
@@ -194,6 +196,7 @@ struct GemvArgs {
   int tiles;     // 16-row MMA tiles covering rows_per (at most 4)
   int32_t* C;    // test hook: non-null stores the int32 accumulator [M, ldc] instead of Y
   int64_t ldc;
+  uint32_t stall;  // test hook: stall mask (ptx.cuh), 0 in normal use
 };
 // Rows per CTA and tiles for a call; false if this kernel does not take the shape.
 bool decode_gemv_plan(int M, int N, int K, int64_t ldk, int num_sms, int* rows_per, int* tiles);
@@ -215,12 +218,12 @@ cudaError_t launch_unshard_columns(const void* blocks, int world, int64_t M, int
                                    void* Y, int64_t ldy, int num_sms, cudaStream_t stream);
 
 // ------------------------------------------------------------------ test hooks
-// Each compiled file keeps its own copy of the wait bound and the stall mask
-// (ptx.cuh); these set them, one per file.
-cudaError_t set_debug_waits_decode_fused(uint64_t limit_ns, uint32_t stall_mask);
-cudaError_t set_debug_waits_decode_gemv(uint64_t limit_ns, uint32_t stall_mask);
-cudaError_t set_debug_waits_gemm_i8(uint64_t limit_ns, uint32_t stall_mask);
-cudaError_t set_debug_waits_gemm_i8_decode(uint64_t limit_ns, uint32_t stall_mask);
-cudaError_t set_debug_waits_quant_act(uint64_t limit_ns, uint32_t stall_mask);
+// Each compiled file keeps its own copy of the wait bound (ptx.cuh); these
+// set it, one per file.  The stall mask travels in the launch arguments.
+cudaError_t set_debug_waits_decode_fused(uint64_t limit_ns);
+cudaError_t set_debug_waits_decode_gemv(uint64_t limit_ns);
+cudaError_t set_debug_waits_gemm_i8(uint64_t limit_ns);
+cudaError_t set_debug_waits_gemm_i8_decode(uint64_t limit_ns);
+cudaError_t set_debug_waits_quant_act(uint64_t limit_ns);
 
 }  // namespace llmint8

@@ -17,27 +17,24 @@ constexpr uint32_t kStatusTimeout = 0x2u;
 // an error status.
 constexpr uint64_t kDefaultWaitLimitNs = 2000ull * 1000ull * 1000ull;
 
-// Test hooks, one copy per compiled file (set together for every file by
-// llmint8_debug_set_waits): the bound of the bounded waits, and a mask of
-// waits that are made to wait for an event that never comes, so that a test
-// can watch the bound run out and the kernel report it through the status
-// word instead of hanging.  Both stay at their defaults in normal use.
+// Test hook, one copy per compiled file (set for every file by
+// llmint8_debug_set_waits): the bound of the bounded waits.  It is read only
+// once a wait has spun for a while, never on a wait that succeeds at once.
 static __device__ uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
-static __device__ uint32_t g_stall_mask = 0u;
 
-// Bits of g_stall_mask (which wait is held back).
+// Bits of the stall mask, the other test hook: waits that are made to wait
+// for an event that never comes, so that a test can watch the bound run out
+// and the kernel report it through the status word instead of hanging.  The
+// mask reaches the kernels as a launch argument (zero in normal use).
 constexpr uint32_t kStallActGridBarrier = 0x1u;  // act_fused_kernel: the grid barrier never completes
 constexpr uint32_t kStallGemvWeight = 0x2u;      // decode_gemv_kernel: the weight copy is never seen to land
 constexpr uint32_t kStallGemmOperands = 0x4u;    // gemm_i8_kernel: the MMA issuer never sees its first stage
 
 __device__ __forceinline__ uint64_t wait_limit_ns() { return *const_cast<volatile uint64_t*>(&g_wait_limit_ns); }
-__device__ __forceinline__ bool stalled(uint32_t bit) { return (g_stall_mask & bit) != 0u; }
 
-// Host side: set this file's copies of the two hooks (synchronous).
-static inline cudaError_t set_debug_waits_in_this_file(uint64_t limit_ns, uint32_t stall_mask) {
-  cudaError_t e = cudaMemcpyToSymbol(g_wait_limit_ns, &limit_ns, sizeof(limit_ns));
-  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_stall_mask, &stall_mask, sizeof(stall_mask));
-  return e;
+// Host side: set this file's copy of the wait bound (synchronous).
+static inline cudaError_t set_debug_waits_in_this_file(uint64_t limit_ns) {
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &limit_ns, sizeof(limit_ns));
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
     int ok = 1;
     // (the stall test hook asks for one arrival more than the grid has: the
     // barrier then never completes and every CTA's wait runs out)
-    const uint32_t last = gridDim.x - 1u + (stalled(kStallActGridBarrier) ? 1u : 0u);
+    const uint32_t last = gridDim.x - 1u + ((ws.stall & kStallActGridBarrier) ? 1u : 0u);
     if (atom_add_acq_rel_gpu_u32(arrived, 1u) == last) {
       *arrived = 0u;                             // for the next call
       st_release_gpu_u32(generation, gen + 1u);  // releases the others
@@ -843,9 +843,7 @@ cudaError_t launch_outlier_stats(const void* X, int64_t M, int64_t K, int64_t ld
                                      static_cast<int>(rows_per), scratch, stats);
 }
 
-// Test hook: this file's wait bound and stall mask (see ptx.cuh).
-cudaError_t set_debug_waits_quant_act(uint64_t limit_ns, uint32_t stall_mask) {
-  return set_debug_waits_in_this_file(limit_ns, stall_mask);
-}
+// Test hook: this file's wait bound (see ptx.cuh).
+cudaError_t set_debug_waits_quant_act(uint64_t limit_ns) { return set_debug_waits_in_this_file(limit_ns); }
 
 }  // namespace llmint8
