@@ -55,6 +55,8 @@ def parse_args():
                     help="skip the supplementary decode-shape measurement")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the supplementary 175B / sweep / ragged measurements")
+    ap.add_argument("--configs", default="",
+                    help="comma-separated subset of the supplementary configurations (default: all)")
     ap.add_argument("--leg-seconds", type=float, default=0.25,
                     help="device time each supplementary leg is replayed for (clock record; long enough that the "
                          "power cap applies: its fractions are also given against the sustained peak)")
@@ -467,10 +469,13 @@ def measure_config(L, torch, dev, peaks, clocks, name, tau, leg_s):
     return out
 
 
-def measure_supplementary(L, torch, dev, peaks, clocks, leg_s):
+def measure_supplementary(L, torch, dev, peaks, clocks, leg_s, only=""):
     out = {}
+    pick = {x for x in only.split(",") if x}
     for name, tau in SUPPLEMENTARY:
         key = name if tau is None else f"{name}_tau_" + ("inf" if math.isinf(tau) else format(tau, "g"))
+        if pick and key not in pick:
+            continue
         out[key] = measure_config(L, torch, dev, peaks, clocks, name, tau, leg_s)
     return out
 
@@ -741,7 +746,7 @@ def run_ours(args, wl_, dist):
     if not args.no_configs and M > 32 and dist.world == 1:
         sets.clear()
         torch.cuda.empty_cache()
-        line["configs"] = measure_supplementary(L, torch, dev, peaks, clocks, args.leg_seconds)
+        line["configs"] = measure_supplementary(L, torch, dev, peaks, clocks, args.leg_seconds, args.configs)
     clocks.stop()
     if dist.rank == 0:
         print(json.dumps(line), flush=True)

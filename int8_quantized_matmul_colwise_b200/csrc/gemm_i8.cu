@@ -56,6 +56,12 @@ constexpr uint32_t kTmemCols = 2 * kAccCols;
 constexpr int kChunk = 32;     // accumulator columns per tcgen05.ld (raw int32 epilogue)
 constexpr int kSG = 16;        // outlier rows of W staged per pass over a tile (one k16 MMA step)
 constexpr int kWoStride = BN + 8;  // halves per staged row: 528 bytes, conflict-free ldmatrix
+// More than kSG outliers: the epilogue walks the tile's 64-column chunks
+// outermost and stages up to kRound outlier rows of W for one chunk at a time,
+// so that each accumulator chunk is read from TMEM once and every pass's MMAs
+// run on it in registers.
+constexpr int kRound = 96;
+constexpr int kWo2Stride = 72;  // halves per staged row of a chunk: 144 bytes, conflict-free ldmatrix
 
 template <bool kPair>
 struct Geo {
@@ -66,8 +72,10 @@ struct Geo {
   static constexpr uint32_t kBytesB = kRowsB * BK;
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kStages * kBytesA;
-  static constexpr uint32_t kOffWo = kOffB + kStages * kBytesB;     // fp16 [kSG][kWoStride]
-  static constexpr uint32_t kOffCs = kOffWo + kSG * kWoStride * 2;  // fp32 [BN]
+  static constexpr uint32_t kOffWo = kOffB + kStages * kBytesB;     // fp16 [kSG][kWoStride] or [kRound][kWo2Stride]
+  static constexpr uint32_t kWoBytes =
+      kSG * kWoStride * 2 > kRound * kWo2Stride * 2 ? kSG * kWoStride * 2 : kRound * kWo2Stride * 2;
+  static constexpr uint32_t kOffCs = kOffWo + kWoBytes;  // fp32 [BN]
   static constexpr uint32_t kOffBias = kOffCs + BN * 4;              // fp32 [BN]
   // per epilogue warp, 16 rows x 64 fp16 columns of Y in the 128-byte swizzle
   static constexpr uint32_t kOffY = (kOffBias + BN * 4 + 1023) & ~1023u;
@@ -288,36 +296,41 @@ __device__ __forceinline__ void stage_scales(const GemmArgs& p, const Shared& s,
   }
 }
 
-// Outlier rows O[t0 .. t0+tn) of W over the tile's BN columns into shared
-// memory (fp16, rows kWoStride apart); rows up to the next multiple of 16 are
-// zero so that a partly used k16 step adds exact zeros.
-__device__ __forceinline__ void stage_outlier_rows(const GemmArgs& p, const Shared& s, int nb, int t0, int tn,
-                                                   int et, bool w_vec) {
+// Outlier rows O[t0 .. t0+tn) of W over the tile's BN columns, as the pieces
+// (8 columns each) this epilogue thread stages: rows up to the next multiple
+// of 16 are zero so that a partly used k16 step adds exact zeros.  Loaded into
+// registers first (load_outlier_rows), so that the loads of the next pass are
+// in flight while the current pass computes, then stored to shared memory
+// (store_outlier_rows, rows kWoStride apart).
+constexpr int kWoPieces = (kSG * (BN / 8) + kEpiThreads - 1) / kEpiThreads;  // pieces per thread (2)
+
+__device__ __forceinline__ void load_outlier_rows(const GemmArgs& p, int nb, int t0, int tn, int et, bool w_vec,
+                                                  uint4 (&u)[kWoPieces]) {
   const __half* W = static_cast<const __half*>(p.W);
   const int n0 = nb * BN;
-  const int rows = (tn + 15) & ~15;
-  const int pieces = rows * (BN / 8);  // 8 columns each
-  for (int pc = et; pc < pieces; pc += kEpiThreads) {
+#pragma unroll
+  for (int k = 0; k < kWoPieces; ++k) {
+    const int pc = et + k * kEpiThreads;
     const int t = pc / (BN / 8);
     const int cc = 8 * (pc % (BN / 8));
     const int c = n0 + cc;
-    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    u[k] = make_uint4(0u, 0u, 0u, 0u);
     if (t < tn && W == nullptr) {  // no fp16 weight kept: the rows recovered from Wq
-      const int64_t k = __ldg(p.O + t0 + t);
+      const int64_t kk = __ldg(p.O + t0 + t);
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int n = c + 2 * e;
-        const uint32_t lo = n < p.N ? dequant_weight_bits(p.Wq[int64_t(n) * p.ldk + k], __ldg(p.cs + n)) : 0u;
+        const uint32_t lo = n < p.N ? dequant_weight_bits(p.Wq[int64_t(n) * p.ldk + kk], __ldg(p.cs + n)) : 0u;
         const uint32_t hi =
-            n + 1 < p.N ? dequant_weight_bits(p.Wq[int64_t(n + 1) * p.ldk + k], __ldg(p.cs + n + 1)) : 0u;
+            n + 1 < p.N ? dequant_weight_bits(p.Wq[int64_t(n + 1) * p.ldk + kk], __ldg(p.cs + n + 1)) : 0u;
         w[e] = lo | (hi << 16);
       }
-      u = make_uint4(w[0], w[1], w[2], w[3]);
+      u[k] = make_uint4(w[0], w[1], w[2], w[3]);
     } else if (t < tn) {
       const __half* wr = W + static_cast<int64_t>(__ldg(p.O + t0 + t)) * p.ldw + c;
       if (w_vec && c + 8 <= p.N) {
-        u = __ldg(reinterpret_cast<const uint4*>(wr));
+        u[k] = __ldg(reinterpret_cast<const uint4*>(wr));
       } else {
         uint32_t w[4];
 #pragma unroll
@@ -326,10 +339,74 @@ __device__ __forceinline__ void stage_outlier_rows(const GemmArgs& p, const Shar
           const uint32_t hi = (c + 2 * e + 1 < p.N) ? __half_as_ushort(wr[2 * e + 1]) : 0u;
           w[e] = lo | (hi << 16);
         }
-        u = make_uint4(w[0], w[1], w[2], w[3]);
+        u[k] = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
-    *reinterpret_cast<uint4*>(s.wo + t * kWoStride + cc) = u;
+  }
+}
+
+__device__ __forceinline__ void store_outlier_rows(const Shared& s, int et, const uint4 (&u)[kWoPieces]) {
+#pragma unroll
+  for (int k = 0; k < kWoPieces; ++k) {
+    const int pc = et + k * kEpiThreads;
+    if (pc < kSG * (BN / 8)) {
+      const int t = pc / (BN / 8);
+      const int cc = 8 * (pc % (BN / 8));
+      *reinterpret_cast<uint4*>(s.wo + t * kWoStride + cc) = u[k];
+    }
+  }
+}
+
+// The same for one 64-column chunk c of the tile and up to kRound outlier rows
+// O[t0 .. t0+tn) (rows kWo2Stride apart, zero up to the next multiple of 16).
+constexpr int kWo2Pieces = (kRound * 8 + kEpiThreads - 1) / kEpiThreads;  // pieces per thread (3)
+
+__device__ __forceinline__ void load_outlier_chunk(const GemmArgs& p, int nb, int c, int t0, int tn, int et,
+                                                   bool w_vec, uint4 (&u)[kWo2Pieces]) {
+  const __half* W = static_cast<const __half*>(p.W);
+  const int n0 = nb * BN + 64 * c;
+#pragma unroll
+  for (int k = 0; k < kWo2Pieces; ++k) {
+    const int pc = et + k * kEpiThreads;
+    const int t = pc >> 3;
+    const int col = n0 + 8 * (pc & 7);
+    u[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (t < tn && W == nullptr) {  // no fp16 weight kept: the rows recovered from Wq
+      const int64_t kk = __ldg(p.O + t0 + t);
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int n = col + 2 * e;
+        const uint32_t lo = n < p.N ? dequant_weight_bits(p.Wq[int64_t(n) * p.ldk + kk], __ldg(p.cs + n)) : 0u;
+        const uint32_t hi =
+            n + 1 < p.N ? dequant_weight_bits(p.Wq[int64_t(n + 1) * p.ldk + kk], __ldg(p.cs + n + 1)) : 0u;
+        w[e] = lo | (hi << 16);
+      }
+      u[k] = make_uint4(w[0], w[1], w[2], w[3]);
+    } else if (t < tn) {
+      const __half* wr = W + static_cast<int64_t>(__ldg(p.O + t0 + t)) * p.ldw + col;
+      if (w_vec && col + 8 <= p.N) {
+        u[k] = __ldg(reinterpret_cast<const uint4*>(wr));
+      } else {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t lo = (col + 2 * e < p.N) ? __half_as_ushort(wr[2 * e]) : 0u;
+          const uint32_t hi = (col + 2 * e + 1 < p.N) ? __half_as_ushort(wr[2 * e + 1]) : 0u;
+          w[e] = lo | (hi << 16);
+        }
+        u[k] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void store_outlier_chunk(const Shared& s, int et, int tn, const uint4 (&u)[kWo2Pieces]) {
+  const int rows = (tn + 15) & ~15;
+#pragma unroll
+  for (int k = 0; k < kWo2Pieces; ++k) {
+    const int pc = et + k * kEpiThreads;
+    if ((pc >> 3) < rows) *reinterpret_cast<uint4*>(s.wo + (pc >> 3) * kWo2Stride + 8 * (pc & 7)) = u[k];
   }
 }
 
@@ -406,7 +483,15 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
     if constexpr (!kRaw) {
       named_bar_sync(1, kEpiThreads);  // the previous tile's readers of the staged data are done
       stage_scales(p, s, nb, et, cs_vec);
-      stage_outlier_rows(p, s, nb, 0, min(n_use, kSG), et, w_vec);
+      if (passes > 1) {  // many outliers: the first chunk's rows of the first round
+        uint4 u[kWo2Pieces];
+        load_outlier_chunk(p, nb, 0, 0, min(n_use, kRound), et, w_vec, u);
+        store_outlier_chunk(s, et, min(n_use, kRound), u);
+      } else {
+        uint4 u[kWoPieces];
+        load_outlier_rows(p, nb, 0, min(n_use, kSG), et, w_vec, u);
+        store_outlier_rows(s, et, u);
+      }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int r = r0 + g + 8 * h;
@@ -442,118 +527,173 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
         }
       }
     } else {
-#pragma unroll 1
-      for (int ps = 0; ps < passes; ++ps) {
-        const int t0 = ps * kSG;
-        const int tn = min(kSG, n_use - t0);
-        const bool last = ps == passes - 1;
-        if (ps > 0) {
-          named_bar_sync(1, kEpiThreads);  // the previous pass's rows are no longer read
-          stage_outlier_rows(p, s, nb, t0, tn, et, w_vec);
-          load_xo_fragment(p, r0, t0, t0 + tn, lane, afr);
-          named_bar_sync(1, kEpiThreads);
+      // a finished 64-column chunk: the bias, then fp16 Y (TMA store through
+      // the swizzled staging tile, or direct stores); an unfinished one (more
+      // rounds of outliers to come) is parked in its own TMEM columns
+      auto finish = [&](int c, float (&d)[8][4], bool last, uint32_t taddr, uint32_t (&v)[32]) {
+        if (last && p.bias != nullptr) {  // the linear layer's bias, added last
+#pragma unroll
+          for (int n = 0; n < 8; ++n) {
+            const float2 b2 = *reinterpret_cast<const float2*>(s.bias + c * 64 + 8 * n + 2 * t4);
+            d[n][0] += b2.x;
+            d[n][1] += b2.y;
+            d[n][2] += b2.x;
+            d[n][3] += b2.y;
+          }
         }
-        {
+        if (last && p.y_tma) {
+          uint32_t lo[8], hi[8];
+#pragma unroll
+          for (int n = 0; n < 8; ++n) {
+            float y0 = d[n][0], y1 = d[n][1], y2 = d[n][2], y3 = d[n][3];
+            if (overflow) y0 = y1 = y2 = y3 = __int_as_float(0x7fc00000);
+            const __half2 a = __floats2half2_rn(y0, y1), bb = __floats2half2_rn(y2, y3);
+            lo[n] = *reinterpret_cast<const uint32_t*>(&a);
+            hi[n] = *reinterpret_cast<const uint32_t*>(&bb);
+          }
+          if (lane == 0) bulk_wait_read_all();  // the previous store has left the staging tile
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t rr = (lane & 7) + 8 * ((lane >> 3) & 1);
+            const uint32_t nn = 2 * i + (lane >> 4);
+            stmatrix_x4(ystage + rr * 128u + ((nn ^ (rr & 7)) << 4), lo[2 * i], hi[2 * i], lo[2 * i + 1],
+                        hi[2 * i + 1]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, s.ystage + ystage_off, nb * BN + c * 64, r0);
+            bulk_commit();
+          }
+        } else if (last) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int r = r0 + g + 8 * h;
+            if (r < p.M) {
+              __half* yr = Y + static_cast<int64_t>(r) * p.ldy;
+#pragma unroll
+              for (int n = 0; n < 8; ++n) {
+                const int col = nb * BN + c * 64 + 8 * n + 2 * t4;
+                float y0 = d[n][2 * h], y1 = d[n][2 * h + 1];
+                if (overflow) y0 = y1 = __int_as_float(0x7fc00000);
+                if (y_pair && col + 1 < p.N) {
+                  *reinterpret_cast<__half2*>(yr + col) = __floats2half2_rn(y0, y1);
+                } else {
+                  if (col < p.N) yr[col] = __float2half_rn(y0);
+                  if (col + 1 < p.N) yr[col + 1] = __float2half_rn(y1);
+                }
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int n = 0; n < 8; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[4 * n + e] = __float_as_uint(d[n][e]);
+          tmem_st_16x256b_x8(taddr, v);
+        }
+      };
+      // dequantize: acc * rs[row] * cs[col] / 127^2
+      auto dequant = [&](int c, const uint32_t (&v)[32], float (&d)[8][4]) {
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+          const float2 c2 = *reinterpret_cast<const float2*>(s.cs + c * 64 + 8 * n + 2 * t4);
+          d[n][0] = i2f_exact(static_cast<int32_t>(v[4 * n + 0])) * rsc[0] * c2.x;
+          d[n][1] = i2f_exact(static_cast<int32_t>(v[4 * n + 1])) * rsc[0] * c2.y;
+          d[n][2] = i2f_exact(static_cast<int32_t>(v[4 * n + 2])) * rsc[1] * c2.x;
+          d[n][3] = i2f_exact(static_cast<int32_t>(v[4 * n + 3])) * rsc[1] * c2.y;
+        }
+      };
+      if (passes <= 1) {
+        // at most 16 outliers: their W rows over the whole tile were staged
+        // before the accumulator wait; one k16 step of the 16-bit product
 #pragma unroll 1
-          for (int c = 0; c < BN / 64; ++c) {  // 64 accumulator columns at a time
+        for (int c = 0; c < BN / 64; ++c) {  // 64 accumulator columns at a time
+          const uint32_t taddr = tacc + c * 64;
+          uint32_t v[32];
+          tmem_ld_16x256b_x8(taddr, v);
+          tmem_ld_wait();
+          float d[8][4];
+          dequant(c, v, d);
+          // 16-bit outlier product on the tensor cores: d += Xo[rows, k] * W[O[k], cols]
+          if (n_use > 0) {
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+              uint32_t b0, b1, b2, b3;
+              ldmatrix_x4_trans(wo_lane + 2u * static_cast<uint32_t>(c * 64 + 16 * np), b0, b1, b2, b3);
+              mma_m16n8k16_f16f32(d[2 * np], afr, b0, b1);
+              mma_m16n8k16_f16f32(d[2 * np + 1], afr, b2, b3);
+            }
+          }
+          finish(c, d, true, taddr, v);
+        }
+      } else {
+        // more than 16 outliers: rounds of up to kRound, and inside a round
+        // the 64-column chunks outermost, each staging the round's W rows for
+        // its 64 columns (the next chunk's rows loaded into registers while this
+        // one computes); the accumulator chunk is read once per round and all
+        // the round's k16 steps run on it in registers
+        const int rounds = (n_use + kRound - 1) / kRound;
+        const uint32_t wo2_lane =
+            smem_u32(s.wo) + 2u * static_cast<uint32_t>(((lane & 7) + 8 * ((lane >> 3) & 1)) * kWo2Stride + 8 * (lane >> 4));
+        uint4 wn[kWo2Pieces];
+        uint32_t ax[kRound / kSG][4];  // Xo fragments of the round's k16 steps
+#pragma unroll 1
+        for (int rnd = 0; rnd < rounds; ++rnd) {
+          const int tr0 = rnd * kRound;
+          const int trn = min(kRound, n_use - tr0);
+          const int pr = (trn + kSG - 1) / kSG;
+          const bool last = rnd == rounds - 1;
+#pragma unroll
+          for (int q = 0; q < kRound / kSG; ++q)
+            if (q < pr) load_xo_fragment(p, r0, tr0 + kSG * q, tr0 + min(kSG * (q + 1), trn), lane, ax[q]);
+#pragma unroll 1
+          for (int c = 0; c < BN / 64; ++c) {
+            if (rnd > 0 || c > 0) {
+              named_bar_sync(1, kEpiThreads);  // the previous chunk's rows are no longer read
+              store_outlier_chunk(s, et, trn, wn);
+              named_bar_sync(1, kEpiThreads);
+            }
+            {
+              int nrd = rnd, nc = c + 1;
+              if (nc == BN / 64) {
+                nc = 0;
+                ++nrd;
+              }
+              if (nrd < rounds)
+                load_outlier_chunk(p, nb, nc, nrd * kRound, min(kRound, n_use - nrd * kRound), et, w_vec, wn);
+            }
             const uint32_t taddr = tacc + c * 64;
             uint32_t v[32];
             tmem_ld_16x256b_x8(taddr, v);
             tmem_ld_wait();
             float d[8][4];
-            if (ps == 0) {
-              // dequantize: acc * rs[row] * cs[col] / 127^2
-#pragma unroll
-              for (int n = 0; n < 8; ++n) {
-                const float2 c2 = *reinterpret_cast<const float2*>(s.cs + c * 64 + 8 * n + 2 * t4);
-                d[n][0] = i2f_exact(static_cast<int32_t>(v[4 * n + 0])) * rsc[0] * c2.x;
-                d[n][1] = i2f_exact(static_cast<int32_t>(v[4 * n + 1])) * rsc[0] * c2.y;
-                d[n][2] = i2f_exact(static_cast<int32_t>(v[4 * n + 2])) * rsc[1] * c2.x;
-                d[n][3] = i2f_exact(static_cast<int32_t>(v[4 * n + 3])) * rsc[1] * c2.y;
-              }
+            if (rnd == 0) {
+              dequant(c, v, d);
             } else {
 #pragma unroll
               for (int n = 0; n < 8; ++n)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) d[n][e] = __uint_as_float(v[4 * n + e]);
             }
-            // 16-bit outlier product on the tensor cores: d += Xo[rows, k] * W[O[k], cols]
-            if (tn > 0) {
 #pragma unroll
-              for (int np = 0; np < 4; ++np) {
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4_trans(wo_lane + 2u * static_cast<uint32_t>(c * 64 + 16 * np), b0, b1, b2, b3);
-                mma_m16n8k16_f16f32(d[2 * np], afr, b0, b1);
-                mma_m16n8k16_f16f32(d[2 * np + 1], afr, b2, b3);
-              }
-            }
-            if (last && p.bias != nullptr) {  // the linear layer's bias, added last
+            for (int q = 0; q < kRound / kSG; ++q) {
+              if (q < pr) {
 #pragma unroll
-              for (int n = 0; n < 8; ++n) {
-                const float2 b2 = *reinterpret_cast<const float2*>(s.bias + c * 64 + 8 * n + 2 * t4);
-                d[n][0] += b2.x;
-                d[n][1] += b2.y;
-                d[n][2] += b2.x;
-                d[n][3] += b2.y;
-              }
-            }
-            if (last && p.y_tma) {
-              // fp16 fragment -> swizzled staging tile (stmatrix) -> TMA store
-              uint32_t lo[8], hi[8];
-#pragma unroll
-              for (int n = 0; n < 8; ++n) {
-                float y0 = d[n][0], y1 = d[n][1], y2 = d[n][2], y3 = d[n][3];
-                if (overflow) y0 = y1 = y2 = y3 = __int_as_float(0x7fc00000);
-                const __half2 a = __floats2half2_rn(y0, y1), bb = __floats2half2_rn(y2, y3);
-                lo[n] = *reinterpret_cast<const uint32_t*>(&a);
-                hi[n] = *reinterpret_cast<const uint32_t*>(&bb);
-              }
-              if (lane == 0) bulk_wait_read_all();  // the previous store has left the staging tile
-              __syncwarp();
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const uint32_t rr = (lane & 7) + 8 * ((lane >> 3) & 1);
-                const uint32_t nn = 2 * i + (lane >> 4);
-                stmatrix_x4(ystage + rr * 128u + ((nn ^ (rr & 7)) << 4), lo[2 * i], hi[2 * i], lo[2 * i + 1],
-                            hi[2 * i + 1]);
-              }
-              fence_proxy_async_smem();
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_2d(&tmY, s.ystage + ystage_off, nb * BN + c * 64, r0);
-                bulk_commit();
-              }
-            } else if (last) {
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int r = r0 + g + 8 * h;
-                if (r < p.M) {
-                  __half* yr = Y + static_cast<int64_t>(r) * p.ldy;
-#pragma unroll
-                  for (int n = 0; n < 8; ++n) {
-                    const int col = nb * BN + c * 64 + 8 * n + 2 * t4;
-                    float y0 = d[n][2 * h], y1 = d[n][2 * h + 1];
-                    if (overflow) y0 = y1 = __int_as_float(0x7fc00000);
-                    if (y_pair && col + 1 < p.N) {
-                      *reinterpret_cast<__half2*>(yr + col) = __floats2half2_rn(y0, y1);
-                    } else {
-                      if (col < p.N) yr[col] = __float2half_rn(y0);
-                      if (col + 1 < p.N) yr[col + 1] = __float2half_rn(y1);
-                    }
-                  }
+                for (int np = 0; np < 4; ++np) {
+                  uint32_t b0, b1, b2, b3;
+                  ldmatrix_x4_trans(wo2_lane + 2u * static_cast<uint32_t>(q * kSG * kWo2Stride + 16 * np), b0, b1,
+                                    b2, b3);
+                  mma_m16n8k16_f16f32(d[2 * np], ax[q], b0, b1);
+                  mma_m16n8k16_f16f32(d[2 * np + 1], ax[q], b2, b3);
                 }
               }
-            } else {
-              // park the partial sum in the accumulator's own TMEM columns
-#pragma unroll
-              for (int n = 0; n < 8; ++n)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) v[4 * n + e] = __float_as_uint(d[n][e]);
-              tmem_st_16x256b_x8(taddr, v);
             }
+            finish(c, d, last, taddr, v);
           }
+          if (!last) tmem_st_wait();
         }
-        if (!last) tmem_st_wait();
       }
     }
     // this warp's TMEM reads of buffer b are complete: free it for the MMA

@@ -162,6 +162,19 @@ __device__ __forceinline__ void build_outlier_set(int64_t K, const ActWs& ws, ui
   __syncthreads();
 }
 
+// Column of the t-th outlier (t < n_o) from the bitmask and its word prefix.
+__device__ __forceinline__ int outlier_col(int t, const uint32_t* mask, const uint32_t* pre, int nwords) {
+  int lo = 0, hi = nwords - 1;  // last word whose prefix is <= t
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (static_cast<int>(pre[mid]) <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  uint32_t bits = mask[lo];
+  for (int skip = t - static_cast<int>(pre[lo]); skip > 0; --skip) bits &= bits - 1;
+  return lo * 32 + __ffs(bits) - 1;
+}
+
 // ----------------------------------------------------------------- a2-a4
 // Row quantizer: a group of G threads owns one row and holds its CPT chunks
 // of 8 columns in registers (G * CPT * 8 >= K).  256 threads per CTA, 256 / G
@@ -208,25 +221,21 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_kernel(const __half* __r
 #pragma unroll
   for (int j = 0; j < CPT; ++j) any_outlier |= flags(j);
 
-  // a4: gather X[row, O[t]] for the outlier product, from the registers: the
-  // outlier column c sits at position prefix(word) + popcount(lower bits).
-  // Outlier columns are then zeroed in the registers (0 quantizes to 0).
+  // a4: gather X[row, O[t]] for the outlier product by outlier number: thread
+  // gt of the row's group takes outliers gt, gt + G, .. (the row is in L2:
+  // its loads were just issued), so the stores to Xo are contiguous and no
+  // thread walks its chunks for outlier bits.
+  if (Xo != nullptr && row_ok) {
+    const int n_o = static_cast<int>(s_pre[nwords - 1]) + __popc(s_mask[nwords - 1]);
+    const int n = static_cast<int>(min(int64_t(n_o), cap));
+    for (int t = gt; t < n; t += G) Xo[row * ldo + t] = xr[outlier_col(t, s_mask, s_pre, static_cast<int>(nwords))];
+  }
+  // outlier columns are zeroed in the registers (0 quantizes to 0)
   if (any_outlier != 0u) {
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
       const uint32_t om = flags(j);
       if (om != 0u) {
-        const int64_t c = 8 * (int64_t(gt) + int64_t(j) * G);
-        const uint32_t word = s_mask[c >> 5];
-        const uint32_t base = s_pre[c >> 5];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if ((om >> e) & 1u) {
-            const int b = static_cast<int>((c & 31) + e);
-            const int64_t pos = base + __popc(word & ((1u << b) - 1u));
-            if (Xo != nullptr && row_ok && pos < cap) Xo[row * ldo + pos] = __ushort_as_half(half_bits_at(h[j], e));
-          }
-        }
         uint32_t* w = reinterpret_cast<uint32_t*>(&h[j]);
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -347,11 +356,12 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
   griddep_wait();  // X may be written by the preceding kernel
   griddep_launch_dependents();
   if (tid == 0) {
-    s_gen = ld_acquire_gpu_u32(generation);
-    // this CTA's rows, one bulk copy each
+    // this CTA's rows, one bulk copy each, issued before the generation word
+    // is read (an L2 round trip the copies need not wait for)
     mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nr) * static_cast<uint32_t>(K) * 2u);
     for (int r = 0; r < nr; ++r)
       bulk_load_1d(s_x + size_t(r) * size_t(K), X + (r0 + r) * ldx, static_cast<uint32_t>(K) * 2u, &bar);
+    s_gen = ld_acquire_gpu_u32(generation);
   }
   __syncthreads();
   const uint32_t gen = s_gen;
