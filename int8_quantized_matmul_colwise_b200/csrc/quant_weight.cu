@@ -15,101 +15,127 @@ namespace llmint8 {
 namespace {
 
 constexpr int kStripCols = 64;   // columns of W per CTA
-constexpr int kKBlock = 128;     // rows of W per transpose block
+constexpr int kMaxRows = 256;    // rows of W per CTA in the column-maximum pass
+constexpr int kKBlock = 128;     // rows of W per CTA in the quantize pass (one transposed block)
 constexpr int kTStride = 144;    // bytes per transposed row in shared memory
 
 // Load 8 consecutive fp16 of row k starting at column c (zero outside N).
-__device__ __forceinline__ void load8(const __half* __restrict__ W, int64_t ldw, int64_t N, int64_t k, int64_t c,
-                                      bool vec_ok, float (&x)[8]) {
+__device__ __forceinline__ uint4 load8w(const __half* __restrict__ W, int64_t ldw, int64_t N, int64_t k, int64_t c,
+                                        bool vec_ok) {
   const __half* p = W + k * ldw + c;
-  if (vec_ok && c + 8 <= N) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-    const __half2* h = reinterpret_cast<const __half2*>(&u);
+  if (vec_ok && c + 8 <= N) return __ldg(reinterpret_cast<const uint4*>(p));
+  uint32_t w[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __half22float2(h[e]);
-      x[2 * e] = f.x;
-      x[2 * e + 1] = f.y;
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] = (c + e < N) ? __half2float(p[e]) : 0.0f;
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t lo = (c + 2 * e < N) ? __half_as_ushort(p[2 * e]) : 0u;
+    const uint32_t hi = (c + 2 * e + 1 < N) ? __half_as_ushort(p[2 * e + 1]) : 0u;
+    w[e] = lo | (hi << 16);
   }
+  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// One CTA owns a strip of 64 columns over all K rows: first the exact column
-// absmax, then quantization of 128-row blocks transposed through shared memory
-// so that each column of W becomes one K-contiguous row of Wq.
-__global__ void __launch_bounds__(256) quantize_weight_colwise_kernel(const __half* __restrict__ W, int64_t K,
-                                                                      int64_t N, int64_t ldw, bool vec_ok,
-                                                                      int8_t* __restrict__ Wq, int64_t ldk,
-                                                                      float* __restrict__ col_scale) {
+// Pass 1: column maxima of |W| over a block of kMaxRows rows and a strip of 64
+// columns, merged into col_scale (zero-filled first) by an atomic max on the
+// bit patterns (non-negative floats order like their bits; NaN never wins).
+__global__ void __launch_bounds__(256) weight_colmax_kernel(const __half* __restrict__ W, int64_t K, int64_t N,
+                                                            int64_t ldw, bool vec_ok, float* __restrict__ col_scale) {
   __shared__ float s_red[32][kStripCols + 1];
-  __shared__ float s_scale[kStripCols];
-  __shared__ float s_inv[kStripCols];
-  __shared__ __align__(16) int8_t s_t[kStripCols][kTStride];
-
   const int64_t c0 = int64_t(blockIdx.x) * kStripCols;
+  const int64_t k0 = int64_t(blockIdx.y) * kMaxRows;
   const int tx = threadIdx.x & 7;   // column group: 8 columns
   const int ty = threadIdx.x >> 3;  // row phase 0..31
   const int64_t cg = c0 + 8 * tx;
-
-  float m[8];
+  __half2 m[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) m[e] = 0.0f;
-  for (int64_t k = ty; k < K; k += 32) {
-    float x[8];
-    load8(W, ldw, N, k, cg, vec_ok, x);
+  for (int e = 0; e < 4; ++e) m[e] = __half2half2(__ushort_as_half(0));
+  uint4 u[kMaxRows / 32];  // all of the thread's loads in flight together
 #pragma unroll
-    for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(x[e]));
+  for (int r = 0; r < kMaxRows / 32; ++r) {
+    const int64_t k = k0 + ty + 32 * r;
+    u[r] = (k < K && cg < N) ? load8w(W, ldw, N, k, cg, vec_ok) : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) s_red[ty][8 * tx + e] = m[e];
+  for (int r = 0; r < kMaxRows / 32; ++r) {
+    const __half2* h2 = reinterpret_cast<const __half2*>(&u[r]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) m[e] = __hmax2(m[e], __habs2(h2[e]));  // NaN never wins
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(m[e]);
+    s_red[ty][8 * tx + 2 * e] = f.x;
+    s_red[ty][8 * tx + 2 * e + 1] = f.y;
+  }
   __syncthreads();
+  if (threadIdx.x < kStripCols && c0 + threadIdx.x < N) {
+    float v = 0.0f;
+    for (int r = 0; r < 32; ++r) v = fmaxf(v, s_red[r][threadIdx.x]);
+    if (v > 0.0f) atomicMax(reinterpret_cast<unsigned int*>(col_scale) + c0 + threadIdx.x, __float_as_uint(v));
+  }
+}
+
+// Pass 2: codes of a block of 128 rows x 64 columns, transposed through shared
+// memory so that each column of W becomes one K-contiguous run of Wq (rows k
+// in [K, ldk) are written as zero).  Per value: r = x * fl(127 / s) rounded to
+// the nearest integer, which is the exact round-half-away-from-zero result
+// unless r lies within 2^-15 of a half-integer; then the exact comparisons
+// decide (quantize_exact).
+__global__ void __launch_bounds__(256) weight_quantize_kernel(const __half* __restrict__ W, int64_t K, int64_t N,
+                                                              int64_t ldw, bool vec_ok,
+                                                              const float* __restrict__ col_scale,
+                                                              int8_t* __restrict__ Wq, int64_t ldk) {
+  __shared__ float s_scale[kStripCols];
+  __shared__ float s_k[kStripCols];
+  __shared__ float s_inv[kStripCols];
+  __shared__ __align__(16) int8_t s_t[kStripCols][kTStride];
+  const int64_t c0 = int64_t(blockIdx.x) * kStripCols;
+  const int64_t k0 = int64_t(blockIdx.y) * kKBlock;
+  const int tx = threadIdx.x & 7;
+  const int ty = threadIdx.x >> 3;
+  const int64_t cg = c0 + 8 * tx;
+  uint4 u[kKBlock / 32];
+#pragma unroll
+  for (int r = 0; r < kKBlock / 32; ++r) {
+    const int64_t k = k0 + ty + 32 * r;
+    u[r] = (k < K && cg < N) ? load8w(W, ldw, N, k, cg, vec_ok) : make_uint4(0u, 0u, 0u, 0u);
+  }
   if (threadIdx.x < kStripCols) {
-    float s = 0.0f;
-    for (int r = 0; r < 32; ++r) s = fmaxf(s, s_red[r][threadIdx.x]);
-    s_scale[threadIdx.x] = s;
-    s_inv[threadIdx.x] = s > 0.0f ? __frcp_rn(s) : 0.0f;
-    if (c0 + threadIdx.x < N) col_scale[c0 + threadIdx.x] = s;
+    const float sc = c0 + threadIdx.x < N ? __ldg(col_scale + c0 + threadIdx.x) : 0.0f;
+    s_scale[threadIdx.x] = sc;
+    s_k[threadIdx.x] = sc > 0.0f ? __fdiv_rn(127.0f, sc) : 0.0f;
+    s_inv[threadIdx.x] = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
   }
   __syncthreads();
-
-  // Transposed write-out: thread -> (column wc, 32-byte segment ws).
+  constexpr float kSafe = 0.499969482421875f;  // 1/2 - 2^-15
+  constexpr float kBias = 12582912.0f;         // 1.5 * 2^23
+#pragma unroll
+  for (int r = 0; r < kKBlock / 32; ++r) {
+    const int kr = ty + 32 * r;
+    const __half2* h2 = reinterpret_cast<const __half2*>(&u[r]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int c = 8 * tx + e;
+      const float x = (e & 1) ? __high2float(h2[e >> 1]) : __low2float(h2[e >> 1]);
+      const float rr = __fmul_rn(x, s_k[c]);
+      const float t = __fadd_rn(rr, kBias);
+      const float qf = __fadd_rn(t, -kBias);
+      int q = static_cast<int>(static_cast<int8_t>(__float_as_uint(t) & 0xFFu));
+      if (!(fabsf(__fadd_rn(rr, -qf)) < kSafe)) q = s_scale[c] > 0.0f ? quantize_exact(x, s_scale[c], s_inv[c]) : 0;
+      s_t[c][kr] = static_cast<int8_t>(q);
+    }
+  }
+  __syncthreads();
+  // thread -> (column wc, 32-byte segment): two 16-byte stores
   const int wc = threadIdx.x >> 2;
   const int wseg = threadIdx.x & 3;
-  for (int64_t k0 = 0; k0 < ldk; k0 += kKBlock) {
+  const int64_t col = c0 + wc;
+  if (col < N) {
 #pragma unroll
-    for (int r = 0; r < kKBlock / 32; ++r) {
-      const int kr = ty + 32 * r;
-      const int64_t k = k0 + kr;
-      float x[8];
-      if (k < K) {
-        load8(W, ldw, N, k, cg, vec_ok, x);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = 0.0f;
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int c = 8 * tx + e;
-        const float s = s_scale[c];
-        s_t[c][kr] = static_cast<int8_t>(s > 0.0f ? quantize_exact(x[e], s, s_inv[c]) : 0);
-      }
+    for (int h = 0; h < 2; ++h) {
+      const int64_t kk = k0 + 32 * wseg + 16 * h;
+      if (kk < ldk)  // ldk % 16 == 0, so a 16-byte piece is either in or out
+        *reinterpret_cast<uint4*>(Wq + col * ldk + kk) = *reinterpret_cast<const uint4*>(&s_t[wc][32 * wseg + 16 * h]);
     }
-    __syncthreads();
-    const int64_t col = c0 + wc;
-    if (col < N) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t kk = k0 + 32 * wseg + 16 * h;
-        if (kk < ldk) {  // ldk % 16 == 0, so a 16-byte piece is either in or out
-          *reinterpret_cast<uint4*>(Wq + col * ldk + kk) =
-              *reinterpret_cast<const uint4*>(&s_t[wc][32 * wseg + 16 * h]);
-        }
-      }
-    }
-    __syncthreads();
   }
 }
 
@@ -118,9 +144,16 @@ __global__ void __launch_bounds__(256) quantize_weight_colwise_kernel(const __ha
 cudaError_t launch_quantize_weight_colwise(const void* W, int64_t K, int64_t N, int64_t ldw, int8_t* Wq,
                                            int64_t ldk, float* col_scale, cudaStream_t stream) {
   const bool vec_ok = (ldw % 8 == 0) && (reinterpret_cast<uintptr_t>(W) % 16 == 0);
-  const unsigned grid = static_cast<unsigned>((N + kStripCols - 1) / kStripCols);
-  quantize_weight_colwise_kernel<<<grid, 256, 0, stream>>>(static_cast<const __half*>(W), K, N, ldw, vec_ok, Wq,
-                                                           ldk, col_scale);
+  const __half* w = static_cast<const __half*>(W);
+  const unsigned strips = static_cast<unsigned>((N + kStripCols - 1) / kStripCols);
+  cudaError_t e = cudaMemsetAsync(col_scale, 0, size_t(N) * sizeof(float), stream);
+  if (e != cudaSuccess) return e;
+  weight_colmax_kernel<<<dim3(strips, static_cast<unsigned>((K + kMaxRows - 1) / kMaxRows)), 256, 0, stream>>>(
+      w, K, N, ldw, vec_ok, col_scale);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  weight_quantize_kernel<<<dim3(strips, static_cast<unsigned>((ldk + kKBlock - 1) / kKBlock)), 256, 0, stream>>>(
+      w, K, N, ldw, vec_ok, col_scale, Wq, ldk);
   return cudaGetLastError();
 }
 
