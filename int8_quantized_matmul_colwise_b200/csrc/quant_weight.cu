@@ -76,10 +76,13 @@ __global__ void __launch_bounds__(256) weight_colmax_kernel(const __half* __rest
 
 // Pass 2: codes of a block of 128 rows x 64 columns, transposed through shared
 // memory so that each column of W becomes one K-contiguous run of Wq (rows k
-// in [K, ldk) are written as zero).  Per value: r = x * fl(127 / s) rounded to
-// the nearest integer, which is the exact round-half-away-from-zero result
-// unless r lies within 2^-15 of a half-integer; then the exact comparisons
-// decide (quantize_exact).
+// in [K, ldk) are written as zero).  Thread (tx, rg) holds columns 8 tx .. +7
+// of rows 4 rg .. 4 rg + 3, so each column's four codes are one 32-bit word;
+// the 16-byte pieces of a transposed row are permuted by the writer's column
+// group (piece index XOR tx), which puts a warp's 32 stores in 32 different
+// banks.  Per value: r = x * fl(127 / s) rounded to the nearest integer, which
+// is the exact round-half-away-from-zero result unless r lies within 2^-15 of
+// a half-integer; then the exact comparisons decide (quantize_exact).
 __global__ void __launch_bounds__(256) weight_quantize_kernel(const __half* __restrict__ W, int64_t K, int64_t N,
                                                               int64_t ldw, bool vec_ok,
                                                               const float* __restrict__ col_scale,
@@ -90,14 +93,14 @@ __global__ void __launch_bounds__(256) weight_quantize_kernel(const __half* __re
   __shared__ __align__(16) int8_t s_t[kStripCols][kTStride];
   const int64_t c0 = int64_t(blockIdx.x) * kStripCols;
   const int64_t k0 = int64_t(blockIdx.y) * kKBlock;
-  const int tx = threadIdx.x & 7;
-  const int ty = threadIdx.x >> 3;
+  const int tx = threadIdx.x & 7;   // column group: columns 8 tx .. 8 tx + 7
+  const int rg = threadIdx.x >> 3;  // row group: rows 4 rg .. 4 rg + 3 of the block
   const int64_t cg = c0 + 8 * tx;
-  uint4 u[kKBlock / 32];
+  uint4 u[4];
 #pragma unroll
-  for (int r = 0; r < kKBlock / 32; ++r) {
-    const int64_t k = k0 + ty + 32 * r;
-    u[r] = (k < K && cg < N) ? load8w(W, ldw, N, k, cg, vec_ok) : make_uint4(0u, 0u, 0u, 0u);
+  for (int j = 0; j < 4; ++j) {
+    const int64_t k = k0 + 4 * rg + j;
+    u[j] = (k < K && cg < N) ? load8w(W, ldw, N, k, cg, vec_ok) : make_uint4(0u, 0u, 0u, 0u);
   }
   if (threadIdx.x < kStripCols) {
     const float sc = c0 + threadIdx.x < N ? __ldg(col_scale + c0 + threadIdx.x) : 0.0f;
@@ -108,33 +111,40 @@ __global__ void __launch_bounds__(256) weight_quantize_kernel(const __half* __re
   __syncthreads();
   constexpr float kSafe = 0.499969482421875f;  // 1/2 - 2^-15
   constexpr float kBias = 12582912.0f;         // 1.5 * 2^23
+  // byte offset of rows 4 rg .. 4 rg + 3 inside a transposed row: piece (rg / 4) ^ tx
+  const int wofs = 16 * ((rg >> 2) ^ tx) + 4 * (rg & 3);
 #pragma unroll
-  for (int r = 0; r < kKBlock / 32; ++r) {
-    const int kr = ty + 32 * r;
-    const __half2* h2 = reinterpret_cast<const __half2*>(&u[r]);
+  for (int e = 0; e < 8; ++e) {
+    const int c = 8 * tx + e;
+    const float kc = s_k[c];
+    uint32_t word = 0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int c = 8 * tx + e;
+    for (int j = 0; j < 4; ++j) {
+      const __half2* h2 = reinterpret_cast<const __half2*>(&u[j]);
       const float x = (e & 1) ? __high2float(h2[e >> 1]) : __low2float(h2[e >> 1]);
-      const float rr = __fmul_rn(x, s_k[c]);
+      const float rr = __fmul_rn(x, kc);
       const float t = __fadd_rn(rr, kBias);
       const float qf = __fadd_rn(t, -kBias);
-      int q = static_cast<int>(static_cast<int8_t>(__float_as_uint(t) & 0xFFu));
-      if (!(fabsf(__fadd_rn(rr, -qf)) < kSafe)) q = s_scale[c] > 0.0f ? quantize_exact(x, s_scale[c], s_inv[c]) : 0;
-      s_t[c][kr] = static_cast<int8_t>(q);
+      uint32_t q = __float_as_uint(t) & 0xFFu;  // the low byte of rint(r), two's complement
+      if (!(fabsf(__fadd_rn(rr, -qf)) < kSafe))
+        q = static_cast<uint32_t>(s_scale[c] > 0.0f ? quantize_exact(x, s_scale[c], s_inv[c]) : 0) & 0xFFu;
+      word |= q << (8 * j);
     }
+    *reinterpret_cast<uint32_t*>(&s_t[c][wofs]) = word;
   }
   __syncthreads();
-  // thread -> (column wc, 32-byte segment): two 16-byte stores
+  // thread -> (column wc, 32-byte segment): two 16-byte pieces, un-permuted
   const int wc = threadIdx.x >> 2;
   const int wseg = threadIdx.x & 3;
+  const int wperm = (wc >> 3) & 7;  // the column group that wrote row wc
   const int64_t col = c0 + wc;
   if (col < N) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int64_t kk = k0 + 32 * wseg + 16 * h;
+      const int piece = 2 * wseg + h;
+      const int64_t kk = k0 + 16 * piece;
       if (kk < ldk)  // ldk % 16 == 0, so a 16-byte piece is either in or out
-        *reinterpret_cast<uint4*>(Wq + col * ldk + kk) = *reinterpret_cast<const uint4*>(&s_t[wc][32 * wseg + 16 * h]);
+        *reinterpret_cast<uint4*>(Wq + col * ldk + kk) = *reinterpret_cast<const uint4*>(&s_t[wc][16 * (piece ^ wperm)]);
     }
   }
 }

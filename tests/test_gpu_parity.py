@@ -527,6 +527,34 @@ def test_bias_every_kernel(L, M, N, K, how):
     y_close(Y, r["Y"])
 
 
+@pytest.mark.parametrize("M,N,K,n_out,ldy_pad", [
+    (129, 257, 520, 40, 0),      # one round of the chunk-outer epilogue (more than 16 outliers), ragged N
+    (300, 512, 1024, 96, 0),     # exactly one full round
+    (300, 512, 1024, 97, 8),     # two rounds (partial sums parked in TMEM), TMA stores with a padded ldy
+    (100, 600, 2048, 250, 3),    # three rounds, single-CTA tiles, direct stores (rows not 16-byte aligned)
+])
+def test_many_outliers_epilogue_rounds(L, M, N, K, n_out, ldy_pad):
+    """The GEMM epilogue with more than 16 outlier columns: the tile's
+    64-column chunks outermost, rounds of up to 96 outlier rows, the bias added
+    in the last round, for the fp16 weight and the int8-only weight."""
+    rng = np.random.default_rng(M + N + K + n_out)
+    X, W, _ = wl.random_small(rng, M, K, N, 0)
+    cols = np.sort(rng.choice(K, size=n_out, replace=False))
+    X[:, cols] = (rng.standard_normal((M, n_out), dtype=np.float32) * 20.0 + 10.0).astype(np.float16)
+    b = (rng.standard_normal(N) * 0.5).astype(np.float16)
+    Wd = dev(W)
+    Wq, cs = L.quantize_weight_colwise(Wd)
+    for keep in (True, False):
+        big = torch.zeros((M, N + ldy_pad), dtype=torch.float16, device="cuda")
+        Y = big[:, :N]
+        ws = L.empty_workspace(M, N, K, K)
+        L.mixed_matmul(dev(X), Wq, cs, Wd if keep else None, 6.0, Y=Y, ws=ws, bias=dev(b))
+        assert_status_ok(L, ws)
+        assert int(L.workspace_views(ws, M, N, K, K)["n_outlier"].item()) >= n_out
+        r = oracle.mixed_matmul(X, W, 6.0, bias=b, int8_weight=not keep)
+        y_close(host(Y), r["Y"])
+
+
 @pytest.mark.parametrize("keep", [False, True])
 @pytest.mark.parametrize("lead,K,N", [((2, 3), 520, 300), ((4, 50), 1032, 257), ((1,), 4096, 4096)])
 def test_int8_linear_module(L, keep, lead, K, N):
