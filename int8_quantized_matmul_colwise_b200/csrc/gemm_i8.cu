@@ -148,16 +148,38 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, ui
   }
 }
 
-// Tiles are ordered with the M index fastest, so that the tiles in flight at
-// one time share their Wq columns and all of Xq stays in L2.
-__device__ __forceinline__ void tile_coords(int tile, int num_m, int& mb, int& nb) {
-  mb = tile % num_m;
-  nb = tile / num_m;
-}
+// Tile order: the M tiles are split into groups of group_m consecutive tiles
+// (Xq strips of at most kGroupBytes together); a group's tiles run before the
+// next group's, M index fastest within it.  The tiles in flight at one time
+// then share a few Wq strips, and the group's Xq strips stay in L2 for all of
+// its N tiles, so that Xq is read from HBM once and Wq once per group.  With
+// M fastest over all of M every wave reads all of Xq, and once that is more
+// than L2 keeps, each wave re-reads it from HBM.
+constexpr int64_t kGroupBytes = int64_t(20) << 20;
 
 struct Sched {
-  int first, stride, num_tiles, num_m, num_k;
+  int first, stride, num_tiles, num_m, num_k, group_m;
 };
+
+// M tiles per group for tiles of tile_m rows and K bytes per row: groups of
+// equal size (the last one may be smaller) under the byte budget.
+__device__ __forceinline__ int tile_group_m(int num_m, int tile_m, int K) {
+  const int64_t by_bytes = kGroupBytes / (int64_t(tile_m) * int64_t(K > 0 ? K : 1));
+  const int cap = by_bytes < 1 ? 1 : (by_bytes > num_m ? num_m : static_cast<int>(by_bytes));
+  const int groups = (num_m + cap - 1) / cap;
+  return (num_m + groups - 1) / groups;
+}
+
+__device__ __forceinline__ void tile_coords(int tile, const Sched& sc, int& mb, int& nb) {
+  const int num_n = sc.num_tiles / sc.num_m;
+  const int per_group = sc.group_m * num_n;
+  const int g = tile / per_group;
+  const int r = tile - g * per_group;
+  const int m0 = g * sc.group_m;
+  const int rows = sc.num_m - m0 < sc.group_m ? sc.num_m - m0 : sc.group_m;
+  mb = m0 + r % rows;
+  nb = r / rows;
+}
 
 template <bool kPair>
 __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const Shared& s, const Sched& sc,
@@ -170,7 +192,7 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
   bool ok = true;
   for (int tile = sc.first; tile < sc.num_tiles && ok; tile += sc.stride) {
     int mb, nb;
-    tile_coords(tile, sc.num_m, mb, nb);
+    tile_coords(tile, sc, mb, nb);
     const int ya = mb * G::kTileM + (kPair ? static_cast<int>(rank) * BM : 0);
     const int yb = nb * BN + (kPair ? static_cast<int>(rank) * G::kRowsB : 0);
     for (int kb = 0; kb < sc.num_k; ++kb) {
@@ -472,7 +494,7 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
     const uint32_t b = it & 1u;
     const uint32_t use = (it >> 1) & 1u;
     int mb, nb;
-    tile_coords(tile, sc.num_m, mb, nb);
+    tile_coords(tile, sc, mb, nb);
     const int wrow0 = mb * G::kTileM + (kPair ? static_cast<int>(rank) * BM : 0) + static_cast<int>(q * 32);
     const int r0 = wrow0 + 16 * ab;  // this warp's 16 rows
     const uint32_t tacc = tmem_base + ((q * 32u + 16u * ab) << 16) + b * kAccCols;
@@ -724,6 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   sc.num_m = (p.M + G::kTileM - 1) / G::kTileM;
   sc.num_k = (p.K + BK - 1) / BK;
   sc.num_tiles = sc.num_m * ((p.N + BN - 1) / BN);
+  sc.group_m = tile_group_m(sc.num_m, G::kTileM, p.K);
   sc.first = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   sc.stride = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
