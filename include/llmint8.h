@@ -209,8 +209,10 @@ int llmint8_mixed_matmul_kernels(int64_t M, int64_t N, int64_t K, int64_t ldx, c
 /* The kernels llmint8_mixed_matmul launches for these arguments, by name, in
  * launch order and comma-separated: "decode_gemv_kernel" (M <= 8, whole Wq
  * rows per CTA), "decode_fused_kernel" (M <= 32, cluster split-K), or the
- * activation step ("act_fused_kernel", or "scan_columns_kernel" then
- * "quantize_rows_kernel" / "quantize_rows_long_kernel") followed by the GEMM
+ * activation step ("act_fused_kernel"; "scan_stream_kernel" then
+ * "quantize_stream_kernel" for many 16-byte aligned rows with 2048 <= K <=
+ * 16384; else "scan_columns_kernel" then "quantize_rows_kernel" /
+ * "quantize_rows_long_kernel") followed by the GEMM
  * ("gemm_i8_decode_kernel" for M <= 32, else "gemm_i8_kernel").  ldk is the
  * leading dimension of the Wq the call will get.  The string is static (do
  * not free it).  NULL for arguments the call rejects as invalid, or when no

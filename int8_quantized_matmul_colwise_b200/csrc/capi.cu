@@ -273,6 +273,9 @@ const char* llmint8_mixed_matmul_path(int64_t M, int64_t N, int64_t K, int64_t l
   const bool decode = M <= kDecodeMaxM;
   if (act_fused_plan(M, K, ldx, X, num_sms))
     return decode ? "act_fused_kernel,gemm_i8_decode_kernel" : "act_fused_kernel,gemm_i8_kernel";
+  if (act_stream_plan(M, K, ldx, X, num_sms))
+    return decode ? "scan_stream_kernel,quantize_stream_kernel,gemm_i8_decode_kernel"
+                  : "scan_stream_kernel,quantize_stream_kernel,gemm_i8_kernel";
   // the row kernel takes rows of up to 2048 chunks of 8 columns; longer rows the long-row kernel
   if ((K + 7) / 8 > 2048)
     return decode ? "scan_columns_kernel,quantize_rows_long_kernel,gemm_i8_decode_kernel"

@@ -12,7 +12,7 @@ namespace llmint8 {
 struct ActWs {
   uint32_t* colmax;       // [K] fp16 bit patterns of the column maxima; zero between calls
   uint32_t* blk_counter;  // [ceil(K/256)] scan CTAs finished per column block; zero between calls
-  uint32_t* bitmask;      // [ceil(K/32)] outlier flags of this call
+  uint32_t* bitmask;      // [ceil(K/32)] outlier flags of this call; zero between calls
   uint32_t* status;       // status word
   // One-kernel activation step (optional, nullptr: not used): a 64-bit grid
   // arrival counter followed by two outlier bitmasks of ceil(K/32) words each
@@ -41,9 +41,16 @@ cudaError_t launch_quantize_weight_colwise(const void* W, int64_t K, int64_t N, 
 // in shared memory spread over num_sms CTAs and its rows allow 16-byte loads).
 bool act_fused_plan(int64_t M, int64_t K, int64_t ldx, const void* X, int num_sms);
 
+// Whether the activation step for these arguments runs as the two streaming
+// kernels (many rows, 16-byte aligned, K % 8 == 0, kStreamMinK <= K <= kStreamMaxK).
+constexpr int64_t kStreamMinK = 2048;
+constexpr int64_t kStreamMaxK = 16384;
+bool act_stream_plan(int64_t M, int64_t K, int64_t ldx, const void* X, int num_sms);
+
 // num_sms > 0 and ws.fused set: shapes whose X fits in shared memory across
 // the SMs run as one persistent kernel (grid barrier between the column scan
-// and the row quantization); otherwise two kernels.
+// and the row quantization); otherwise two kernels (the streaming pair when
+// act_stream_plan holds).
 cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx, float tau, int8_t* Xq,
                                 int64_t ldq, float* rs, int32_t* O, int64_t cap, int32_t* n_out, void* Xo,
                                 int64_t ldo, ActWs ws, cudaStream_t stream, bool pdl, int num_sms = 0);

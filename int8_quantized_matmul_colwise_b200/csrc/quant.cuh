@@ -8,7 +8,8 @@
 
 namespace llmint8 {
 
-// q = round-half-away-from-zero(127 * x / s) for fp16 values |x| <= s, s > 0,
+// q = round-half-away-from-zero(127 * x / s) for fp16 values |x| <= s, s > 0
+// (s = 0, a vector whose values are all zero or NaN, and NaN x give 0),
 // computed without a division and exactly:
 //  * t = 127 |x| is exact in binary32 (11-bit times 7-bit significands);
 //  * r = t * (1/s) is within 2^-22 relative of t/s, so rint(r) is within one
@@ -19,7 +20,7 @@ namespace llmint8 {
 //    exactly.  __fmul_rn/__fadd_rn keep the compiler from fusing them.
 __device__ __forceinline__ int quantize_exact(float x, float s, float inv_s) {
   const float t = __fmul_rn(127.0f, fabsf(x));
-  if (!(t == t)) return 0;  // NaN input: code 0
+  if (!(t == t) || !(s > 0.0f)) return 0;  // NaN input, or a vector without a finite nonzero value: code 0
   float q = rintf(__fmul_rn(t, inv_s));
   if (__fmul_rn(__fadd_rn(q, 0.5f), s) <= t) {
     q = __fadd_rn(q, 1.0f);
@@ -129,6 +130,53 @@ __device__ __forceinline__ uint2 quantize8(uint4 u, float k, bool& tie_risk) {
     t[2 * e] = __float_as_uint(tb.x);
     t[2 * e + 1] = __float_as_uint(tb.y);
   }
+  uint2 out;
+  out.x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+  out.y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+  return out;
+}
+
+// max(a, b) that returns NaN when either is NaN (fmaxf drops a NaN operand).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// quantize8 with fused multiply-adds (fewer instructions, more registers:
+// for kernels with registers to spare).  With k = fl(127/s), the exact
+// product x k is within 127 * 2^-24 < 2^-17 of v = 127 x / s (|x| <= s).  One
+// fused multiply-add gives t = fl(x k + 1.5 * 2^23): for |x k| < 2^22 the sum
+// lies in [2^23, 2^24) where the spacing is 1, so t - 1.5 * 2^23 = q is x k
+// rounded to an integer (ties to even), exactly, and the low byte of t's bit
+// pattern is q's low byte (two's complement).  A second one, with -k, gives
+// d = fl(q - x k), within 2^-25 of q - x k.  When |d| < 1/2 - 2^-15,
+// |v - q| < 1/2 - 2^-15 + 2^-25 + 2^-17 < 1/2: q is the integer nearest to v
+// and v is no tie, so q is its round-half-away-from-zero value.  Otherwise
+// (about one value in 16000, or NaN: the maximum of |d| over the chunk
+// propagates NaN) tie_risk is set and the caller redoes the chunk with quantize8_exact.  The
+// arithmetic runs two values per instruction on the FMA pipe.
+__device__ __forceinline__ uint2 quantize8_fma(uint4 u, float k, bool& tie_risk) {
+  constexpr float kSafe = 0.499969482421875f;  // 1/2 - 2^-15
+  constexpr float kBias = 12582912.0f;         // 1.5 * 2^23
+  const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+  uint32_t t[8];
+  const float2 k2 = make_float2(k, k);
+  const float2 nk2 = make_float2(-k, -k);
+  const float2 b2 = make_float2(kBias, kBias);
+  const float2 nb2 = make_float2(-kBias, -kBias);
+  float dmax = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 x = __half22float2(h2[e]);
+    const float2 tb = __ffma2_rn(x, k2, b2);
+    const float2 q = __fadd2_rn(tb, nb2);
+    const float2 d = __ffma2_rn(x, nk2, q);
+    dmax = fmax_nan(dmax, fmax_nan(fabsf(d.x), fabsf(d.y)));
+    t[2 * e] = __float_as_uint(tb.x);
+    t[2 * e + 1] = __float_as_uint(tb.y);
+  }
+  tie_risk |= !(dmax < kSafe);  // true for NaN as well
   uint2 out;
   out.x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
   out.y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);

@@ -162,6 +162,21 @@ __device__ __forceinline__ void build_outlier_set(int64_t K, const ActWs& ws, ui
   __syncthreads();
 }
 
+// Every CTA has copied the call's bitmask into shared memory (the caller's
+// __syncthreads is behind it): the last one to get here returns the bitmask
+// and the counter to zero.
+__device__ __forceinline__ void release_bitmask(const ActWs& ws, int64_t nwords, int* s_last) {
+  if (threadIdx.x == 0) {
+    __threadfence();
+    *s_last = atomicAdd(ws.blk_counter, 1u) == gridDim.x - 1u ? 1 : 0;
+  }
+  __syncthreads();
+  if (*s_last) {
+    for (int64_t w = threadIdx.x; w < nwords; w += blockDim.x) ws.bitmask[w] = 0u;
+    if (threadIdx.x == 0) ws.blk_counter[0] = 0u;
+  }
+}
+
 // Column of the t-th outlier (t < n_o) from the bitmask and its word prefix.
 __device__ __forceinline__ int outlier_col(int t, const uint32_t* mask, const uint32_t* pre, int nwords) {
   int lo = 0, hi = nwords - 1;  // last word whose prefix is <= t
@@ -191,6 +206,7 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_kernel(const __half* __r
   constexpr int kRowsPerCta = 256 / G;
   __shared__ float s_part[8];
   __shared__ int s_warp[8];
+  __shared__ int s_last;
 
   griddep_wait();  // the column maxima come from the scan kernel
   griddep_launch_dependents();
@@ -211,6 +227,7 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_kernel(const __half* __r
   const int64_t nwords = (K + 31) / 32;
   uint32_t* s_pre = s_mask + nwords;
   build_outlier_set(K, ws, s_mask, s_pre, s_warp, O, cap, n_out);
+  release_bitmask(ws, nwords, &s_last);
 
   // outlier flags of chunk j's 8 columns (chunks past K: none, data is zero)
   auto flags = [&](int j) -> uint32_t {
@@ -277,7 +294,7 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_kernel(const __half* __r
       const int64_t c = 8 * (int64_t(gt) + int64_t(j) * G);
       if (c < ldq) {
         bool tie_risk = false;
-        *reinterpret_cast<uint2*>(qr + c) = quantize8(h[j], k, tie_risk);
+        *reinterpret_cast<uint2*>(qr + c) = quantize8_fma(h[j], k, tie_risk);
         risk |= static_cast<uint32_t>(tie_risk) << j;
       }
     }
@@ -295,24 +312,38 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_kernel(const __half* __r
 
 // ----------------------------------------------------------------- a1-a4 in one kernel
 // For shapes whose X fits in shared memory spread over the SMs: one CTA per SM
-// (all resident), each holding a block of rows.  The CTA bulk-copies its rows
-// into shared memory; thread t then holds R of those rows for one 8-column
-// chunk in registers for the whole kernel (chunks padded to a multiple of 32
-// so that a warp never straddles two row groups).  Phase 1 ORs the rows'
-// outlier flags (column maxima >= tau) into the call's global bitmask, one
-// atomic per non-zero 32-column word; after a grid barrier, phase 2 reads the
-// call's bitmask and its prefix, gathers the outlier values, zeroes them, takes
-// the row maxima (transposed warp reduction, one shared atomic max per row and
-// warp) and writes the codes.  X is read from HBM once.
+// (all resident: cooperative launch), each holding a block of rows.  The CTA
+// bulk-copies its rows into shared memory; thread t then holds R of those rows
+// for one 8-column chunk in registers for the whole kernel (chunks padded to a
+// multiple of 32 so that a warp never straddles two row groups).
 //
-// ws.fused: word 0 counts the CTAs that reached the grid barrier (the last one
-// returns it to zero), word 1 is the call generation g (the last CTA bumps
+// The outlier set is the union of every CTA's column flags, known only after a
+// grid barrier.  The barrier is split: a CTA ORs its own flags into the call's
+// global bitmask and arrives, then quantizes its rows against its own flags
+// while the other CTAs arrive (row maxima over the columns it has not flagged,
+// row scales, codes), and only then waits.  Its own flags are a subset of the
+// call's; when the two agree, which is the rule for outlier features that are
+// systematic across tokens, the codes already written are the answer.
+// Otherwise the CTA zeroes the further columns in its registers and quantizes
+// its rows again.  Last, the outlier values are gathered from the rows in
+// shared memory into Xo by their position in the call's outlier list.  X is
+// read from HBM once.
+//
+// ws.fused: word 0 counts the CTAs that arrived at the grid barrier (the last
+// one returns it to zero), word 1 is the call generation g (the last CTA bumps
 // it, which releases the others), words 4.. hold bitmask buffers 0 and 1 of
 // ceil(K/32) words.  A call of generation g ORs into buffer g & 1 and zeroes
 // buffer (g + 1) & 1, which the previous call used and the next will use.
 constexpr int kActFusedThreads = 1024;
 constexpr int kActFusedMaxRows = 16;  // rows per CTA
 constexpr size_t kActFusedSmemMax = 200 * 1024;
+
+// Dynamic shared memory of the kernel: the rows, three bitmask-sized word
+// arrays (16-byte multiples) and the column-maximum exchange.
+inline size_t act_fused_smem(int64_t rows_per, int64_t K) {
+  const size_t words = static_cast<size_t>((K + 31) / 32);
+  return size_t(rows_per) * size_t(K) * 2 + 3 * ((words * 4 + 15) / 16 * 16) + size_t(kActFusedThreads) * 16;
+}
 
 template <int R>
 __global__ void __launch_bounds__(kActFusedThreads, 1)
@@ -322,17 +353,19 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
                      int cpad) {
   extern __shared__ __align__(128) uint8_t smem_a[];
   const int nwords = static_cast<int>((K + 31) / 32);
+  const int nw4 = (nwords + 3) & ~3;
   const int nchunks = static_cast<int>(K / 8);  // K % 8 == 0 on this path
   __half* s_x = reinterpret_cast<__half*>(smem_a);  // [rows_per][K]
-  uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem_a + size_t(rows_per) * size_t(K) * 2);
-  uint32_t* s_pre = s_mask + ((nwords + 3) & ~3);
-  uint4* s_cm = reinterpret_cast<uint4*>(s_pre + ((nwords + 3) & ~3));  // [kActFusedThreads] column maxima
+  uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem_a + size_t(rows_per) * size_t(K) * 2);  // the call's flags
+  uint32_t* s_pre = s_mask + nw4;   // outliers before each word
+  uint32_t* s_own = s_pre + nw4;    // this CTA's flags
+  uint4* s_cm = reinterpret_cast<uint4*>(s_own + nw4);  // [kActFusedThreads] column maxima
   __shared__ uint64_t bar;
-  __shared__ int s_warp[kActFusedThreads / 32];
   __shared__ uint32_t s_gen;
-  __shared__ int s_ok;
-  __shared__ uint32_t s_rmax[kActFusedMaxRows];
+  __shared__ int s_released, s_more, s_nout;
+  __shared__ float s_part[kActFusedThreads / 32][8];  // row maxima per warp
   __shared__ float s_k[kActFusedMaxRows];
+  __shared__ float s_sc[kActFusedMaxRows];
   __shared__ float s_inv[kActFusedMaxRows];
 
   const int tid = static_cast<int>(threadIdx.x);
@@ -352,7 +385,6 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
     mbar_init(&bar, 1);
     fence_mbar_init();
   }
-  if (tid < kActFusedMaxRows) s_rmax[tid] = 0u;
   griddep_wait();  // X may be written by the preceding kernel
   griddep_launch_dependents();
   if (tid == 0) {
@@ -399,168 +431,182 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
       for (int e = 0; e < 4; ++e) cm[e] = __hmax2(cm[e], o2[e]);
     }
   }
-  uint32_t fl = 0;
+  uint32_t own = 0;  // bit e: column 8 cc + e is an outlier in this CTA's rows
   if (col_ok) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 f = __half22float2(cm[e]);
-      fl |= (f.x >= tau ? 1u : 0u) << (2 * e);
-      fl |= (f.y >= tau ? 1u : 0u) << (2 * e + 1);
+      own |= (f.x >= tau ? 1u : 0u) << (2 * e);
+      own |= (f.y >= tau ? 1u : 0u) << (2 * e + 1);
     }
   }
-  uint32_t word = fl << ((8 * cc) & 31);
+  uint32_t word = own << ((8 * cc) & 31);
   word |= __shfl_xor_sync(0xffffffffu, word, 1);
   word |= __shfl_xor_sync(0xffffffffu, word, 2);
-  if (g == 0 && col_ok && (cc & 3) == 0 && word != 0u) atomicOr(buf + (cc >> 2), word);
+  if (g == 0 && col_ok && (cc & 3) == 0) {
+    s_own[cc >> 2] = word;
+    if (word != 0u) {
+      atomicOr(buf + (cc >> 2), word);
+      __threadfence();
+    }
+  }
 
-  // grid barrier (every CTA of the grid is resident: at most one per SM); bounded
+  // grid barrier, arrival (every CTA of the grid is resident: cooperative launch)
   __syncthreads();
   if (tid == 0) {
-    int ok = 1;
     // (the stall test hook asks for one arrival more than the grid has: the
     // barrier then never completes and every CTA's wait runs out)
     const uint32_t last = gridDim.x - 1u + ((ws.stall & kStallActGridBarrier) ? 1u : 0u);
+    int released = 0;
     if (atom_add_acq_rel_gpu_u32(arrived, 1u) == last) {
       *arrived = 0u;                             // for the next call
       st_release_gpu_u32(generation, gen + 1u);  // releases the others
-    } else {
+      released = 1;
+    }
+    s_released = released;
+  }
+
+  // a2, a3 for the columns in `flags` (a superset of the ones zeroed so far):
+  // zero them, row maxima over the rest, row scales, codes
+  auto quantize_rows = [&](uint32_t flags, bool pad) {
+    if (flags != 0u) {
+      const uint32_t k0 = ((flags & 1u) ? 0u : 0xFFFFu) | ((flags & 2u) ? 0u : 0xFFFF0000u);
+      const uint32_t k1 = ((flags & 4u) ? 0u : 0xFFFFu) | ((flags & 8u) ? 0u : 0xFFFF0000u);
+      const uint32_t k2 = ((flags & 16u) ? 0u : 0xFFFFu) | ((flags & 32u) ? 0u : 0xFFFF0000u);
+      const uint32_t k3 = ((flags & 64u) ? 0u : 0xFFFFu) | ((flags & 128u) ? 0u : 0xFFFF0000u);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        h[r].x &= k0;
+        h[r].y &= k1;
+        h[r].z &= k2;
+        h[r].w &= k3;
+      }
+    }
+    float pm[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const __half2* h2 = reinterpret_cast<const __half2*>(&h[r]);
+      const __half2 m2 = __hmax2(__hmax2(__habs2(h2[0]), __habs2(h2[1])), __hmax2(__habs2(h2[2]), __habs2(h2[3])));
+      pm[r] = fmaxf(__low2float(m2), __high2float(m2));
+    }
+    int prow = 0;
+    const float pmax = rows_max_transposed<R>(pm, 32, lane, prow);
+    if ((lane & (32 / R - 1)) == 0) s_part[warp][prow] = pmax;
+    __syncthreads();
+    if (tid < nr) {  // row tid: group tid / R, its warps' partial maxima
+      const int wpg = cpad / 32;
+      const int wa = (tid / R) * wpg;
+      float sc = 0.0f;
+      for (int w = wa; w < wa + wpg; ++w) sc = fmaxf(sc, s_part[w][tid % R]);
+      rs[r0 + tid] = sc;
+      s_sc[tid] = sc;
+      s_k[tid] = sc > 0.0f ? __fdiv_rn(127.0f, sc) : 0.0f;
+      s_inv[tid] = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+    }
+    __syncthreads();
+    if (col_ok) {
+      int8_t* q = Xq + (r0 + m0) * ldq + 8 * cc;
+      uint32_t risk_rows = 0;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (m0 + r < nr) {
+          bool risk = false;
+          const uint2 code = quantize8(h[r], s_k[m0 + r], risk);
+          risk_rows |= static_cast<uint32_t>(risk) << r;
+          *reinterpret_cast<uint2*>(q) = code;
+        }
+        q += ldq;
+      }
+      if (risk_rows != 0u) {  // rare: a value within 2^-15 of a rounding boundary; redo its chunk exactly
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          if ((risk_rows >> r) & 1u)
+            *reinterpret_cast<uint2*>(Xq + (r0 + m0 + r) * ldq + 8 * cc) = quantize8_exact(h[r], s_sc[m0 + r], s_inv[m0 + r]);
+      }
+    }
+    if (pad) {  // Xq columns [K, ldq) are zero
+      const int npad = static_cast<int>((ldq - K) / 8);
+      for (int i = tid; i < npad * nr; i += kActFusedThreads)
+        *reinterpret_cast<uint2*>(Xq + (r0 + i / npad) * ldq + K + 8 * (i % npad)) = make_uint2(0u, 0u);
+    }
+  };
+  quantize_rows(own, true);
+
+  // grid barrier, wait; then warp 0 reads the call's bitmask, compares it with
+  // this CTA's flags and builds the popcount prefix (CTA 0 writes O and n_o)
+  if (warp == 0) {
+    if (lane == 0 && !s_released) {
       const uint64_t t0 = globaltimer_ns();
       uint32_t n = 0;
       while (ld_acquire_gpu_u32(generation) == gen) {
         if ((++n & 255u) == 0u && globaltimer_ns() - t0 > wait_limit_ns()) {
           atomicOr(ws.status, kStatusTimeout);
-          ok = 0;
           break;
         }
       }
     }
-    s_ok = ok && loaded;
-  }
-  __syncthreads();
-
-  // phase 2: the call's bitmask and its popcount prefix
-  int cnt = 0;
-  const int wpt = (nwords + kActFusedThreads - 1) / kActFusedThreads;
-  const int w0 = tid * wpt;
-  for (int w = w0; w < w0 + wpt && w < nwords; ++w) {
-    const uint32_t bw = __ldcg(buf + w);
-    s_mask[w] = bw;
-    cnt += __popc(bw);
-  }
-  int x = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) s_warp[warp] = x;
-  __syncthreads();
-  int before = 0, total = 0;
-#pragma unroll
-  for (int w = 0; w < kActFusedThreads / 32; ++w) {
-    before += w < warp ? s_warp[w] : 0;
-    total += s_warp[w];
-  }
-  int pos = before + x - cnt;
-  for (int w = w0; w < w0 + wpt && w < nwords; ++w) {
-    s_pre[w] = static_cast<uint32_t>(pos);
-    if (blockIdx.x == 0) {
-      uint32_t bits = s_mask[w];
-      int q = pos;
-      while (bits) {
-        const int bb = __ffs(bits) - 1;
-        bits &= bits - 1;
-        if (q < cap) O[q] = w * 32 + bb;
-        ++q;
-      }
+    __syncwarp();
+    const int wpl = (nwords + 31) / 32;  // contiguous words per lane
+    const int wa = lane * wpl;
+    const int wb = min(wa + wpl, nwords);
+    int cnt = 0;
+    bool more = false;
+    for (int w = wa; w < wb; ++w) {
+      const uint32_t b = __ldcg(buf + w);
+      s_mask[w] = b;
+      cnt += __popc(b);
+      more |= b != s_own[w];
     }
-    pos += __popc(s_mask[w]);
-  }
-  if (blockIdx.x == 0 && tid == 0) {
-    *n_out = total;
-    if (total > cap) atomicOr(ws.status, kStatusOverflow);
-  }
-  __syncthreads();
-
-  // a4: gather this thread's outlier values; then zero them (0 quantizes to 0)
-  const uint32_t gfl = col_ok ? (s_mask[cc >> 2] >> ((cc & 3) * 8)) & 0xFFu : 0u;
-  if (gfl != 0u) {
-    if (Xo != nullptr) {
-      const int b0 = (8 * cc) & 31;
-      const uint32_t wd = s_mask[cc >> 2];
-      const int base = static_cast<int>(s_pre[cc >> 2]);
-#pragma unroll 1
-      for (int e = 0; e < 8; ++e) {
-        if ((gfl >> e) & 1u) {
-          const int q = base + __popc(wd & ((1u << (b0 + e)) - 1u));
-          if (q < cap) {
+    int incl = cnt;
 #pragma unroll
-            for (int r = 0; r < R; ++r)
-              if (m0 + r < nr) Xo[(r0 + m0 + r) * ldo + q] = __ushort_as_half(half_bits_at(h[r], e));
-          }
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    int pos = incl - cnt;
+    for (int w = wa; w < wb; ++w) {
+      s_pre[w] = static_cast<uint32_t>(pos);
+      if (blockIdx.x == 0) {
+        uint32_t bits = s_mask[w];
+        int q = pos;
+        while (bits) {
+          const int bb = __ffs(bits) - 1;
+          bits &= bits - 1;
+          if (q < cap) O[q] = w * 32 + bb;
+          ++q;
         }
       }
+      pos += __popc(s_mask[w]);
     }
-    const uint32_t k0 = ((gfl & 1u) ? 0u : 0xFFFFu) | ((gfl & 2u) ? 0u : 0xFFFF0000u);
-    const uint32_t k1 = ((gfl & 4u) ? 0u : 0xFFFFu) | ((gfl & 8u) ? 0u : 0xFFFF0000u);
-    const uint32_t k2 = ((gfl & 16u) ? 0u : 0xFFFFu) | ((gfl & 32u) ? 0u : 0xFFFF0000u);
-    const uint32_t k3 = ((gfl & 64u) ? 0u : 0xFFFFu) | ((gfl & 128u) ? 0u : 0xFFFF0000u);
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      h[r].x &= k0;
-      h[r].y &= k1;
-      h[r].z &= k2;
-      h[r].w &= k3;
-    }
-  }
-
-  // a2: row maxima over the non-outlier columns
-  float pm[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const __half2* h2 = reinterpret_cast<const __half2*>(&h[r]);
-    const __half2 m2 = __hmax2(__hmax2(__habs2(h2[0]), __habs2(h2[1])), __hmax2(__habs2(h2[2]), __habs2(h2[3])));
-    pm[r] = fmaxf(__low2float(m2), __high2float(m2));
-  }
-  int prow = 0;
-  const float pmax = rows_max_transposed<R>(pm, 32, lane, prow);
-  if ((lane & (32 / R - 1)) == 0 && g < groups && m0 + prow < nr) atomicMax(&s_rmax[m0 + prow], __float_as_uint(pmax));
-  __syncthreads();
-  if (tid < nr) {
-    const float sc = __uint_as_float(s_rmax[tid]);
-    rs[r0 + tid] = sc;
-    s_k[tid] = sc > 0.0f ? __fdiv_rn(127.0f, sc) : 0.0f;
-    s_inv[tid] = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
-  }
-  __syncthreads();
-
-  // a3: codes
-  if (s_ok && col_ok) {
-    int8_t* q = Xq + (r0 + m0) * ldq + 8 * cc;
-    uint32_t risk_rows = 0;
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      if (m0 + r < nr) {
-        bool risk = false;
-        const uint2 code = quantize8(h[r], s_k[m0 + r], risk);
-        risk_rows |= static_cast<uint32_t>(risk) << r;
-        *reinterpret_cast<uint2*>(q) = code;
+    more = __any_sync(0xffffffffu, more);
+    if (lane == 0) {
+      s_more = more ? 1 : 0;
+      s_nout = total;
+      if (blockIdx.x == 0) {
+        *n_out = total;
+        if (total > cap) atomicOr(ws.status, kStatusOverflow);
       }
-      q += ldq;
-    }
-    if (risk_rows != 0u) {  // rare: a value within 2^-15 of a rounding boundary; redo its chunk exactly
-#pragma unroll
-      for (int r = 0; r < R; ++r)
-        if ((risk_rows >> r) & 1u)
-          *reinterpret_cast<uint2*>(Xq + (r0 + m0 + r) * ldq + 8 * cc) =
-              quantize8_exact(h[r], __uint_as_float(s_rmax[m0 + r]), s_inv[m0 + r]);
     }
   }
-  // Xq columns [K, ldq) are zero
-  if (s_ok) {
-    const int pad = static_cast<int>((ldq - K) / 8);
-    for (int i = tid; i < pad * nr; i += kActFusedThreads)
-      *reinterpret_cast<uint2*>(Xq + (r0 + i / pad) * ldq + K + 8 * (i % pad)) = make_uint2(0u, 0u);
+  __syncthreads();
+
+  // other CTAs flagged columns this one did not: quantize the rows again
+  if (s_more) {
+    const uint32_t all = col_ok ? (s_mask[cc >> 2] >> ((cc & 3) * 8)) & 0xFFu : 0u;
+    quantize_rows(all, false);
+  }
+
+  // a4: X[row, O[q]] for this CTA's rows, from the rows in shared memory
+  if (Xo != nullptr && loaded) {
+    const int nq = static_cast<int>(min(int64_t(s_nout), cap));
+    const int items = nq * nr;
+    for (int i = tid; i < items; i += kActFusedThreads) {
+      const int r = i / nq;
+      const int q = i - r * nq;
+      const int col = outlier_col(q, s_mask, s_pre, nwords);
+      Xo[(r0 + r) * ldo + q] = s_x[size_t(r) * size_t(K) + col];
+    }
   }
 }
 
@@ -660,11 +706,13 @@ __global__ void __launch_bounds__(256) quantize_rows_long_kernel(const __half* _
   extern __shared__ uint32_t s_mask[];
   __shared__ float s_part[8];
   __shared__ int s_warp[8];
+  __shared__ int s_last;
   griddep_wait();
   griddep_launch_dependents();
   const int64_t nwords = (K + 31) / 32;
   uint32_t* s_pre = s_mask + nwords;
   build_outlier_set(K, ws, s_mask, s_pre, s_warp, O, cap, n_out);
+  release_bitmask(ws, nwords, &s_last);
 
   const int64_t row = blockIdx.x;
   const __half* xr = X + row * ldx;
@@ -719,6 +767,325 @@ __global__ void __launch_bounds__(256) quantize_rows_long_kernel(const __half* _
   }
 }
 
+// ----------------------------------------------------------------- a1-a4 streaming (many rows)
+// X with more rows than fit in shared memory over the SMs, rows that allow
+// bulk copies (16-byte aligned, K % 8 == 0) and kStreamMinK <= K <=
+// kStreamMaxK.  Both kernels are persistent (two CTAs per SM), and each CTA
+// streams whole rows of X through a ring of shared-memory stages filled by
+// bulk copies, so that several rows per SM are in flight at any time.
+//  scan:     column maxima of |X| over the CTA's rows, kept in registers; then
+//            one flag per column (maximum >= tau, which a NaN never wins) ORed
+//            into the call's bitmask, which is zero between calls;
+//  quantize: the CTA copies the bitmask and its popcount prefix into shared
+//            memory once (the last CTA to do so returns the bitmask to zero),
+//            then quantizes its rows, walking them from the last row up so
+//            that the rows the scan read last, still in L2, come first.
+constexpr int kStreamThreads = 256;
+constexpr int kStreamMaxStages = 8;
+constexpr size_t kStreamRing = 96 * 1024;  // bytes of row stages per CTA
+constexpr int kStreamListMax = 1024;        // outlier columns listed in shared memory
+
+inline int stream_stages(int64_t K) {
+  const int s = static_cast<int>(kStreamRing / (size_t(K) * 2));
+  return s > kStreamMaxStages ? kStreamMaxStages : s;
+}
+
+// Rows of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
+__device__ __forceinline__ int64_t stream_rows(int64_t M) {
+  return M > int64_t(blockIdx.x) ? (M - 1 - int64_t(blockIdx.x)) / int64_t(gridDim.x) + 1 : 0;
+}
+
+// After a wait gave up at row `from` (stage st, phase parity ph): let the
+// copies issued for rows [from, to) of this CTA land before the CTA exits.
+__device__ __forceinline__ void stream_drain(uint64_t* full, int stages, int64_t from, int64_t to, int st,
+                                             uint32_t ph) {
+  for (int64_t i = from; i < to; ++i) {
+    mbar_wait(&full[st], ph, nullptr);
+    if (++st == stages) {
+      st = 0;
+      ph ^= 1u;
+    }
+  }
+}
+
+template <int CPT>
+__global__ void __launch_bounds__(kStreamThreads, 2)
+    scan_stream_kernel(const __half* __restrict__ X, int64_t M, int64_t K, int64_t ldx, float tau, ActWs ws,
+                       int stages) {
+  extern __shared__ __align__(128) uint8_t smem_s[];
+  __shared__ uint64_t full[kStreamMaxStages];
+  __half* ring = reinterpret_cast<__half*>(smem_s);
+  const int tid = static_cast<int>(threadIdx.x);
+  const int warp = tid >> 5;
+  const int nchunks = static_cast<int>(K / 8);
+  const int64_t nrows = stream_rows(M);
+  const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();  // X may be written by the preceding kernel
+  griddep_launch_dependents();
+  // thread 0 issues row `issued` of this CTA into stage `ist` (rows and stages advance together)
+  int64_t issued = 0;
+  int ist = 0;
+  auto issue = [&]() {
+    mbar_arrive_expect_tx(&full[ist], row_bytes);
+    bulk_load_1d(ring + size_t(ist) * size_t(K), X + (int64_t(blockIdx.x) + issued * gridDim.x) * ldx, row_bytes,
+                 &full[ist]);
+    ++issued;
+    if (++ist == stages) ist = 0;
+  };
+  if (tid == 0)
+    while (issued < stages && issued < nrows) issue();
+
+  __half2 cm[CPT][4];
+#pragma unroll
+  for (int j = 0; j < CPT; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) cm[j][e] = __half2half2(__ushort_as_half(0));
+  // Warp 0 alone waits for each row's copy, the other warps at the row's
+  // barrier (which issues nothing), so that no spinning takes issue slots
+  // from the other CTA on the SM.
+  int st = 0;        // stage of row i
+  uint32_t ph = 0;   // its phase parity
+  if (!__syncthreads_and(warp != 0 || nrows == 0 || mbar_wait(&full[0], 0, ws.status))) {
+    if (tid == 0) stream_drain(full, stages, 0, issued, 0, 0u);  // a copy never landed: timeout bit set
+    return;
+  }
+  for (int64_t i = 0; i < nrows; ++i) {
+    const __half* sr = ring + size_t(st) * size_t(K);
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int c = tid + j * kStreamThreads;
+      if (c < nchunks) {
+        const uint4 u = *reinterpret_cast<const uint4*>(sr + 8 * c);
+        const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cm[j][e] = __hmax2(cm[j][e], __habs2(h2[e]));  // NaN never wins
+      }
+    }
+    const int nst = st + 1 == stages ? 0 : st + 1;  // row i + 1
+    const uint32_t nph = nst == 0 ? ph ^ 1u : ph;
+    if (!__syncthreads_and(warp != 0 || i + 1 >= nrows || mbar_wait(&full[nst], nph, ws.status))) {
+      if (tid == 0) stream_drain(full, stages, i + 1, issued, nst, nph);
+      return;
+    }
+    if (tid == 0 && issued < nrows) issue();  // every thread is done with row i's stage
+    st = nst;
+    ph = nph;
+  }
+
+  // a1: one flag per column, ORed into the call's bitmask (32 columns per word)
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) {
+    const int c = tid + j * kStreamThreads;
+    uint32_t f = 0;
+    if (c < nchunks) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 m = __half22float2(cm[j][e]);
+        f |= (m.x >= tau ? 1u : 0u) << (2 * e);
+        f |= (m.y >= tau ? 1u : 0u) << (2 * e + 1);
+      }
+    }
+    uint32_t word = f << ((8 * c) & 31);
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    word |= __shfl_xor_sync(0xffffffffu, word, 2);
+    if ((c & 3) == 0 && c < nchunks && word != 0u) atomicOr(ws.bitmask + (c >> 2), word);
+  }
+}
+
+template <int CPT>
+__global__ void __launch_bounds__(kStreamThreads, 2)
+    quantize_stream_kernel(const __half* __restrict__ X, int64_t M, int64_t K, int64_t ldx, ActWs ws,
+                           int32_t* __restrict__ O, int32_t* __restrict__ n_out, int64_t cap, int8_t* __restrict__ Xq,
+                           int64_t ldq, float* __restrict__ rs, __half* __restrict__ Xo, int64_t ldo, int stages) {
+  extern __shared__ __align__(128) uint8_t smem_s[];
+  __shared__ uint64_t full[kStreamMaxStages];
+  __shared__ float s_part[2][kStreamThreads / 32];
+  __shared__ int s_warp[kStreamThreads / 32];
+  __shared__ int s_last;
+  const int nwords = static_cast<int>((K + 31) / 32);
+  const int nw4 = (nwords + 3) & ~3;
+  __half* ring = reinterpret_cast<__half*>(smem_s);
+  uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem_s + size_t(stages) * size_t(K) * 2);
+  uint32_t* s_pre = s_mask + nw4;
+  int* s_list = reinterpret_cast<int*>(s_pre + nw4);  // [kStreamListMax] the first outlier columns
+  const int tid = static_cast<int>(threadIdx.x);
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int nchunks = static_cast<int>(K / 8);
+  const int64_t nrows = stream_rows(M);
+  const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
+  auto row_of = [&](int64_t i) { return M - 1 - (int64_t(blockIdx.x) + i * gridDim.x); };  // last row first
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();  // the bitmask comes from the scan kernel
+  griddep_launch_dependents();
+  // thread 0 issues row `issued` of this CTA into stage `ist` (rows and stages advance together)
+  int64_t issued = 0;
+  int ist = 0;
+  auto issue = [&]() {
+    mbar_arrive_expect_tx(&full[ist], row_bytes);
+    bulk_load_1d(ring + size_t(ist) * size_t(K), X + row_of(issued) * ldx, row_bytes, &full[ist]);
+    ++issued;
+    if (++ist == stages) ist = 0;
+  };
+  if (tid == 0)
+    while (issued < stages && issued < nrows) issue();
+
+  // the call's outlier set, once per CTA (CTA 0 writes O and n_o)
+  build_outlier_set(K, ws, s_mask, s_pre, s_warp, O, cap, n_out);
+  for (int w = tid; w < nwords; w += kStreamThreads) {
+    uint32_t bits = s_mask[w];
+    int pos = static_cast<int>(s_pre[w]);
+    while (bits && pos < kStreamListMax) {
+      s_list[pos++] = w * 32 + __ffs(bits) - 1;
+      bits &= bits - 1;
+    }
+  }
+  release_bitmask(ws, nwords, &s_last);  // its barrier also publishes s_list
+  const int n_o = static_cast<int>(s_pre[nwords - 1]) + __popc(s_mask[nwords - 1]);
+  const int nq = static_cast<int>(min(int64_t(n_o), cap));
+
+  // Warp 0 alone waits for each row's copy (for row i + 1 just before row i's
+  // barrier), the other warps at the barrier, which issues nothing.
+  int st = 0;        // stage of row i
+  uint32_t ph = 0;   // its phase parity
+  if (!__syncthreads_and(warp != 0 || nrows == 0 || mbar_wait(&full[0], 0, ws.status))) {
+    if (tid == 0) stream_drain(full, stages, 0, issued, 0, 0u);  // a copy never landed: timeout bit set
+    return;
+  }
+  for (int64_t i = 0; i < nrows; ++i) {
+    const int64_t row = row_of(i);
+    const __half* sr = ring + size_t(st) * size_t(K);
+    uint4 h[CPT];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int c = tid + j * kStreamThreads;
+      h[j] = c < nchunks ? *reinterpret_cast<const uint4*>(sr + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // a3 precondition: outlier columns are zeroed (0 quantizes to 0); a2: row maximum of the rest
+    __half2 m2 = __half2half2(__ushort_as_half(0));
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int c = tid + j * kStreamThreads;
+      const uint32_t om = c < nchunks ? (s_mask[c >> 2] >> ((c & 3) * 8)) & 0xFFu : 0u;
+      if (om != 0u) {
+        uint32_t* w = reinterpret_cast<uint32_t*>(&h[j]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          w[e] &= (((om >> (2 * e)) & 1u) ? 0u : 0xFFFFu) | (((om >> (2 * e + 1)) & 1u) ? 0u : 0xFFFF0000u);
+      }
+      const __half2* h2 = reinterpret_cast<const __half2*>(&h[j]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(h2[e]));
+    }
+    float m = fmaxf(__low2float(m2), __high2float(m2));
+    m = (m == m) ? m : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) s_part[i & 1][warp] = m;
+    const int nst = st + 1 == stages ? 0 : st + 1;  // row i + 1
+    const uint32_t nph = nst == 0 ? ph ^ 1u : ph;
+    if (!__syncthreads_and(warp != 0 || i + 1 >= nrows || mbar_wait(&full[nst], nph, ws.status))) {
+      if (tid == 0) stream_drain(full, stages, i + 1, issued, nst, nph);  // timeout bit set
+      return;
+    }
+    // every thread is done with row i - 1 (its gather included): refill its stage
+    if (tid == 0 && i >= 1 && issued < nrows) issue();
+    float s = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kStreamThreads / 32; ++w) s = fmaxf(s, s_part[i & 1][w]);
+    const float k = s > 0.0f ? __fdiv_rn(127.0f, s) : 0.0f;
+    int8_t* qr = Xq + row * ldq;
+    uint32_t risk = 0;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int c = tid + j * kStreamThreads;
+      if (c < nchunks) {
+        bool r = false;
+        *reinterpret_cast<uint2*>(qr + 8 * c) = quantize8_fma(h[j], k, r);
+        risk |= static_cast<uint32_t>(r) << j;
+      }
+    }
+    if (risk != 0u) {  // rare: a value within 2^-15 of a rounding boundary; redo its chunk exactly
+      const float inv = __frcp_rn(s);
+#pragma unroll
+      for (int j = 0; j < CPT; ++j)
+        if ((risk >> j) & 1u) *reinterpret_cast<uint2*>(qr + 8 * (tid + j * kStreamThreads)) = quantize8_exact(h[j], s, inv);
+    }
+    for (int64_t c = nchunks + tid; c < ldq / 8; c += kStreamThreads)  // Xq columns [K, ldq) are zero
+      *reinterpret_cast<uint2*>(qr + 8 * c) = make_uint2(0u, 0u);
+    if (tid == 0) rs[row] = s;
+    // a4: X[row, O[t]] from the row in shared memory
+    if (Xo != nullptr) {
+      for (int t = tid; t < nq; t += kStreamThreads) {
+        const int col = t < kStreamListMax ? s_list[t] : outlier_col(t, s_mask, s_pre, nwords);
+        Xo[row * ldo + t] = sr[col];
+      }
+    }
+    st = nst;
+    ph = nph;
+  }
+}
+
+template <int CPT>
+cudaError_t launch_stream(cudaLaunchConfig_t cfg, int64_t M, const __half* x, int64_t K, int64_t ldx, float tau,
+                          ActWs ws, int32_t* O, int32_t* n, int64_t cap, int8_t* Xq, int64_t ldq, float* rs,
+                          __half* xo, int64_t ldo, int num_sms) {
+  static bool attr_set[64] = {};
+  static int per_sm[64][2] = {};  // resident CTAs per SM at the largest ring (scan, quantize), per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const int stages = stream_stages(K);
+  const size_t nw4 = static_cast<size_t>(((K + 31) / 32 + 3) & ~int64_t(3));
+  const size_t smem_scan = size_t(stages) * size_t(K) * 2;
+  const size_t smem_q = smem_scan + 2 * nw4 * 4 + size_t(kStreamListMax) * 4;
+  if (!attr_set[dev]) {
+    // two CTAs of ~100 KB per SM need the largest shared-memory carveout
+    e = cudaFuncSetAttribute(scan_stream_kernel<CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kStreamRing));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(scan_stream_kernel<CPT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(quantize_stream_kernel<CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kStreamRing + 2 * 4 * 512 + 4 * kStreamListMax));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(quantize_stream_kernel<CPT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    // persistent grids: as many CTAs as are resident at once (one wave)
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[dev][0], scan_stream_kernel<CPT>, kStreamThreads,
+                                                        kStreamRing);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[dev][1], quantize_stream_kernel<CPT>, kStreamThreads,
+                                                        kStreamRing + 2 * 4 * 512 + 4 * kStreamListMax);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  auto clamp12 = [](int v) { return v < 1 ? 1 : v > 2 ? 2 : v; };
+  const int64_t ctas_scan = int64_t(num_sms) * clamp12(per_sm[dev][0]);
+  const int64_t ctas_q = int64_t(num_sms) * clamp12(per_sm[dev][1]);
+  cfg.blockDim = dim3(kStreamThreads);
+  cfg.gridDim = dim3(static_cast<unsigned>(M < ctas_scan ? M : ctas_scan));
+  cfg.dynamicSmemBytes = smem_scan;
+  e = cudaLaunchKernelEx(&cfg, scan_stream_kernel<CPT>, x, M, K, ldx, tau, ws, stages);
+  if (e != cudaSuccess) return e;
+  cfg.gridDim = dim3(static_cast<unsigned>(M < ctas_q ? M : ctas_q));
+  cfg.dynamicSmemBytes = smem_q;
+  return cudaLaunchKernelEx(&cfg, quantize_stream_kernel<CPT>, x, M, K, ldx, ws, O, n, cap, Xq, ldq, rs, xo, ldo,
+                            stages);
+}
+
 template <int G, int CPT>
 cudaError_t launch_rows(cudaLaunchConfig_t& cfg, int64_t M, const __half* x, int64_t K, int64_t ldx, bool vec_ok,
                         float tau, ActWs ws, int32_t* O, int32_t* n, int64_t cap, int8_t* Xq, int64_t ldq,
@@ -734,6 +1101,11 @@ cudaError_t launch_rows(cudaLaunchConfig_t& cfg, int64_t M, const __half* x, int
 
 }  // namespace
 
+bool act_stream_plan(int64_t M, int64_t K, int64_t ldx, const void* X, int num_sms) {
+  return num_sms > 0 && ldx % 8 == 0 && K % 8 == 0 && reinterpret_cast<uintptr_t>(X) % 16 == 0 &&
+         K >= kStreamMinK && K <= kStreamMaxK && M >= num_sms;
+}
+
 bool act_fused_plan(int64_t M, int64_t K, int64_t ldx, const void* X, int num_sms) {
   if (num_sms <= 0 || ldx % 8 != 0 || K % 8 != 0 || reinterpret_cast<uintptr_t>(X) % 16 != 0) return false;
   const int64_t rows_per = (M + num_sms - 1) / num_sms;
@@ -741,9 +1113,7 @@ bool act_fused_plan(int64_t M, int64_t K, int64_t ldx, const void* X, int num_sm
   if (cpad > kActFusedThreads) return false;
   const int64_t groups = kActFusedThreads / cpad;
   const int64_t r = (rows_per + groups - 1) / groups;
-  const size_t mask_bytes = static_cast<size_t>((K + 31) / 32) * sizeof(uint32_t);
-  const size_t smem = size_t(rows_per) * size_t(K) * 2 + 2 * ((mask_bytes + 15) / 16 * 16) +
-                      size_t(kActFusedThreads) * 16;
+  const size_t smem = act_fused_smem(rows_per, K);
   return r <= 8 && rows_per <= kActFusedMaxRows && smem <= kActFusedSmemMax;
 }
 
@@ -769,8 +1139,7 @@ cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx
     const int64_t rows_per = (M + num_sms - 1) / num_sms;
     const int64_t cpad = ((K / 8) + 31) / 32 * 32;  // chunks padded to whole warps
     const int64_t r = (rows_per + kActFusedThreads / cpad - 1) / (kActFusedThreads / cpad);  // rows per thread
-    const size_t smem = size_t(rows_per) * size_t(K) * 2 + 2 * ((mask_bytes + 15) / 16 * 16) +
-                        size_t(kActFusedThreads) * 16;
+    const size_t smem = act_fused_smem(rows_per, K);
     const int ri = r <= 1 ? 0 : r <= 2 ? 1 : r <= 4 ? 2 : 3;
     auto kern = ri == 0 ? act_fused_kernel<1> : ri == 1 ? act_fused_kernel<2> : ri == 2 ? act_fused_kernel<4>
                                                                                         : act_fused_kernel<8>;
@@ -799,6 +1168,20 @@ cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx
                               ldo, static_cast<int>(rows_per), static_cast<int>(cpad));
   }
 
+  __half* xo = static_cast<__half*>(Xo);
+  // Many rows that allow bulk copies: the two streaming kernels.
+  if (act_stream_plan(M, K, ldx, X, num_sms)) {
+    const int64_t chunks = K / 8;
+#define LLMINT8_STREAM(CPT) \
+  return launch_stream<CPT>(cfg, M, x, K, ldx, tau, ws, O, n_out, cap, Xq, ldq, rs, xo, ldo, num_sms)
+    if (chunks <= kStreamThreads) LLMINT8_STREAM(1);
+    if (chunks <= 2 * kStreamThreads) LLMINT8_STREAM(2);
+    if (chunks <= 4 * kStreamThreads) LLMINT8_STREAM(4);
+    if (chunks <= 6 * kStreamThreads) LLMINT8_STREAM(6);
+    LLMINT8_STREAM(8);
+#undef LLMINT8_STREAM
+  }
+
   cfg.gridDim = dim3(static_cast<unsigned>((K + kScanCols - 1) / kScanCols),
                      static_cast<unsigned>((M + kScanRows - 1) / kScanRows));
   cfg.dynamicSmemBytes = 0;
@@ -807,7 +1190,6 @@ cudaError_t launch_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx
   if (e != cudaSuccess) return e;
 
   cfg.dynamicSmemBytes = 2 * mask_bytes;  // bitmask + popcount prefix
-  __half* xo = static_cast<__half*>(Xo);
   // Row groups: G threads x CPT chunks of 8 columns >= K.  Small M spreads a
   // row over more threads (fewer chunks each) to shorten the critical path.
   const int64_t chunks = (K + 7) / 8;

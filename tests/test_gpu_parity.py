@@ -170,6 +170,116 @@ def test_activation_workspace_reuse_across_shapes(L):
     assert_status_ok(L, ws)
 
 
+@pytest.mark.parametrize("M,K", [(2048, 4096), (300, 512), (1000, 8192)])
+def test_activation_outlier_flagged_by_one_row(L, M, K):
+    """Column c holds 5.9 (< tau) in every row but one, which holds 7.0: it is
+    an outlier column of the call although only one block of rows sees a
+    value >= tau in it, and it carries every other row's largest non-outlier
+    value until it is excluded.  The one-kernel step quantizes each block of
+    rows against the columns that block flagged and must redo the blocks that
+    missed column c; the row scales and codes must equal the oracle's."""
+    rng = np.random.default_rng(M + K)
+    X = rng.standard_normal((M, K)).astype(np.float16)
+    c, c2 = 37, K - 3
+    X[:, c] = np.float16(5.9)
+    X[M // 2, c] = np.float16(7.0)
+    X[:, c2] = np.float16(-5.5)
+    X[M - 1, c2] = np.float16(-20.0)
+    Xd = dev(X)
+    if M == 2048:
+        assert L.llmint8_mixed_matmul_path(Xd, torch.empty((1, K), dtype=torch.int8, device="cuda"),
+                                           K)[0] == "act_fused_kernel"
+    out = check_act(L, X, 6.0)
+    assert_status_ok(L, out["ws"])
+    assert host(out["outlier_idx"])[:int(host(out["n_outlier"])[0])].tolist() == [c, c2]
+
+
+# (M, K, tau, planted columns): shapes that take the two streaming kernels,
+# one per registers-per-thread variant; K = 4104 pads each Xq row by 8 bytes;
+# tau = 0.5 flags most columns (more than the 1024 listed in shared memory)
+STREAM_CASES = [(3000, 2048, 6.0, 5), (4096, 4096, 6.0, 6), (4096, 4104, 6.0, 9), (2000, 8192, 6.0, 3),
+                (600, 12288, 6.0, 25), (200, 16384, 6.0, 7), (3000, 4096, 0.5, 0), (1700, 8192, np.inf, 4)]
+
+
+@pytest.mark.parametrize("M,K,tau,n_planted", STREAM_CASES)
+def test_activation_streaming_kernels(L, M, K, tau, n_planted):
+    rng = np.random.default_rng(M * 7 + K)
+    X, _, _ = wl.random_small(rng, M, K, 1, n_planted)
+    X[M // 3, K // 5] = np.float16(-9.0)  # an outlier column seen by one row only
+    Xd = dev(X)
+    assert L.llmint8_mixed_matmul_path(Xd, torch.empty((1, L.round_up(K, 16)), dtype=torch.int8, device="cuda"),
+                                       K)[:2] == ["scan_stream_kernel", "quantize_stream_kernel"]
+    out = check_act(L, X, tau)
+    assert_status_ok(L, out["ws"])
+
+
+@pytest.mark.parametrize("M,K,strided,first", [(2048, 4096, False, "act_fused_kernel"),
+                                                (4096, 4096, False, "scan_stream_kernel"),
+                                                (300, 4096, True, "scan_columns_kernel"),
+                                                (5, 20000, False, "scan_columns_kernel")])
+def test_activation_nan_and_inf(L, M, K, strided, first):
+    """NaN is never an outlier and codes to 0 (a row of NaN has scale 0);
+    +-Inf makes its column an outlier and is gathered as it is: each
+    activation kernel against the oracle, Xo compared bit for bit."""
+    rng = np.random.default_rng(M + K)
+    X = rng.standard_normal((M, K)).astype(np.float16)
+    X[1, 3] = np.nan
+    X[M - 1, K // 2] = np.nan
+    X[2, :] = np.nan
+    X[M // 2, 7] = np.inf
+    X[0, K - 1] = -np.inf
+    if strided:
+        wide = np.zeros((M, K + 1), np.float16)
+        wide[:, :K] = X
+        Xd = dev(wide)[:, :K]
+    else:
+        Xd = dev(X)
+    assert L.llmint8_mixed_matmul_path(Xd, torch.empty((1, L.round_up(K, 16)), dtype=torch.int8, device="cuda"),
+                                       K)[0] == first
+    out = L.quantize_act_rowwise_outliers(Xd, 6.0)
+    O, rs, Xq = oracle.quantize_activation(X, 6.0)
+    n = int(host(out["n_outlier"])[0])
+    assert n == O.size and {7, K - 1} <= set(O.tolist())
+    assert np.array_equal(host(out["outlier_idx"])[:n], O)
+    assert np.array_equal(host(out["row_scale"]), rs) and rs[2] == 0
+    assert np.array_equal(host(out["Xq"])[:, :K], Xq)
+    Xo_ref, _ = oracle.gather_outliers(X, O)
+    assert np.array_equal(host(out["Xo"])[:, :n].view(np.uint16), Xo_ref.view(np.uint16))
+    assert_status_ok(L, out["ws"])
+
+
+def test_activation_workspace_reuse_across_paths(L):
+    """One workspace through the streaming pair, the one-kernel step and the
+    per-row kernels in turn: the call's bitmask must be back to zero after
+    every call whichever kernels wrote it."""
+    K = 4096
+    ws = L.empty_workspace(4096, 1, K, K)
+    rng = np.random.default_rng(77)
+    seq = [(4096, 6.0, "scan_stream_kernel", False), (40, 6.0, "scan_columns_kernel", True),
+           (4096, 0.5, "scan_stream_kernel", False), (129, 6.0, "act_fused_kernel", False),
+           (4096, np.inf, "scan_stream_kernel", False), (300, 6.0, "scan_columns_kernel", True),
+           (4096, 6.0, "scan_stream_kernel", False)]
+    for M, tau, first, strided in seq:
+        X, _, _ = wl.random_small(rng, M, K, 1, 4)
+        if strided:
+            wide = np.zeros((M, K + 1), np.float16)
+            wide[:, :K] = X
+            Xd = dev(wide)[:, :K]
+        else:
+            Xd = dev(X)
+        assert L.llmint8_mixed_matmul_path(Xd, torch.empty((1, K), dtype=torch.int8, device="cuda"), K)[0] == first
+        out = L.quantize_act_rowwise_outliers(Xd, tau, ws=ws)
+        O, rs, Xq = oracle.quantize_activation(X, tau)
+        n = int(host(out["n_outlier"])[0])
+        assert n == O.size
+        assert np.array_equal(host(out["outlier_idx"])[:n], O)
+        assert np.array_equal(host(out["row_scale"]), rs)
+        assert np.array_equal(host(out["Xq"])[:, :K], Xq)
+        Xo_ref, _ = oracle.gather_outliers(X, O)
+        assert np.array_equal(host(out["Xo"])[:, :n].view(np.uint16), Xo_ref.view(np.uint16))
+    assert_status_ok(L, ws)
+
+
 def test_activation_strided_rows(L):
     X = wl.make_x(wl.get("tiny"))
     wide = np.zeros((X.shape[0], X.shape[1] + 40), np.float16)
@@ -632,7 +742,9 @@ def test_kernel_path_query(L):
     assert path(8, 16384, 1024) == ["decode_fused_kernel"]         # more Wq rows per SM than the kernel holds
     assert path(32, 4096, 4096) == ["decode_fused_kernel"]         # more rows of X
     assert path(2048, 16384, 4096) == ["act_fused_kernel", "gemm_i8_kernel"]
-    assert path(8192, 8192, 8192) == ["scan_columns_kernel", "quantize_rows_kernel", "gemm_i8_kernel"]
+    assert path(8192, 8192, 8192) == ["scan_stream_kernel", "quantize_stream_kernel", "gemm_i8_kernel"]
+    assert path(8192, 8192, 8192, ldx=8193) == ["scan_columns_kernel", "quantize_rows_kernel", "gemm_i8_kernel"]
+    assert path(4096, 1024, 1024) == ["scan_columns_kernel", "quantize_rows_kernel", "gemm_i8_kernel"]  # K < 2048
     assert path(100, 300, 1000, ldx=1001) == ["scan_columns_kernel", "quantize_rows_kernel", "gemm_i8_kernel"]
     assert path(5, 130, 20000) == ["scan_columns_kernel", "quantize_rows_long_kernel", "gemm_i8_decode_kernel"]
 

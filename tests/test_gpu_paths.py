@@ -170,6 +170,14 @@ def check_act_codes(L, X, Xd, expect_kernel):
 
 
 @pytest.mark.parametrize("s", SCALES)
+def test_quantizer_stream_kernel(L, s):
+    """quantize_stream_kernel: 4096 rows of 4096 columns (zero rows pad the
+    sweep), more than the one-kernel step holds."""
+    for X in sweep_rows(s, 4096, rows_per_call=4096):
+        check_act_codes(L, X, dev(X), "quantize_stream_kernel")
+
+
+@pytest.mark.parametrize("s", SCALES)
 def test_quantizer_row_kernel_unaligned_rows(L, s):
     """quantize_rows_kernel: X rows not 16-byte aligned (ldx = K + 1)."""
     for X in sweep_rows(s, 4096):
