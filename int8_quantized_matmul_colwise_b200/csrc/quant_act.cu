@@ -329,11 +329,14 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_kernel(const __half* __r
 // shared memory into Xo by their position in the call's outlier list.  X is
 // read from HBM once.
 //
-// ws.fused: word 0 counts the CTAs that arrived at the grid barrier (the last
-// one returns it to zero), word 1 is the call generation g (the last CTA bumps
-// it, which releases the others), words 4.. hold bitmask buffers 0 and 1 of
-// ceil(K/32) words.  A call of generation g ORs into buffer g & 1 and zeroes
-// buffer (g + 1) & 1, which the previous call used and the next will use.
+// ws.fused: word 1 is the call generation g, words 0 and 2 are arrival
+// counters, words 4.. hold bitmask buffers 0 and 1 of ceil(K/32) words.  A
+// call of generation g counts its arrivals in counter g & 1 and ORs into
+// buffer g & 1; its CTA 0 zeroes counter and buffer (g + 1) & 1, which the
+// previous call used and the next will use, and bumps the generation once
+// every CTA has arrived.  A CTA arrives with a release add that returns
+// nothing (its flags ORed before the CTA barrier ahead of it), so no CTA waits
+// on the arrival itself.
 constexpr int kActFusedThreads = 1024;
 constexpr int kActFusedMaxRows = 16;  // rows per CTA
 constexpr size_t kActFusedSmemMax = 200 * 1024;
@@ -362,7 +365,7 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
   uint4* s_cm = reinterpret_cast<uint4*>(s_own + nw4);  // [kActFusedThreads] column maxima
   __shared__ uint64_t bar;
   __shared__ uint32_t s_gen;
-  __shared__ int s_released, s_more, s_nout;
+  __shared__ int s_more, s_nout;
   __shared__ float s_part[kActFusedThreads / 32][8];  // row maxima per warp
   __shared__ float s_k[kActFusedMaxRows];
   __shared__ float s_sc[kActFusedMaxRows];
@@ -378,7 +381,6 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
   const int g = tid / cpad;
   const bool col_ok = cc < nchunks && g < groups;
   const int m0 = g * R;                         // its first row (of the CTA's)
-  uint32_t* arrived = ws.fused;
   uint32_t* generation = ws.fused + 1;
 
   if (tid == 0) {
@@ -397,10 +399,12 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
   }
   __syncthreads();
   const uint32_t gen = s_gen;
+  uint32_t* arrived = ws.fused + 2 * (gen & 1u);
   uint32_t* buf = ws.fused + 4 + (gen & 1u) * uint32_t(nwords);
   uint32_t* other = ws.fused + 4 + ((gen + 1u) & 1u) * uint32_t(nwords);
   if (blockIdx.x == 0) {
     for (int w = tid; w < nwords; w += kActFusedThreads) other[w] = 0u;
+    if (tid == 0) ws.fused[2 * ((gen + 1u) & 1u)] = 0u;
   }
   const bool loaded = mbar_wait(&bar, 0, ws.status);
 
@@ -445,26 +449,13 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
   word |= __shfl_xor_sync(0xffffffffu, word, 2);
   if (g == 0 && col_ok && (cc & 3) == 0) {
     s_own[cc >> 2] = word;
-    if (word != 0u) {
-      atomicOr(buf + (cc >> 2), word);
-      __threadfence();
-    }
+    if (word != 0u) atomicOr(buf + (cc >> 2), word);
   }
 
-  // grid barrier, arrival (every CTA of the grid is resident: cooperative launch)
+  // grid barrier, arrival (every CTA of the grid is resident: cooperative
+  // launch); the CTA barrier puts every thread's OR before thread 0's release
   __syncthreads();
-  if (tid == 0) {
-    // (the stall test hook asks for one arrival more than the grid has: the
-    // barrier then never completes and every CTA's wait runs out)
-    const uint32_t last = gridDim.x - 1u + ((ws.stall & kStallActGridBarrier) ? 1u : 0u);
-    int released = 0;
-    if (atom_add_acq_rel_gpu_u32(arrived, 1u) == last) {
-      *arrived = 0u;                             // for the next call
-      st_release_gpu_u32(generation, gen + 1u);  // releases the others
-      released = 1;
-    }
-    s_released = released;
-  }
+  if (tid == 0) red_add_release_gpu_u32(arrived, 1u);
 
   // a2, a3 for the columns in `flags` (a superset of the ones zeroed so far):
   // zero them, row maxima over the rest, row scales, codes
@@ -535,15 +526,21 @@ __global__ void __launch_bounds__(kActFusedThreads, 1)
   // grid barrier, wait; then warp 0 reads the call's bitmask, compares it with
   // this CTA's flags and builds the popcount prefix (CTA 0 writes O and n_o)
   if (warp == 0) {
-    if (lane == 0 && !s_released) {
+    if (lane == 0) {
+      // (the stall test hook waits for one arrival more than the grid has:
+      // the barrier then never completes and every CTA's wait runs out)
+      const uint32_t all = gridDim.x + ((ws.stall & kStallActGridBarrier) ? 1u : 0u);
       const uint64_t t0 = globaltimer_ns();
       uint32_t n = 0;
-      while (ld_acquire_gpu_u32(generation) == gen) {
+      bool done = true;
+      while (ld_acquire_gpu_u32(arrived) < all) {
         if ((++n & 255u) == 0u && globaltimer_ns() - t0 > wait_limit_ns()) {
           atomicOr(ws.status, kStatusTimeout);
+          done = false;
           break;
         }
       }
+      if (blockIdx.x == 0 && done) *generation = gen + 1u;  // every CTA has read gen: the next call's
     }
     __syncwarp();
     const int wpl = (nwords + 31) / 32;  // contiguous words per lane
