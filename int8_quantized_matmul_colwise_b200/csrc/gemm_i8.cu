@@ -628,8 +628,16 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
         }
       };
       if (passes <= 1) {
-        // at most 16 outliers: their W rows over the whole tile were staged
-        // before the accumulator wait; one k16 step of the 16-bit product
+        // At most 16 outliers: their W rows over the whole tile were staged
+        // before the accumulator wait.  The 16-bit product runs on the CUDA
+        // cores (fp32 fused multiply-adds of exact fp16 products), not as
+        // mma.sync: legacy tensor-core instructions queue behind the int8
+        // tcgen05 MMAs of the next tile, which stretched the first tile's
+        // epilogue past the next main loop and held the third tile's MMAs
+        // back.  The four lanes of a row pair hold all 16 outlier values of
+        // rows g and g + 8 in their A fragments; a pair of them is one shuffle
+        // per row.
+        const __half* wo = s.wo + 2 * t4;
 #pragma unroll 1
         for (int c = 0; c < BN / 64; ++c) {  // 64 accumulator columns at a time
           const uint32_t taddr = tacc + c * 64;
@@ -638,14 +646,29 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
           tmem_ld_wait();
           float d[8][4];
           dequant(c, v, d);
-          // 16-bit outlier product on the tensor cores: d += Xo[rows, k] * W[O[k], cols]
-          if (n_use > 0) {
+          // d += Xo[rows, k] * W[O[k], cols], k < n_use
+#pragma unroll 1
+          for (int kp = 0; 2 * kp < n_use; ++kp) {  // k = 2 kp, 2 kp + 1 (a W row past n_use is zero)
+            const int src = 4 * g + (kp & 3);
+            const uint32_t xa = __shfl_sync(0xffffffffu, kp < 4 ? afr[0] : afr[2], src);  // row g
+            const uint32_t xb = __shfl_sync(0xffffffffu, kp < 4 ? afr[1] : afr[3], src);  // row g + 8
+            const float2 xg = __half22float2(*reinterpret_cast<const __half2*>(&xa));
+            const float2 xh = __half22float2(*reinterpret_cast<const __half2*>(&xb));
 #pragma unroll
-            for (int np = 0; np < 4; ++np) {
-              uint32_t b0, b1, b2, b3;
-              ldmatrix_x4_trans(wo_lane + 2u * static_cast<uint32_t>(c * 64 + 16 * np), b0, b1, b2, b3);
-              mma_m16n8k16_f16f32(d[2 * np], afr, b0, b1);
-              mma_m16n8k16_f16f32(d[2 * np + 1], afr, b2, b3);
+            for (int h = 0; h < 2; ++h) {
+              const float2 x0 = h ? make_float2(xg.y, xg.y) : make_float2(xg.x, xg.x);
+              const float2 x8 = h ? make_float2(xh.y, xh.y) : make_float2(xh.x, xh.x);
+              const __half* wr = wo + (2 * kp + h) * kWoStride + c * 64;
+#pragma unroll
+              for (int n = 0; n < 8; ++n) {
+                const float2 w2 = __half22float2(*reinterpret_cast<const __half2*>(wr + 8 * n));
+                const float2 lo = __ffma2_rn(x0, w2, make_float2(d[n][0], d[n][1]));
+                const float2 hi = __ffma2_rn(x8, w2, make_float2(d[n][2], d[n][3]));
+                d[n][0] = lo.x;
+                d[n][1] = lo.y;
+                d[n][2] = hi.x;
+                d[n][3] = hi.y;
+              }
             }
           }
           finish(c, d, true, taddr, v);
