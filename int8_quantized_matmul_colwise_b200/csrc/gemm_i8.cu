@@ -474,6 +474,14 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
   const bool overflow = n_o > p.cap;
   const int n_use = overflow ? 0 : n_o;
   const int passes = n_use > 0 ? (n_use + kSG - 1) / kSG : 1;  // outlier row groups staged per tile
+  // Where the 16-bit outlier product runs.  As mma.sync it shares the tensor
+  // cores with the next tile's tcgen05 MMAs and waits behind them (with six
+  // outliers on the 6.7B FFN shape that stretched the first tile's epilogue
+  // past the next main loop and held every later tile back); on the CUDA
+  // cores it costs about 0.56 us per outlier and tile, against a main loop of
+  // about 2.7 ns per unit of K.  So: the CUDA cores while n_o <= K / 256 (the
+  // epilogue stays inside the next main loop), mma.sync past that.
+  const bool core_product = int64_t(n_use) * 256 <= int64_t(p.K);
   __half* Y = static_cast<__half*>(p.Y);
   const bool y_pair = (p.ldy % 2 == 0) && (reinterpret_cast<uintptr_t>(p.Y) % 4 == 0);
   const bool w_vec = (p.ldw % 8 == 0) && (reinterpret_cast<uintptr_t>(p.W) % 16 == 0);
@@ -629,13 +637,10 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
       };
       if (passes <= 1) {
         // At most 16 outliers: their W rows over the whole tile were staged
-        // before the accumulator wait.  The 16-bit product runs on the CUDA
-        // cores (fp32 fused multiply-adds of exact fp16 products), not as
-        // mma.sync: legacy tensor-core instructions queue behind the int8
-        // tcgen05 MMAs of the next tile, which stretched the first tile's
-        // epilogue past the next main loop and held the third tile's MMAs
-        // back.  The four lanes of a row pair hold all 16 outlier values of
-        // rows g and g + 8 in their A fragments; a pair of them is one shuffle
+        // before the accumulator wait; one k16 step of the 16-bit product.
+        // On the CUDA cores: fp32 fused multiply-adds of the exact fp16
+        // products; the four lanes of a row pair hold all 16 outlier values of
+        // rows g and g + 8 in their A fragments, a pair of them is one shuffle
         // per row.
         const __half* wo = s.wo + 2 * t4;
 #pragma unroll 1
@@ -647,8 +652,17 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
           float d[8][4];
           dequant(c, v, d);
           // d += Xo[rows, k] * W[O[k], cols], k < n_use
+          if (!core_product) {
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+              uint32_t b0, b1, b2, b3;
+              ldmatrix_x4_trans(wo_lane + 2u * static_cast<uint32_t>(c * 64 + 16 * np), b0, b1, b2, b3);
+              mma_m16n8k16_f16f32(d[2 * np], afr, b0, b1);
+              mma_m16n8k16_f16f32(d[2 * np + 1], afr, b2, b3);
+            }
+          }
 #pragma unroll 1
-          for (int kp = 0; 2 * kp < n_use; ++kp) {  // k = 2 kp, 2 kp + 1 (a W row past n_use is zero)
+          for (int kp = 0; core_product && 2 * kp < n_use; ++kp) {  // k = 2 kp, 2 kp + 1 (a W row past n_use is zero)
             const int src = 4 * g + (kp & 3);
             const uint32_t xa = __shfl_sync(0xffffffffu, kp < 4 ? afr[0] : afr[2], src);  // row g
             const uint32_t xb = __shfl_sync(0xffffffffu, kp < 4 ? afr[1] : afr[3], src);  // row g + 8
@@ -722,16 +736,49 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
 #pragma unroll
                 for (int e = 0; e < 4; ++e) d[n][e] = __uint_as_float(v[4 * n + e]);
             }
+            if (core_product) {
+              // on the CUDA cores (k = 16 q + 2 kp + h)
 #pragma unroll
-            for (int q = 0; q < kRound / kSG; ++q) {
-              if (q < pr) {
+              for (int q = 0; q < kRound / kSG; ++q) {
+                if (q < pr) {
+#pragma unroll 1
+                  for (int kp = 0; kSG * q + 2 * kp < trn && kp < kSG / 2; ++kp) {
+                    const int src = 4 * g + (kp & 3);
+                    const uint32_t xa = __shfl_sync(0xffffffffu, kp < 4 ? ax[q][0] : ax[q][2], src);
+                    const uint32_t xb = __shfl_sync(0xffffffffu, kp < 4 ? ax[q][1] : ax[q][3], src);
+                    const float2 xg = __half22float2(*reinterpret_cast<const __half2*>(&xa));
+                    const float2 xh = __half22float2(*reinterpret_cast<const __half2*>(&xb));
 #pragma unroll
-                for (int np = 0; np < 4; ++np) {
-                  uint32_t b0, b1, b2, b3;
-                  ldmatrix_x4_trans(wo2_lane + 2u * static_cast<uint32_t>(q * kSG * kWo2Stride + 16 * np), b0, b1,
-                                    b2, b3);
-                  mma_m16n8k16_f16f32(d[2 * np], ax[q], b0, b1);
-                  mma_m16n8k16_f16f32(d[2 * np + 1], ax[q], b2, b3);
+                    for (int h = 0; h < 2; ++h) {
+                      const float2 x0 = h ? make_float2(xg.y, xg.y) : make_float2(xg.x, xg.x);
+                      const float2 x8 = h ? make_float2(xh.y, xh.y) : make_float2(xh.x, xh.x);
+                      const __half* wr = s.wo + (kSG * q + 2 * kp + h) * kWo2Stride + 2 * t4;
+#pragma unroll
+                      for (int n = 0; n < 8; ++n) {
+                        const float2 w2 = __half22float2(*reinterpret_cast<const __half2*>(wr + 8 * n));
+                        const float2 lo = __ffma2_rn(x0, w2, make_float2(d[n][0], d[n][1]));
+                        const float2 hi = __ffma2_rn(x8, w2, make_float2(d[n][2], d[n][3]));
+                        d[n][0] = lo.x;
+                        d[n][1] = lo.y;
+                        d[n][2] = hi.x;
+                        d[n][3] = hi.y;
+                      }
+                    }
+                  }
+                }
+              }
+            } else {
+#pragma unroll
+              for (int q = 0; q < kRound / kSG; ++q) {
+                if (q < pr) {
+#pragma unroll
+                  for (int np = 0; np < 4; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4_trans(wo2_lane + 2u * static_cast<uint32_t>(q * kSG * kWo2Stride + 16 * np), b0,
+                                      b1, b2, b3);
+                    mma_m16n8k16_f16f32(d[2 * np], ax[q], b0, b1);
+                    mma_m16n8k16_f16f32(d[2 * np + 1], ax[q], b2, b3);
+                  }
                 }
               }
             }

@@ -642,11 +642,15 @@ def test_bias_every_kernel(L, M, N, K, how):
     (300, 512, 1024, 96, 0),     # exactly one full round
     (300, 512, 1024, 97, 8),     # two rounds (partial sums parked in TMEM), TMA stores with a padded ldy
     (100, 600, 2048, 250, 3),    # three rounds, single-CTA tiles, direct stores (rows not 16-byte aligned)
+    (200, 300, 8192, 24, 0),     # n_o <= K / 256: the product on the CUDA cores, one round
+    (64, 257, 32768, 100, 8),    # on the CUDA cores, two rounds, padded ldy
+    (129, 257, 1024, 12, 0),     # 16 or fewer outliers but n_o > K / 256: mma.sync in the one-pass epilogue
 ])
 def test_many_outliers_epilogue_rounds(L, M, N, K, n_out, ldy_pad):
     """The GEMM epilogue with more than 16 outlier columns: the tile's
     64-column chunks outermost, rounds of up to 96 outlier rows, the bias added
-    in the last round, for the fp16 weight and the int8-only weight."""
+    in the last round, for the fp16 weight and the int8-only weight; the
+    16-bit product by mma.sync (n_o > K / 256) and on the CUDA cores."""
     rng = np.random.default_rng(M + N + K + n_out)
     X, W, _ = wl.random_small(rng, M, K, N, 0)
     cols = np.sort(rng.choice(K, size=n_out, replace=False))
