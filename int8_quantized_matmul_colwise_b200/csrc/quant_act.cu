@@ -787,6 +787,19 @@ inline int stream_stages(int64_t K) {
   return s > kStreamMaxStages ? kStreamMaxStages : s;
 }
 
+// The quantize pass does more work per row: a smaller ring (at least three
+// stages, which its one-row lookahead needs) lets three CTAs share an SM for
+// rows of up to 8192 columns.
+constexpr size_t kStreamRingQ = 64 * 1024;
+inline int stream_stages_q(int64_t K) {
+  const int s = static_cast<int>(kStreamRingQ / (size_t(K) * 2));
+  return s < 3 ? 3 : s > kStreamMaxStages ? kStreamMaxStages : s;
+}
+// Largest ring of the quantize pass for a CPT instance (its K range).
+constexpr size_t stream_ring_q_max(int CPT) {
+  return CPT <= 4 ? kStreamRingQ : size_t(3) * 2 * 8 * kStreamThreads * CPT;
+}
+
 // Rows of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
 __device__ __forceinline__ int64_t stream_rows(int64_t M) {
   return M > int64_t(blockIdx.x) ? (M - 1 - int64_t(blockIdx.x)) / int64_t(gridDim.x) + 1 : 0;
@@ -895,7 +908,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
 }
 
 template <int CPT>
-__global__ void __launch_bounds__(kStreamThreads, 2)
+__global__ void __launch_bounds__(kStreamThreads, CPT <= 4 ? 3 : 2)
     quantize_stream_kernel(const __half* __restrict__ X, int64_t M, int64_t K, int64_t ldx, ActWs ws,
                            int32_t* __restrict__ O, int32_t* __restrict__ n_out, int64_t cap, int8_t* __restrict__ Xq,
                            int64_t ldq, float* __restrict__ rs, __half* __restrict__ Xo, int64_t ldo, int stages) {
@@ -949,6 +962,19 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
   release_bitmask(ws, nwords, &s_last);  // its barrier also publishes s_list
   const int n_o = static_cast<int>(s_pre[nwords - 1]) + __popc(s_mask[nwords - 1]);
   const int nq = static_cast<int>(min(int64_t(n_o), cap));
+  // a thread's chunks are the same columns in every row: their outlier
+  // columns as AND masks over the fp16 pairs, once per CTA
+  uint4 keep[CPT];
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) {
+    const int c = tid + j * kStreamThreads;
+    const uint32_t om = c < nchunks ? (s_mask[c >> 2] >> ((c & 3) * 8)) & 0xFFu : 0u;
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      w[e] = (((om >> (2 * e)) & 1u) ? 0u : 0xFFFFu) | (((om >> (2 * e + 1)) & 1u) ? 0u : 0xFFFF0000u);
+    keep[j] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
 
   // Warp 0 alone waits for each row's copy (for row i + 1 just before row i's
   // barrier), the other warps at the barrier, which issues nothing.
@@ -971,14 +997,10 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
     __half2 m2 = __half2half2(__ushort_as_half(0));
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
-      const int c = tid + j * kStreamThreads;
-      const uint32_t om = c < nchunks ? (s_mask[c >> 2] >> ((c & 3) * 8)) & 0xFFu : 0u;
-      if (om != 0u) {
-        uint32_t* w = reinterpret_cast<uint32_t*>(&h[j]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          w[e] &= (((om >> (2 * e)) & 1u) ? 0u : 0xFFFFu) | (((om >> (2 * e + 1)) & 1u) ? 0u : 0xFFFF0000u);
-      }
+      h[j].x &= keep[j].x;
+      h[j].y &= keep[j].y;
+      h[j].z &= keep[j].z;
+      h[j].w &= keep[j].w;
       const __half2* h2 = reinterpret_cast<const __half2*>(&h[j]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(h2[e]));
@@ -1043,11 +1065,13 @@ cudaError_t launch_stream(cudaLaunchConfig_t cfg, int64_t M, const __half* x, in
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   const int stages = stream_stages(K);
+  const int stages_q = stream_stages_q(K);
   const size_t nw4 = static_cast<size_t>(((K + 31) / 32 + 3) & ~int64_t(3));
   const size_t smem_scan = size_t(stages) * size_t(K) * 2;
-  const size_t smem_q = smem_scan + 2 * nw4 * 4 + size_t(kStreamListMax) * 4;
+  const size_t smem_q = size_t(stages_q) * size_t(K) * 2 + 2 * nw4 * 4 + size_t(kStreamListMax) * 4;
+  constexpr size_t kSmemQMax = stream_ring_q_max(CPT) + 2 * 4 * 512 + 4 * kStreamListMax;
   if (!attr_set[dev]) {
-    // two CTAs of ~100 KB per SM need the largest shared-memory carveout
+    // two or three CTAs of 64-100 KB per SM need the largest shared-memory carveout
     e = cudaFuncSetAttribute(scan_stream_kernel<CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kStreamRing));
     if (e == cudaSuccess)
@@ -1055,7 +1079,7 @@ cudaError_t launch_stream(cudaLaunchConfig_t cfg, int64_t M, const __half* x, in
                                cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(quantize_stream_kernel<CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kStreamRing + 2 * 4 * 512 + 4 * kStreamListMax));
+                               static_cast<int>(kSmemQMax));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(quantize_stream_kernel<CPT>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                cudaSharedmemCarveoutMaxShared);
@@ -1065,13 +1089,13 @@ cudaError_t launch_stream(cudaLaunchConfig_t cfg, int64_t M, const __half* x, in
                                                         kStreamRing);
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[dev][1], quantize_stream_kernel<CPT>, kStreamThreads,
-                                                        kStreamRing + 2 * 4 * 512 + 4 * kStreamListMax);
+                                                        kSmemQMax);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  auto clamp12 = [](int v) { return v < 1 ? 1 : v > 2 ? 2 : v; };
-  const int64_t ctas_scan = int64_t(num_sms) * clamp12(per_sm[dev][0]);
-  const int64_t ctas_q = int64_t(num_sms) * clamp12(per_sm[dev][1]);
+  auto clamp = [](int v, int hi) { return v < 1 ? 1 : v > hi ? hi : v; };
+  const int64_t ctas_scan = int64_t(num_sms) * clamp(per_sm[dev][0], 2);
+  const int64_t ctas_q = int64_t(num_sms) * clamp(per_sm[dev][1], 3);
   cfg.blockDim = dim3(kStreamThreads);
   cfg.gridDim = dim3(static_cast<unsigned>(M < ctas_scan ? M : ctas_scan));
   cfg.dynamicSmemBytes = smem_scan;
@@ -1080,7 +1104,7 @@ cudaError_t launch_stream(cudaLaunchConfig_t cfg, int64_t M, const __half* x, in
   cfg.gridDim = dim3(static_cast<unsigned>(M < ctas_q ? M : ctas_q));
   cfg.dynamicSmemBytes = smem_q;
   return cudaLaunchKernelEx(&cfg, quantize_stream_kernel<CPT>, x, M, K, ldx, ws, O, n, cap, Xq, ldq, rs, xo, ldo,
-                            stages);
+                            stages_q);
 }
 
 template <int G, int CPT>
