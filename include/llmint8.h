@@ -133,10 +133,13 @@ llmint8_status llmint8_quantize_weight_colwise(const void* W, int64_t K, int64_t
  * All outputs are device-side; nothing is copied to the host.  When X's rows
  * are 16-byte aligned (ldx % 8 == 0, K % 8 == 0) and X fits in shared memory
  * spread over the SMs (at most 16 rows and 200 KB per SM), the step is one
- * persistent kernel: X is read once, the CTAs meet at a grid barrier between
- * the column scan and the row quantization, and no other kernel may hold SMs
- * for long on other streams meanwhile (the barrier gives up after 2 s and sets
- * LLMINT8_STATUS_TIMEOUT).  Otherwise two kernels (column scan, rows). */
+ * cooperative kernel (the driver guarantees its CTAs are resident together):
+ * X is read once, and the CTAs meet at a grid barrier between the column scan
+ * and the row quantization (bounded: after 2 s it sets
+ * LLMINT8_STATUS_TIMEOUT, and the workspace must be zero-filled again before
+ * reuse).  Otherwise two kernels: for many such rows with 2048 <= K <= 16384
+ * a column scan and a row pass that stream whole rows through shared memory,
+ * else a column scan and a per-row kernel. */
 llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, int64_t K, int64_t ldx,
                                                      float tau, int8_t* Xq, int64_t ldq, float* row_scale,
                                                      int32_t* outlier_idx, int64_t outlier_cap,
