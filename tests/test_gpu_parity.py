@@ -327,6 +327,41 @@ def test_int8_gemm_extreme_codes(L):
     assert np.all(C[0::2] == 127 * 127 * K) and np.all(C[1::2] == -127 * 127 * K)
 
 
+K_MAX = 133143  # the largest K the library takes: 127^2 * K < 2^31
+
+
+def test_int8_gemm_extreme_codes_at_the_largest_k(L):
+    """All +-127 codes at K = 133143: the int32 sums reach +-(2^31 - 20201)."""
+    M, N, K = 130, 40, K_MAX
+    ldq = L.round_up(K, 16)
+    Xq = np.zeros((M, ldq), np.int8)
+    Xq[:, :K] = 127
+    Xq[1::2, :K] = -127
+    Wq = np.zeros((N, ldq), np.int8)
+    Wq[:, :K] = 127
+    C = host(L.debug_int8_gemm_i32(dev(Xq), dev(Wq), K))
+    assert 127 * 127 * K < 2 ** 31
+    assert np.all(C[0::2] == 127 * 127 * K) and np.all(C[1::2] == -127 * 127 * K)
+
+
+@pytest.mark.parametrize("M", [2, 130])
+def test_mixed_matmul_at_the_largest_k(L, M):
+    """The whole path at K = 133143 (long-row activation kernel; split-K
+    decode GEMM for M = 2, tcgen05 GEMM for M = 130): X rows of +-0.5 and W
+    columns of 2^-10 quantize to +-127 everywhere, so every accumulator is
+    +-127^2 K; Y = +-K / 2048, within fp16 range, against the oracle."""
+    N, K = 24, K_MAX
+    X = np.full((M, K), 0.5, np.float16)
+    X[1::2] = -0.5
+    W = np.full((K, N), 2.0 ** -10, np.float16)
+    Y, ws, v, (Wq, cs), (st, flags) = run_path(L, X, W, np.inf)
+    assert st == 0 and flags == 0
+    assert np.array_equal(host(v["xq"])[:, :K], np.where(X > 0, 127, -127).astype(np.int8))
+    r = oracle.mixed_matmul(X, W, np.inf)
+    y_close(host(Y), r["Y"])
+    assert np.allclose(host(Y).astype(np.float64)[0], K / 2048.0, rtol=1e-3)
+
+
 # ------------------------------------------------------------------ a0-a7: the whole path
 
 def run_path(L, X, W, tau, cap=None, rows=None):
