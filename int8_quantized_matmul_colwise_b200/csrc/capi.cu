@@ -80,33 +80,89 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// A 2D tensor map with the 128-byte swizzle (out-of-range reads give 0).  A
+// map depends only on its arguments, so the last kMapCache maps encoded on
+// this thread are kept and handed out again for the same arguments: a call
+// that repeats the previous calls' buffers and shapes encodes nothing.
+constexpr int kMapCache = 64;
+struct MapKey {
+  CUtensorMapDataType type;
+  const void* base;
+  uint64_t cols, rows, stride;
+  uint32_t box_cols, box_rows;
+  bool operator==(const MapKey& o) const {
+    return type == o.type && base == o.base && cols == o.cols && rows == o.rows && stride == o.stride &&
+           box_cols == o.box_cols && box_rows == o.box_rows;
+  }
+};
+struct MapCache {
+  MapKey key[kMapCache];
+  CUtensorMap map[kMapCache];
+  int size = 0, next = 0;
+};
+
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, int64_t cols, int64_t rows,
+               int64_t stride_bytes, uint32_t box_cols, uint32_t box_rows) {
+  thread_local MapCache cache;
+  const MapKey k = {type, base, static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
+                    static_cast<uint64_t>(stride_bytes), box_cols, box_rows};
+  for (int i = 0; i < cache.size; ++i) {
+    if (cache.key[i] == k) {
+      *map = cache.map[i];
+      return true;
+    }
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride_bytes)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  if (fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  cache.key[cache.next] = k;
+  cache.map[cache.next] = *map;
+  cache.next = (cache.next + 1) % kMapCache;
+  if (cache.size < kMapCache) ++cache.size;
+  return true;
+}
+
 // int8 matrix [rows, cols] with row stride ld (bytes), read in boxes of
 // box_rows x 128 bytes with the 128-byte swizzle; out-of-range reads are 0.
 bool encode_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
                         uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemmBK), box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, cols, rows, ld, kGemmBK, box_rows);
+}
+
+// fp16 operand of the tensor-core outlier product: [rows, 128] contiguous,
+// read in boxes of 128 rows x 64 columns (128 bytes) with the 128-byte swizzle.
+bool encode_outlier_map(CUtensorMap* map, const void* base, int64_t rows) {
+  return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, kOutlierMmaMax, rows, 2 * kOutlierMmaMax, 64, 128);
+}
+
+// The tensor-core outlier product of a CTA-pair GEMM: its two counters sit in
+// the workspace header (zero between calls), its gathered operands (Xo
+// [M, 128] then W^T [N, 128], fp16) at `data`.  Leaves a.om_ok false (the
+// epilogue computes the product) when the maps cannot be made.
+void prepare_outlier_mma(GemmArgs& a, CUtensorMap* tmXo, CUtensorMap* tmWo, void* ws, uint8_t* data) {
+  std::memset(tmXo, 0, sizeof(*tmXo));
+  std::memset(tmWo, 0, sizeof(*tmWo));
+  a.om_ok = false;
+  if (!gemm_uses_pair(a.M) || data == nullptr) return;
+  uint8_t* wo_t = data + size_t(a.M) * 2 * kOutlierMmaMax;
+  if (!encode_outlier_map(tmXo, data, a.M) || !encode_outlier_map(tmWo, wo_t, a.N)) return;
+  a.xo_p = data;
+  a.wo_t = wo_t;
+  a.om_sync = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + 16);
+  a.om_ok = true;
 }
 
 // fp16 output Y [rows, cols] with row stride ld (elements), written in boxes of
 // 16 rows x 64 columns with the 128-byte swizzle.  Needs 16-byte aligned rows.
 bool encode_output_map(CUtensorMap* map, void* base, int64_t rows, int64_t cols, int64_t ld) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-  const cuuint32_t box[2] = {64, 16};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, cols, rows, 2 * ld, 64, 16);
 }
 
 // Y through TMA stores when its rows are 16-byte aligned; direct stores otherwise.
@@ -117,7 +173,7 @@ bool prepare_output(CUtensorMap* map, void* Y, int64_t M, int64_t N, int64_t ldy
 }
 
 // ------------------------------------------------------------------ workspace
-// [0, 256)        header: status u32 @0, n_o i32 @8
+// [0, 256)        header: status u32 @0, n_o i32 @8, outlier-product counters u32 [2] @16 (zero between calls)
 // colmax          u32 [K]                 zero between calls
 // blk_counter     u32 [ceil(K/256)]       zero between calls
 // bitmask         u32 [ceil(K/32)]
@@ -126,8 +182,9 @@ bool prepare_output(CUtensorMap* map, void* Y, int64_t M, int64_t N, int64_t ldy
 // xq              i8  [M, ldq]
 // xo              f16 [M, ldo]
 // decode          (M <= kDecodeMaxM) split-K partial sums + tile counters, zero between calls
+// outlier operands (CTA-pair GEMMs) fp16 Xo [M, 128] + W^T [N, 128] of the tensor-core outlier product
 bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t* colmax, size_t* bitmask,
-                 int64_t N = 0, size_t* decode = nullptr) {
+                 int64_t N = 0, size_t* decode = nullptr, size_t* outlier_ops = nullptr) {
   if (M < 1 || K < 1 || K > kMaxK || cap < 0 || cap > K) return false;
   size_t off = 256;
   *colmax = off;
@@ -151,6 +208,11 @@ bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t
   off = align_up(off + 2 * size_t(M) * size_t(L->ldo), 256);
   if (decode) *decode = off;
   if (M <= kDecodeMaxM && N > 0) off += decode_scratch_bytes(static_cast<int>(M), static_cast<int>(N));
+  if (N > 0 && gemm_uses_pair(static_cast<int>(M))) {
+    off = align_up(off, 256);
+    if (outlier_ops) *outlier_ops = off;
+    off += outlier_mma_bytes(M, N);
+  }
   L->total = off;
   return true;
 }
@@ -354,8 +416,9 @@ llmint8_status mixed_matmul_impl(const void* X, int64_t M, int64_t K, int64_t ld
       !aligned(bias, 2))
     return LLMINT8_ERR_INVALID_ARG;
   llmint8_ws_layout L;
-  size_t colmax_off, bitmask_off, decode_off;
-  if (!make_layout(M, K, outlier_cap, &L, &colmax_off, &bitmask_off, N, &decode_off)) return LLMINT8_ERR_INVALID_ARG;
+  size_t colmax_off, bitmask_off, decode_off, om_off = 0;
+  if (!make_layout(M, K, outlier_cap, &L, &colmax_off, &bitmask_off, N, &decode_off, &om_off))
+    return LLMINT8_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return LLMINT8_ERR_WORKSPACE;
   int num_sms = 0;
   llmint8_status st = current_device(&num_sms);
@@ -506,14 +569,15 @@ llmint8_status mixed_matmul_impl(const void* X, int64_t M, int64_t K, int64_t ld
   a.ldc = ldc;
   a.status = reinterpret_cast<uint32_t*>(b + L.status);
   a.stall = stall_mask();
-  CUtensorMap tmY;
+  CUtensorMap tmY, tmXo, tmWo;
   if (C) {
     std::memset(&tmY, 0, sizeof(tmY));
     a.y_tma = false;
   } else {
     a.y_tma = prepare_output(&tmY, Y, M, N, ldy);
   }
-  return cuda_status(launch_gemm_i8(tmA, tmB, tmY, a, C != nullptr, num_sms, s, true));
+  prepare_outlier_mma(a, &tmXo, &tmWo, ws, om_off ? b + om_off : nullptr);
+  return cuda_status(launch_gemm_i8(tmA, tmB, tmY, tmXo, tmWo, a, C != nullptr, num_sms, s, true));
 }
 
 }  // namespace
@@ -628,9 +692,18 @@ llmint8_status llmint8_mixed_gemm(const int8_t* Xq, int64_t ldq, const float* ro
   a.ldy = ldy;
   a.status = static_cast<uint32_t*>(ws);
   a.stall = stall_mask();
-  CUtensorMap tmY;
+  CUtensorMap tmY, tmXo, tmWo;
   a.y_tma = prepare_output(&tmY, Y, M, N, ldy);
-  return cuda_status(launch_gemm_i8(tmA, tmB, tmY, a, false, num_sms, static_cast<cudaStream_t>(stream), true));
+  // The outlier operands where llmint8_mixed_matmul keeps them, when the
+  // workspace is that large: past the activation step's scratch and its Xq
+  // and Xo, so the same workspace serves both entry points.
+  llmint8_ws_layout Lw;
+  size_t colmax_off, bitmask_off, om_off = 0;
+  const bool om_room = make_layout(M, K, outlier_cap, &Lw, &colmax_off, &bitmask_off, N, nullptr, &om_off) &&
+                       om_off != 0 && ws_bytes >= Lw.total;
+  prepare_outlier_mma(a, &tmXo, &tmWo, ws, om_room ? static_cast<uint8_t*>(ws) + om_off : nullptr);
+  return cuda_status(
+      launch_gemm_i8(tmA, tmB, tmY, tmXo, tmWo, a, false, num_sms, static_cast<cudaStream_t>(stream), true));
 }
 
 llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const int8_t* Wq, int64_t ldk,
@@ -674,10 +747,12 @@ llmint8_status llmint8_debug_int8_gemm_i32(const int8_t* Xq, int64_t ldq, const 
   a.C = C;
   a.ldc = ldc;
   a.status = static_cast<uint32_t*>(ws);
-  CUtensorMap tmY;
+  CUtensorMap tmY, tmXo, tmWo;
   std::memset(&tmY, 0, sizeof(tmY));
   a.y_tma = false;
-  return cuda_status(launch_gemm_i8(tmA, tmB, tmY, a, true, num_sms, static_cast<cudaStream_t>(stream), false));
+  prepare_outlier_mma(a, &tmXo, &tmWo, ws, nullptr);  // no outlier product in the raw accumulator dump
+  return cuda_status(
+      launch_gemm_i8(tmA, tmB, tmY, tmXo, tmWo, a, true, num_sms, static_cast<cudaStream_t>(stream), false));
 }
 
 llmint8_status llmint8_unshard_columns(const void* blocks, int64_t world, int64_t M, int64_t ld_block,

@@ -62,6 +62,18 @@ constexpr int kWoStride = BN + 8;  // halves per staged row: 528 bytes, conflict
 // run on it in registers.
 constexpr int kRound = 96;
 constexpr int kWo2Stride = 72;  // halves per staged row of a chunk: 144 bytes, conflict-free ldmatrix
+// Many outliers on CTA pairs (K/256 < n_o <= kOutlierMmaMax): the outlier
+// product runs on the tensor cores.  The epilogue dequantizes the tile in
+// TMEM (int32 -> fp32 in place) and the MMA thread accumulates Xo * W[O, :]
+// onto it with kind::f16 MMAs (fp16 operands, fp32 accumulation).  Each block
+// of 64 outlier columns is one ring stage (128 rows of Xo and 128 rows of the
+// gathered W^T, 128 bytes each, per CTA), and a tile's blocks enter the ring
+// kOmLag blocks into the next tile's main loop, by which time the epilogue has
+// the tile dequantized.
+constexpr int kOmLag = 4;
+constexpr int kOmCols = kOutlierMmaMax;   // fp16 columns of the gathered operands
+constexpr int kOmUnit = 32;               // rows of W^T or Xo per gather unit
+constexpr int kOmStride = kOmCols + 8;    // halves per row of the transposing tile: 272 bytes
 
 template <bool kPair>
 struct Geo {
@@ -81,12 +93,14 @@ struct Geo {
   static constexpr uint32_t kOffY = (kOffBias + BN * 4 + 1023) & ~1023u;
   static constexpr uint32_t kYBytes = 16 * 128;
   static constexpr uint32_t kOffBars = kOffY + kEpiWarps * kYBytes;
-  static constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;  // full, empty, tmem full/empty, drain
+  // full, empty, tmem full/empty, drain, dequantized (pair leader), outlier product done
+  static constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1 + 2 + 2;
   static constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
   static constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
   // Arrivals that free a TMEM accumulator: one per epilogue warp of each CTA.
   static constexpr uint32_t kTmemEmptyArrivals = kPair ? 2 * kEpiWarps : kEpiWarps;
   static_assert(kBytesA % 1024 == 0 && kBytesB % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static_assert(kOmUnit * kOmStride * 2 <= kWoBytes, "the gather's transposing tile fits the staging area");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -102,6 +116,8 @@ struct Shared {
   uint64_t* tfull;
   uint64_t* tempty;
   uint64_t* drain;
+  uint64_t* deq;    // [2] the epilogue has written the dequantized tile to TMEM (pair leader)
+  uint64_t* ofull;  // [2] the outlier MMAs on that tile are done
   uint32_t* tmem_slot;
   volatile int* abort;
 };
@@ -123,6 +139,8 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
   s.tfull = bars + 2 * G::kStages;
   s.tempty = bars + 2 * G::kStages + 2;
   s.drain = bars + 2 * G::kStages + 4;
+  s.deq = bars + 2 * G::kStages + 5;
+  s.ofull = bars + 2 * G::kStages + 7;
   s.tmem_slot = reinterpret_cast<uint32_t*>(base + G::kOffMisc);
   s.abort = reinterpret_cast<volatile int*>(base + G::kOffMisc + 4);
   return s;
@@ -181,44 +199,106 @@ __device__ __forceinline__ void tile_coords(int tile, const Sched& sc, int& mb, 
   nb = r / rows;
 }
 
+// Blocks of 64 outlier columns the tensor-core outlier product takes for this
+// call (0: the epilogue computes the product itself).  Every role of every CTA
+// derives the same value from n_o.
+__device__ __forceinline__ int outlier_mma_blocks(const GemmArgs& p) {
+  if (!p.om_ok) return 0;
+  const int n_o = *p.n_o;
+  if (n_o > p.cap || n_o > kOmCols || int64_t(n_o) * 256 <= int64_t(p.K)) return 0;
+  return (n_o + 63) / 64;
+}
+
+// Bounded wait until a global counter reaches `target` (acquire).
+__device__ __forceinline__ bool wait_counter(const uint32_t* ctr, uint32_t target, uint32_t* status,
+                                             volatile int* abort) {
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t n = 0;
+  while (ld_acquire_gpu_u32(ctr) < target) {
+    if ((++n & 63u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > wait_limit_ns()) {
+        atomicOr(status, kStatusTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
 template <bool kPair>
-__device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const Shared& s, const Sched& sc,
-                             uint32_t rank, uint32_t* status) {
+__device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmXo,
+                             const CUtensorMap* tmWo, const Shared& s, const Sched& sc, uint32_t rank,
+                             const GemmArgs& p, bool om_possible) {
   using G = Geo<kPair>;
   const uint64_t hint = policy_evict_last();
   uint32_t stage = 0, phase = 0;
   uint32_t issued = 0;        // bit s: stage s has had a load issued
   uint32_t issued_phase = 0;  // bit s: the phase of that load
+  uint32_t* const status = p.status;
+  // Blocks of the tensor-core outlier product, read where they are first
+  // needed (one tile into the main loop), so n_o's load never delays the
+  // first copies.
+  int om = om_possible ? -1 : 0;
+  auto om_blocks = [&]() {
+    if (om < 0) om = outlier_mma_blocks(p);
+    return om;
+  };
+  bool gathered = false;      // the gathered outlier operands are complete in global memory
+  // one ring stage: the box at column x of both maps
+  auto load = [&](const CUtensorMap* ta, const CUtensorMap* tb, int x, int ya, int yb) -> bool {
+    if (!wait_or_abort(&s.empty[stage], phase ^ 1u, status, s.abort)) return false;
+    if constexpr (kPair) {
+      // both CTAs' bytes are counted on the leader's full barrier
+      if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * (G::kBytesA + G::kBytesB));
+      const uint32_t bar = mapa_shared(smem_u32(&s.full[stage]), 0);
+      tma_load_2d_pair(s.a + stage * G::kBytesA, ta, bar, x, ya, hint);
+      tma_load_2d_pair(s.b + stage * G::kBytesB, tb, bar, x, yb, hint);
+    } else {
+      mbar_arrive_expect_tx(&s.full[stage], G::kBytesA + G::kBytesB);
+      tma_load_2d(s.a + stage * G::kBytesA, ta, &s.full[stage], x, ya, hint);
+      tma_load_2d(s.b + stage * G::kBytesB, tb, &s.full[stage], x, yb, hint);
+    }
+    issued |= 1u << stage;
+    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+    if (++stage == G::kStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+    return true;
+  };
+  // a tile's outlier blocks: 64 columns of Xo (A) and of W^T (B) each
+  auto load_outliers = [&](int ya, int yb) -> bool {
+    if (!gathered) {  // every CTA's share of the gather, then TMA reads of it
+      if (!wait_counter(p.om_sync, gridDim.x, status, s.abort)) return false;
+      fence_proxy_async_global();
+      gathered = true;
+    }
+    for (int ob = 0; ob < om; ++ob)
+      if (!load(tmXo, tmWo, ob * 64, ya, yb)) return false;
+    return true;
+  };
   bool ok = true;
+  bool prev = false;
+  int pya = 0, pyb = 0;  // the previous tile's rows
+  const int ins = sc.num_k < kOmLag ? sc.num_k : kOmLag;
   for (int tile = sc.first; tile < sc.num_tiles && ok; tile += sc.stride) {
     int mb, nb;
     tile_coords(tile, sc, mb, nb);
     const int ya = mb * G::kTileM + (kPair ? static_cast<int>(rank) * BM : 0);
     const int yb = nb * BN + (kPair ? static_cast<int>(rank) * G::kRowsB : 0);
-    for (int kb = 0; kb < sc.num_k; ++kb) {
-      if (!wait_or_abort(&s.empty[stage], phase ^ 1u, status, s.abort)) {
-        ok = false;
-        break;
-      }
-      if constexpr (kPair) {
-        // both CTAs' bytes are counted on the leader's full barrier
-        if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * (G::kBytesA + G::kBytesB));
-        const uint32_t bar = mapa_shared(smem_u32(&s.full[stage]), 0);
-        tma_load_2d_pair(s.a + stage * G::kBytesA, tmA, bar, kb * BK, ya, hint);
-        tma_load_2d_pair(s.b + stage * G::kBytesB, tmB, bar, kb * BK, yb, hint);
-      } else {
-        mbar_arrive_expect_tx(&s.full[stage], G::kBytesA + G::kBytesB);
-        tma_load_2d(s.a + stage * G::kBytesA, tmA, &s.full[stage], kb * BK, ya, hint);
-        tma_load_2d(s.b + stage * G::kBytesB, tmB, &s.full[stage], kb * BK, yb, hint);
-      }
-      issued |= 1u << stage;
-      issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-      if (++stage == G::kStages) {
-        stage = 0;
-        phase ^= 1u;
-      }
+    // the main loop's blocks in two runs, the previous tile's outlier blocks between them
+    for (int run = 0; run < 2 && ok; ++run) {
+      if (run == 1 && prev && om != 0 && om_blocks() > 0) ok = load_outliers(pya, pyb);
+      const int k_end = run == 0 ? ins : sc.num_k;
+      for (int kb = run == 0 ? 0 : ins; kb < k_end && ok; ++kb) ok = load(tmA, tmB, kb * BK, ya, yb);
     }
+    prev = true;
+    pya = ya;
+    pyb = yb;
   }
+  if (ok && prev && om != 0 && om_blocks() > 0) ok = load_outliers(pya, pyb);
   if (!ok && (!kPair || rank == 0)) {
     // Let the copies already in flight land before the CTA exits.
     for (int st = 0; st < G::kStages; ++st)
@@ -227,16 +307,56 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
 }
 
 template <bool kPair>
-__device__ void run_mma(const Shared& s, uint32_t tmem_base, const Sched& sc, uint32_t* status, uint32_t stall) {
+__device__ void run_mma(const Shared& s, uint32_t tmem_base, const Sched& sc, const GemmArgs& p, bool om_possible) {
   using G = Geo<kPair>;
+  uint32_t* const status = p.status;
+  const uint32_t stall = p.stall;
+  int om = om_possible ? -1 : 0;  // read where first needed, as in the producer
+  auto om_blocks = [&]() {
+    if (om < 0) om = outlier_mma_blocks(p);
+    return om;
+  };
   constexpr uint32_t idesc = idesc_i8(G::kTileM, BN);
   uint32_t stage = 0, phase = 0, it = 0;
   bool ok = true;
   bool any = false;
+  // The outlier product of the tile in accumulator pb (its use-th use): once
+  // both CTAs' epilogues have dequantized it in TMEM, fp16 MMAs accumulate
+  // onto it, and the commit tells both epilogues that it is done.
+  auto outliers = [&](uint32_t pb, uint32_t puse) -> bool {
+    if constexpr (kPair) {
+      constexpr uint32_t idesc_o = idesc_f16(G::kTileM, BN);
+      if (!wait_or_abort(&s.deq[pb], puse, status, s.abort)) return false;
+      tc_fence_after();
+      const uint32_t d = tmem_base + pb * kAccCols;
+      for (int ob = 0; ob < om; ++ob) {
+        if (!wait_or_abort(&s.full[stage], phase, status, s.abort)) return false;
+        tc_fence_after();
+        const uint64_t da = smem_desc_k_sw128(smem_u32(s.a + stage * G::kBytesA));
+        const uint64_t db = smem_desc_k_sw128(smem_u32(s.b + stage * G::kBytesB));
+#pragma unroll
+        for (int kk = 0; kk < BK / 32; ++kk)  // K = 16 fp16 = 32 bytes per MMA, as for int8
+          mma_f16_pair(d, da + 2u * kk, db + 2u * kk, idesc_o, 1u);
+        any = true;
+        mma_commit_pair(&s.empty[stage], 0x3);
+        if (++stage == G::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      mma_commit_pair(&s.ofull[pb], 0x3);
+      return true;
+    } else {
+      (void)pb;
+      (void)puse;
+      return false;
+    }
+  };
   // (the stall test hook first waits on the drain barrier, which nothing has
   // arrived on yet: the wait runs out before any MMA is issued and the CTA
   // takes the abort path)
   if ((stall & kStallGemmOperands) && !wait_or_abort(s.drain, 0, status, s.abort)) ok = false;
+  const int ins = sc.num_k < kOmLag ? sc.num_k : kOmLag;
   for (int tile = sc.first; tile < sc.num_tiles && ok; tile += sc.stride, ++it) {
     const uint32_t b = it & 1u;
     const uint32_t use = (it >> 1) & 1u;
@@ -246,31 +366,39 @@ __device__ void run_mma(const Shared& s, uint32_t tmem_base, const Sched& sc, ui
     }
     tc_fence_after();
     const uint32_t d = tmem_base + b * kAccCols;
-    for (int kb = 0; kb < sc.num_k; ++kb) {
-      if (!wait_or_abort(&s.full[stage], phase, status, s.abort)) {
+    // the main loop's blocks in two runs, the previous tile's outlier blocks between them
+    for (int run = 0; run < 2 && ok; ++run) {
+      if (run == 1 && it > 0 && om != 0 && om_blocks() > 0 && !outliers(b ^ 1u, ((it - 1) >> 1) & 1u)) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      const uint64_t da = smem_desc_k_sw128(smem_u32(s.a + stage * G::kBytesA));
-      const uint64_t db = smem_desc_k_sw128(smem_u32(s.b + stage * G::kBytesB));
+      const int k_end = run == 0 ? ins : sc.num_k;
+      for (int kb = run == 0 ? 0 : ins; kb < k_end; ++kb) {
+        if (!wait_or_abort(&s.full[stage], phase, status, s.abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t da = smem_desc_k_sw128(smem_u32(s.a + stage * G::kBytesA));
+        const uint64_t db = smem_desc_k_sw128(smem_u32(s.b + stage * G::kBytesB));
 #pragma unroll
-      for (int kk = 0; kk < BK / 32; ++kk) {
-        // +32 bytes along K inside the 128-byte swizzle atom = +2 in the
-        // descriptor's 16-byte address units.
+        for (int kk = 0; kk < BK / 32; ++kk) {
+          // +32 bytes along K inside the 128-byte swizzle atom = +2 in the
+          // descriptor's 16-byte address units.
+          if constexpr (kPair)
+            mma_i8_pair(d, da + 2u * kk, db + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          else
+            mma_i8(d, da + 2u * kk, db + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        any = true;
         if constexpr (kPair)
-          mma_i8_pair(d, da + 2u * kk, db + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          mma_commit_pair(&s.empty[stage], 0x3);
         else
-          mma_i8(d, da + 2u * kk, db + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-      }
-      any = true;
-      if constexpr (kPair)
-        mma_commit_pair(&s.empty[stage], 0x3);
-      else
-        mma_commit(&s.empty[stage]);
-      if (++stage == G::kStages) {
-        stage = 0;
-        phase ^= 1u;
+          mma_commit(&s.empty[stage]);
+        if (++stage == G::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
     }
     if (ok) {
@@ -280,6 +408,8 @@ __device__ void run_mma(const Shared& s, uint32_t tmem_base, const Sched& sc, ui
         mma_commit(&s.tfull[b]);
     }
   }
+  // the last tile's outlier product
+  if (ok && it > 0 && om != 0 && om_blocks() > 0 && !outliers((it - 1) & 1u, ((it - 1) >> 1) & 1u)) ok = false;
   if (!ok && any) {
     // Make sure no MMA is still writing TMEM before it is freed.
     if constexpr (kPair)
@@ -463,9 +593,77 @@ __device__ __forceinline__ void load_xo_fragment(const GemmArgs& p, int r0, int 
   }
 }
 
+// This CTA's share of the operands of the tensor-core outlier product, by all
+// epilogue threads before the first tile: W^T [N, 128] (row j of column n is
+// W[O[j], n], or the row recovered from Wq without an fp16 weight) and Xo
+// [M, 128], zero past n_o, in units of kOmUnit rows.  W rows are read along N
+// and transposed through shared memory so that both sides are coalesced.
+__device__ void gather_outlier_operands(const GemmArgs& p, const Shared& s, int et) {
+  const int n_o = *p.n_o;
+  const int units_n = (p.N + kOmUnit - 1) / kOmUnit;
+  const int units = units_n + (p.M + kOmUnit - 1) / kOmUnit;
+  const __half* W = static_cast<const __half*>(p.W);
+  const __half* Xo = static_cast<const __half*>(p.Xo);
+  uint16_t* wt = static_cast<uint16_t*>(p.wo_t);
+  uint16_t* xp = static_cast<uint16_t*>(p.xo_p);
+  const bool w_vec = (p.ldw % 8 == 0) && (reinterpret_cast<uintptr_t>(p.W) % 16 == 0);
+  uint16_t* tile = reinterpret_cast<uint16_t*>(s.wo);  // [kOmUnit][kOmStride]
+  for (int u = static_cast<int>(blockIdx.x); u < units; u += static_cast<int>(gridDim.x)) {
+    if (u >= units_n) {  // Xo rows
+      const int m0 = (u - units_n) * kOmUnit;
+      for (int i = et; i < kOmUnit * kOmCols; i += kEpiThreads) {
+        const int m = m0 + i / kOmCols, j = i % kOmCols;
+        if (m < p.M) xp[int64_t(m) * kOmCols + j] = j < n_o ? __half_as_ushort(Xo[int64_t(m) * p.ldo + j]) : 0;
+      }
+      continue;
+    }
+    const int n0 = u * kOmUnit;
+    if (W == nullptr) {  // no fp16 weight kept: the rows recovered from Wq
+      for (int i = et; i < kOmUnit * kOmCols; i += kEpiThreads) {
+        const int n = n0 + i / kOmCols, j = i % kOmCols;
+        if (n < p.N)
+          wt[int64_t(n) * kOmCols + j] =
+              j < n_o ? dequant_weight_bits(p.Wq[int64_t(n) * p.ldk + __ldg(p.O + j)], __ldg(p.cs + n)) : 0;
+      }
+      continue;
+    }
+    // pieces of 8 columns of a W row into the transposing tile
+    for (int pc = et; pc < kOmCols * (kOmUnit / 8); pc += kEpiThreads) {
+      const int j = pc / (kOmUnit / 8), c = 8 * (pc % (kOmUnit / 8));
+      uint16_t v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (j < n_o) {
+        const __half* wr = W + int64_t(__ldg(p.O + j)) * p.ldw + n0 + c;
+        if (w_vec && n0 + c + 8 <= p.N) {
+          const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(wr));
+          const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            v[2 * e] = static_cast<uint16_t>(w[e] & 0xFFFFu);
+            v[2 * e + 1] = static_cast<uint16_t>(w[e] >> 16);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if (n0 + c + e < p.N) v[e] = __half_as_ushort(wr[e]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) tile[(c + e) * kOmStride + j] = v[e];
+    }
+    named_bar_sync(1, kEpiThreads);
+    for (int pc = et; pc < kOmUnit * (kOmCols / 8); pc += kEpiThreads) {
+      const int r = pc / (kOmCols / 8), c = 8 * (pc % (kOmCols / 8));
+      if (n0 + r < p.N)
+        *reinterpret_cast<uint4*>(wt + int64_t(n0 + r) * kOmCols + c) =
+            *reinterpret_cast<const uint4*>(tile + r * kOmStride + c);
+    }
+    named_bar_sync(1, kEpiThreads);  // the tile is free for the next unit
+  }
+}
+
 template <bool kRaw, bool kPair>
 __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Shared& s, uint32_t tmem_base,
-                             const Sched& sc, uint32_t rank, uint32_t warp, uint32_t lane) {
+                             const Sched& sc, uint32_t rank, uint32_t warp, uint32_t lane, int om) {
   using G = Geo<kPair>;
   const uint32_t q = warp & 3u;             // TMEM lane quarter this warp may access
   const int ab = static_cast<int>(warp - 2) >> 2;  // which 16 rows of the quarter
@@ -496,6 +694,16 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
   // this warp's Y staging tile (1024-byte aligned: the 128-byte swizzle repeats every 8 rows)
   const uint32_t ystage_off = static_cast<uint32_t>(warp - 2) * G::kYBytes;
   const uint32_t ystage = smem_u32(s.ystage) + ystage_off;
+  // the pair leader's dequantized-tile barriers (tensor-core outlier product)
+  const uint32_t deq_leader = kPair ? mapa_shared(smem_u32(s.deq), 0) : smem_u32(s.deq);
+  if (om > 0) {
+    // this CTA's share of the gathered operands, then one release per CTA
+    // (the producers wait for all of them before their first outlier block)
+    gather_outlier_operands(p, s, et);
+    fence_proxy_async_global();
+    named_bar_sync(1, kEpiThreads);
+    if (et == 0) red_add_release_gpu_u32(p.om_sync, 1u);
+  }
 
   uint32_t it = 0;
   for (int tile = sc.first; tile < sc.num_tiles; tile += sc.stride, ++it) {
@@ -513,7 +721,9 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
     if constexpr (!kRaw) {
       named_bar_sync(1, kEpiThreads);  // the previous tile's readers of the staged data are done
       stage_scales(p, s, nb, et, cs_vec);
-      if (passes > 1) {  // many outliers: the first chunk's rows of the first round
+      if (om > 0) {
+        // the outlier product runs on the tensor cores: nothing to stage
+      } else if (passes > 1) {  // many outliers: the first chunk's rows of the first round
         uint4 u[kWo2Pieces];
         load_outlier_chunk(p, nb, 0, 0, min(n_use, kRound), et, w_vec, u);
         store_outlier_chunk(s, et, min(n_use, kRound), u);
@@ -527,7 +737,7 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
         const int r = r0 + g + 8 * h;
         if (r < p.M) rsc[h] = __ldg(p.rs + r) * (1.0f / 16129.0f);
       }
-      if (n_use > 0) load_xo_fragment(p, r0, 0, min(n_use, kSG), lane, afr);
+      if (n_use > 0 && om == 0) load_xo_fragment(p, r0, 0, min(n_use, kSG), lane, afr);
     }
 
     const bool got = wait_or_abort(&s.tfull[b], use, p.status, s.abort);
@@ -635,7 +845,37 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
           d[n][3] = i2f_exact(static_cast<int32_t>(v[4 * n + 3])) * rsc[1] * c2.y;
         }
       };
-      if (passes <= 1) {
+      if (om > 0) {
+        // Tensor-core outlier product: dequantize the tile in place (fp32 over
+        // the int32 accumulator), hand it to the MMA thread, and finish each
+        // chunk once the outlier MMAs have accumulated onto it.
+#pragma unroll 1
+        for (int c = 0; c < BN / 64; ++c) {
+          const uint32_t taddr = tacc + c * 64;
+          uint32_t v[32];
+          tmem_ld_16x256b_x8(taddr, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int n = 0; n < 8; ++n) {  // acc * rs[row] * cs[col] / 127^2, in place
+            const float2 c2 = *reinterpret_cast<const float2*>(s.cs + c * 64 + 8 * n + 2 * t4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              v[4 * n + e] = __float_as_uint(i2f_exact(static_cast<int32_t>(v[4 * n + e])) * rsc[e >> 1] *
+                                             ((e & 1) ? c2.y : c2.x));
+          }
+          tmem_st_16x256b_x8(taddr, v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (kPair) mbar_arrive_cluster(deq_leader + b * 8u);
+        }
+        const bool done = wait_or_abort(&s.ofull[b], use, p.status, s.abort);
+        if (!named_bar_and(2, kEpiThreads, done)) break;
+        tc_fence_after();
+      }
+      if (om > 0 || passes <= 1) {
         // At most 16 outliers: their W rows over the whole tile were staged
         // before the accumulator wait; one k16 step of the 16-bit product.
         // On the CUDA cores: fp32 fused multiply-adds of the exact fp16
@@ -650,9 +890,16 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
           tmem_ld_16x256b_x8(taddr, v);
           tmem_ld_wait();
           float d[8][4];
-          dequant(c, v, d);
+          if (om > 0) {  // dequantized, with the outlier product added by the tensor cores
+#pragma unroll
+            for (int n = 0; n < 8; ++n)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) d[n][e] = __uint_as_float(v[4 * n + e]);
+          } else {
+            dequant(c, v, d);
+          }
           // d += Xo[rows, k] * W[O[k], cols], k < n_use
-          if (!core_product) {
+          if (!core_product && om == 0) {
 #pragma unroll
             for (int np = 0; np < 4; ++np) {
               uint32_t b0, b1, b2, b3;
@@ -805,7 +1052,8 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
 template <bool kRaw, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmY, const GemmArgs p) {
+                   const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmXo,
+                   const __grid_constant__ CUtensorMap tmWo, const GemmArgs p) {
   using G = Geo<kPair>;
   extern __shared__ uint8_t smem_raw[];
   const Shared s = carve<kPair>(smem_raw);
@@ -830,6 +1078,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.tempty[i], G::kTmemEmptyArrivals);
     }
     mbar_init(s.drain, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.deq[i], G::kTmemEmptyArrivals);
+      mbar_init(&s.ofull[i], 1);
+    }
     *s.abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -856,18 +1108,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   // library waits (griddepcontrol.wait) for this grid to complete before it
   // touches memory this grid reads or writes.
   griddep_launch_dependents();
+  const bool om_possible = kPair && !kRaw && p.om_ok;
 
   if (warp == 0) {
-    if (lane == 0) run_producer<kPair>(&tmA, &tmB, s, sc, rank, p.status);
+    if (lane == 0) {
+      if (om_possible) {
+        prefetch_l1(p.n_o);
+        tma_prefetch_desc(&tmXo);
+        tma_prefetch_desc(&tmWo);
+      }
+      run_producer<kPair>(&tmA, &tmB, &tmXo, &tmWo, s, sc, rank, p, om_possible);
+    }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) run_mma<kPair>(s, tmem_base, sc, p.status, p.stall);
+    if (lane == 0 && rank == 0) {
+      if (om_possible) prefetch_l1(p.n_o);
+      run_mma<kPair>(s, tmem_base, sc, p, om_possible);
+    }
   } else {
-    run_epilogue<kRaw, kPair>(p, tmY, s, tmem_base, sc, rank, warp, lane);
+    run_epilogue<kRaw, kPair>(p, tmY, s, tmem_base, sc, rank, warp, lane, om_possible ? outlier_mma_blocks(p) : 0);
   }
 
   tc_fence_before();
   __syncthreads();
   if constexpr (kPair) cluster_sync();  // no CTA leaves while its pair may still signal it
+  if (om_possible && threadIdx.x == 0 && outlier_mma_blocks(p) > 0) {
+    // the last CTA out returns the gather counters to zero for the next call
+    // (every CTA has released its gather share and no producer waits any more)
+    if (atomicAdd(p.om_sync + 1, 1u) == gridDim.x - 1) {
+      p.om_sync[0] = 0u;
+      p.om_sync[1] = 0u;
+    }
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -880,7 +1151,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <bool kRaw, bool kPair>
 cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY,
-                           const GemmArgs& a, int num_sms, cudaStream_t stream, bool pdl) {
+                           const CUtensorMap& tmXo, const CUtensorMap& tmWo, const GemmArgs& a, int num_sms,
+                           cudaStream_t stream, bool pdl) {
   using G = Geo<kPair>;
   static bool attr_set[64] = {};  // per device
   static int max_units[64] = {};  // CTAs (or CTA pairs) that fit at once, per device
@@ -942,7 +1214,7 @@ cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const
   cfg.stream = stream;
   cfg.attrs = n_attr ? attr : nullptr;
   cfg.numAttrs = n_attr;
-  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmY, a);
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmY, tmXo, tmWo, a);
 }
 
 }  // namespace
@@ -950,14 +1222,17 @@ cudaError_t launch_variant(const CUtensorMap& tmA, const CUtensorMap& tmB, const
 bool gemm_uses_pair(int M) { return M > BM; }
 
 cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY,
-                           const GemmArgs& a, bool raw_i32, int num_sms, cudaStream_t stream, bool pdl) {
+                           const CUtensorMap& tmXo, const CUtensorMap& tmWo, const GemmArgs& a, bool raw_i32,
+                           int num_sms, cudaStream_t stream, bool pdl) {
   const bool pair = gemm_uses_pair(a.M);
+  GemmArgs b = a;
+  b.om_ok = a.om_ok && pair && !raw_i32 && a.xo_p != nullptr && a.wo_t != nullptr && a.om_sync != nullptr;
   if (raw_i32) {
-    return pair ? launch_variant<true, true>(tmA, tmB, tmY, a, num_sms, stream, pdl)
-                : launch_variant<true, false>(tmA, tmB, tmY, a, num_sms, stream, pdl);
+    return pair ? launch_variant<true, true>(tmA, tmB, tmY, tmXo, tmWo, b, num_sms, stream, pdl)
+                : launch_variant<true, false>(tmA, tmB, tmY, tmXo, tmWo, b, num_sms, stream, pdl);
   }
-  return pair ? launch_variant<false, true>(tmA, tmB, tmY, a, num_sms, stream, pdl)
-              : launch_variant<false, false>(tmA, tmB, tmY, a, num_sms, stream, pdl);
+  return pair ? launch_variant<false, true>(tmA, tmB, tmY, tmXo, tmWo, b, num_sms, stream, pdl)
+              : launch_variant<false, false>(tmA, tmB, tmY, tmXo, tmWo, b, num_sms, stream, pdl);
 }
 
 // Test hook: this file's wait bound (see ptx.cuh).

@@ -679,13 +679,17 @@ def test_bias_every_kernel(L, M, N, K, how):
     (100, 600, 2048, 250, 3),    # three rounds, single-CTA tiles, direct stores (rows not 16-byte aligned)
     (200, 300, 8192, 24, 0),     # n_o <= K / 256: the product on the CUDA cores, one round
     (64, 257, 32768, 100, 8),    # on the CUDA cores, two rounds, padded ldy
-    (129, 257, 1024, 12, 0),     # 16 or fewer outliers but n_o > K / 256: mma.sync in the one-pass epilogue
+    (100, 257, 1024, 12, 0),     # 16 or fewer outliers but n_o > K / 256: mma.sync in the one-pass epilogue
+    (300, 512, 1024, 129, 0),    # CTA pairs past the tensor-core product's 128 columns: mma.sync rounds
+    (129, 257, 1024, 250, 3),    # the same, three rounds, direct stores
 ])
 def test_many_outliers_epilogue_rounds(L, M, N, K, n_out, ldy_pad):
     """The GEMM epilogue with more than 16 outlier columns: the tile's
     64-column chunks outermost, rounds of up to 96 outlier rows, the bias added
     in the last round, for the fp16 weight and the int8-only weight; the
-    16-bit product by mma.sync (n_o > K / 256) and on the CUDA cores."""
+    16-bit product by mma.sync (n_o > K / 256) and on the CUDA cores.  (CTA
+    pairs with K / 256 < n_o <= 128 take the tensor-core product, tested
+    below.)"""
     rng = np.random.default_rng(M + N + K + n_out)
     X, W, _ = wl.random_small(rng, M, K, N, 0)
     cols = np.sort(rng.choice(K, size=n_out, replace=False))
@@ -702,6 +706,65 @@ def test_many_outliers_epilogue_rounds(L, M, N, K, n_out, ldy_pad):
         assert int(L.workspace_views(ws, M, N, K, K)["n_outlier"].item()) >= n_out
         r = oracle.mixed_matmul(X, W, 6.0, bias=b, int8_weight=not keep)
         y_close(host(Y), r["Y"])
+
+
+OM_CASES = [
+    (129, 257, 520, 40, 0),      # one block of 64 outlier columns, ragged M and N, one tile per CTA pair
+    (257, 520, 4096, 17, 0),     # just past K / 256
+    (300, 512, 1024, 64, 0),     # exactly one block
+    (300, 512, 1024, 65, 8),     # two blocks, padded ldy
+    (300, 512, 1024, 128, 0),    # two full blocks (the most it takes)
+    (513, 1000, 1000, 50, 3),    # direct stores (rows not 16-byte aligned), K not a multiple of 128
+    (2048, 4096, 1024, 40, 0),   # several tiles per CTA pair: each tile's blocks enter the next tile's main loop
+    (1024, 8192, 256, 20, 0),    # main loops shorter than the lag: the blocks follow the next tile's main loop
+    (129, 257, 1024, 12, 0),     # 16 or fewer outliers (one block, mostly zero padding)
+]
+
+
+@pytest.mark.parametrize("M,N,K,n_out,ldy_pad", OM_CASES)
+def test_outlier_product_on_the_tensor_cores(L, M, N, K, n_out, ldy_pad):
+    """CTA-pair GEMMs with K / 256 < n_o <= 128: the epilogue dequantizes the
+    tile in TMEM and kind::f16 MMAs add the outlier product onto it from the
+    gathered Xo and W^T (fp16 weight, int8-only weight, the split entry point),
+    with the bias.  Y against the oracle; repeated calls on one workspace give
+    the same bits and leave the gather counters at zero."""
+    rng = np.random.default_rng(7 * M + N + K + n_out)
+    X, W, _ = wl.random_small(rng, M, K, N, 0)
+    cols = np.sort(rng.choice(K, size=n_out, replace=False))
+    X[:, cols] = (rng.standard_normal((M, n_out), dtype=np.float32) * 20.0 + 10.0).astype(np.float16)
+    b = (rng.standard_normal(N) * 0.5).astype(np.float16)
+    Wd = dev(W)
+    Wq, cs = L.quantize_weight_colwise(Wd)
+    ws = L.empty_workspace(M, N, K, K)
+    for keep in (True, False):
+        r = oracle.mixed_matmul(X, W, 6.0, bias=b, int8_weight=not keep)
+        assert r["O"].size == n_out
+        first = None
+        for rep in range(2):
+            big = torch.full((M, N + ldy_pad), float("nan"), dtype=torch.float16, device="cuda")
+            Y = big[:, :N]
+            L.mixed_matmul(dev(X), Wq, cs, Wd if keep else None, 6.0, Y=Y, ws=ws, bias=dev(b))
+            assert_status_ok(L, ws)
+            assert not host(ws[16:24]).any()  # the gather counters are back at zero
+            y = host(Y)
+            y_close(y, r["Y"])
+            assert np.isnan(host(big[:, N:]).astype(np.float32)).all()  # nothing past column N
+            if first is None:
+                first = y
+            else:
+                assert np.array_equal(y.view(np.uint16), first.view(np.uint16))
+    # the split entry points (activation step, then the GEMM on its outputs),
+    # both on one workspace, twice: the GEMM's gathered operands must leave the
+    # activation step's scratch as the next call needs it
+    ref = oracle.mixed_matmul(X, W, 6.0, bias=b)["Y"]
+    ws2 = L.empty_workspace(M, N, K, K)
+    for rep in range(2):
+        act = L.quantize_act_rowwise_outliers(dev(X), 6.0, ws=ws2)
+        Y2 = host(L.mixed_gemm(act, Wq, cs, Wd, ws=ws2, bias=dev(b)))
+        assert_status_ok(L, ws2)
+        assert int(host(act["n_outlier"])[0]) == n_out
+        assert not host(ws2[16:24]).any()
+        y_close(Y2, ref)
 
 
 @pytest.mark.parametrize("keep", [False, True])
