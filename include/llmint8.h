@@ -183,12 +183,12 @@ llmint8_status llmint8_quantize_act_rowwise_outliers(const void* X, int64_t M, i
  * receives the same Xq, row scales, O, n_o and Xo.
  * Where the 16-bit outlier product runs in the prefill GEMM's epilogue: for
  * n_o <= K / 256 on the CUDA cores (fp32 FMAs of the exact fp16 products);
- * with CTA-pair tiles (M > 128) and K / 256 < n_o <= 128 on the 5th-generation
- * tensor cores: the epilogue dequantizes the tile in TMEM, the MMA issuer
- * accumulates Xo . W[O, :] onto it (tcgen05.mma kind::f16, fp32) from
- * operands the kernel gathers into the workspace (Xo and W[O, :]^T, zero
- * padded to 128 columns), and the epilogue rounds the result; otherwise by
- * warp-level mma.sync.  All three accumulate the exact fp16 products in fp32.
+ * with K / 256 < n_o <= 256 on the 5th-generation tensor cores: the epilogue
+ * dequantizes the tile in TMEM, the MMA issuer accumulates Xo . W[O, :] onto
+ * it (tcgen05.mma kind::f16, fp32) from operands the kernel gathers into the
+ * workspace (Xo and W[O, :]^T, zero padded to whole 64-column blocks), and
+ * the epilogue rounds the result; past 256 outliers by warp-level mma.sync.
+ * All three accumulate the exact fp16 products in fp32.
  * llmint8_mixed_matmul_path names the kernels of a call.  No host
  * synchronisation. */
 llmint8_status llmint8_mixed_matmul(const void* X, int64_t M, int64_t K, int64_t ldx, const int8_t* Wq,
@@ -243,7 +243,7 @@ const char* llmint8_mixed_matmul_path(int64_t M, int64_t N, int64_t K, int64_t l
  *                    splits K across CTAs when ws also holds its reduction
  *                    scratch (a workspace of llmint8_workspace_size(M, N, K,
  *                    outlier_cap) bytes, zero-filled once, does); the scratch is
- *                    the end of ws and is left at zero.  For M > 128 such a
+ *                    the end of ws and is left at zero.  For M > 32 such a
  *                    workspace also holds the operands of the tensor-core
  *                    outlier product (see llmint8_mixed_matmul), at the same
  *                    place as for llmint8_mixed_matmul: past the activation

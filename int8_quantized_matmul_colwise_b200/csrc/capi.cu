@@ -136,23 +136,28 @@ bool encode_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_
   return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, cols, rows, ld, kGemmBK, box_rows);
 }
 
-// fp16 operand of the tensor-core outlier product: [rows, 128] contiguous,
-// read in boxes of 128 rows x 64 columns (128 bytes) with the 128-byte swizzle.
-bool encode_outlier_map(CUtensorMap* map, const void* base, int64_t rows) {
-  return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, kOutlierMmaMax, rows, 2 * kOutlierMmaMax, 64, 128);
+// fp16 operand of the tensor-core outlier product: [rows, kOutlierMmaMax]
+// contiguous, read in boxes of box_rows x 64 columns (128 bytes) with the
+// 128-byte swizzle.
+bool encode_outlier_map(CUtensorMap* map, const void* base, int64_t rows, uint32_t box_rows) {
+  return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, kOutlierMmaMax, rows, 2 * kOutlierMmaMax, 64,
+                   box_rows);
 }
 
-// The tensor-core outlier product of a CTA-pair GEMM: its two counters sit in
+// The tensor-core outlier product of the prefill GEMM: its two counters sit in
 // the workspace header (zero between calls), its gathered operands (Xo
-// [M, 128] then W^T [N, 128], fp16) at `data`.  Leaves a.om_ok false (the
-// epilogue computes the product) when the maps cannot be made.
+// [M, kOutlierMmaMax] then W^T [N, kOutlierMmaMax], fp16) at `data`.  Leaves
+// a.om_ok false (the epilogue computes the product) when the maps cannot be
+// made.
 void prepare_outlier_mma(GemmArgs& a, CUtensorMap* tmXo, CUtensorMap* tmWo, void* ws, uint8_t* data) {
   std::memset(tmXo, 0, sizeof(*tmXo));
   std::memset(tmWo, 0, sizeof(*tmWo));
   a.om_ok = false;
-  if (!gemm_uses_pair(a.M) || data == nullptr) return;
+  if (data == nullptr) return;
   uint8_t* wo_t = data + size_t(a.M) * 2 * kOutlierMmaMax;
-  if (!encode_outlier_map(tmXo, data, a.M) || !encode_outlier_map(tmWo, wo_t, a.N)) return;
+  if (!encode_outlier_map(tmXo, data, a.M, kGemmBM) ||
+      !encode_outlier_map(tmWo, wo_t, a.N, gemm_b_box_rows(a.M)))
+    return;
   a.xo_p = data;
   a.wo_t = wo_t;
   a.om_sync = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + 16);
@@ -182,7 +187,7 @@ bool prepare_output(CUtensorMap* map, void* Y, int64_t M, int64_t N, int64_t ldy
 // xq              i8  [M, ldq]
 // xo              f16 [M, ldo]
 // decode          (M <= kDecodeMaxM) split-K partial sums + tile counters, zero between calls
-// outlier operands (CTA-pair GEMMs) fp16 Xo [M, 128] + W^T [N, 128] of the tensor-core outlier product
+// outlier operands (M > 32) fp16 Xo [M, 256] + W^T [N, 256] of the tensor-core outlier product
 bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t* colmax, size_t* bitmask,
                  int64_t N = 0, size_t* decode = nullptr, size_t* outlier_ops = nullptr) {
   if (M < 1 || K < 1 || K > kMaxK || cap < 0 || cap > K) return false;
@@ -208,7 +213,7 @@ bool make_layout(int64_t M, int64_t K, int64_t cap, llmint8_ws_layout* L, size_t
   off = align_up(off + 2 * size_t(M) * size_t(L->ldo), 256);
   if (decode) *decode = off;
   if (M <= kDecodeMaxM && N > 0) off += decode_scratch_bytes(static_cast<int>(M), static_cast<int>(N));
-  if (N > 0 && gemm_uses_pair(static_cast<int>(M))) {
+  if (N > 0 && M > kDecodeMaxM) {
     off = align_up(off, 256);
     if (outlier_ops) *outlier_ops = off;
     off += outlier_mma_bytes(M, N);

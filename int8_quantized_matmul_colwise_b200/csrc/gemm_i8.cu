@@ -62,18 +62,18 @@ constexpr int kWoStride = BN + 8;  // halves per staged row: 528 bytes, conflict
 // run on it in registers.
 constexpr int kRound = 96;
 constexpr int kWo2Stride = 72;  // halves per staged row of a chunk: 144 bytes, conflict-free ldmatrix
-// Many outliers on CTA pairs (K/256 < n_o <= kOutlierMmaMax): the outlier
-// product runs on the tensor cores.  The epilogue dequantizes the tile in
-// TMEM (int32 -> fp32 in place) and the MMA thread accumulates Xo * W[O, :]
-// onto it with kind::f16 MMAs (fp16 operands, fp32 accumulation).  Each block
-// of 64 outlier columns is one ring stage (128 rows of Xo and 128 rows of the
-// gathered W^T, 128 bytes each, per CTA), and a tile's blocks enter the ring
+// Many outliers (K/256 < n_o <= kOutlierMmaMax): the outlier product runs on
+// the tensor cores.  The epilogue dequantizes the tile in TMEM (int32 -> fp32
+// in place) and the MMA thread accumulates Xo * W[O, :] onto it with kind::f16
+// MMAs (fp16 operands, fp32 accumulation).  Each block of 64 outlier columns
+// is one ring stage with the int8 stage's geometry (the tile's rows of Xo and
+// of the gathered W^T, 128 bytes each), and a tile's blocks enter the ring
 // kOmLag blocks into the next tile's main loop, by which time the epilogue has
 // the tile dequantized.
 constexpr int kOmLag = 4;
-constexpr int kOmCols = kOutlierMmaMax;   // fp16 columns of the gathered operands
-constexpr int kOmUnit = 32;               // rows of W^T or Xo per gather unit
-constexpr int kOmStride = kOmCols + 8;    // halves per row of the transposing tile: 272 bytes
+constexpr int kOmCols = kOutlierMmaMax;   // fp16 columns (row stride) of the gathered operands
+constexpr int kOmUnit = 16;               // rows of W^T or Xo per gather unit
+constexpr int kOmStride = kOmCols + 8;    // halves per row of the transposing tile: 528 bytes
 
 template <bool kPair>
 struct Geo {
@@ -324,33 +324,37 @@ __device__ void run_mma(const Shared& s, uint32_t tmem_base, const Sched& sc, co
   // both CTAs' epilogues have dequantized it in TMEM, fp16 MMAs accumulate
   // onto it, and the commit tells both epilogues that it is done.
   auto outliers = [&](uint32_t pb, uint32_t puse) -> bool {
-    if constexpr (kPair) {
-      constexpr uint32_t idesc_o = idesc_f16(G::kTileM, BN);
-      if (!wait_or_abort(&s.deq[pb], puse, status, s.abort)) return false;
+    constexpr uint32_t idesc_o = idesc_f16(G::kTileM, BN);
+    if (!wait_or_abort(&s.deq[pb], puse, status, s.abort)) return false;
+    tc_fence_after();
+    const uint32_t d = tmem_base + pb * kAccCols;
+    for (int ob = 0; ob < om; ++ob) {
+      if (!wait_or_abort(&s.full[stage], phase, status, s.abort)) return false;
       tc_fence_after();
-      const uint32_t d = tmem_base + pb * kAccCols;
-      for (int ob = 0; ob < om; ++ob) {
-        if (!wait_or_abort(&s.full[stage], phase, status, s.abort)) return false;
-        tc_fence_after();
-        const uint64_t da = smem_desc_k_sw128(smem_u32(s.a + stage * G::kBytesA));
-        const uint64_t db = smem_desc_k_sw128(smem_u32(s.b + stage * G::kBytesB));
+      const uint64_t da = smem_desc_k_sw128(smem_u32(s.a + stage * G::kBytesA));
+      const uint64_t db = smem_desc_k_sw128(smem_u32(s.b + stage * G::kBytesB));
 #pragma unroll
-        for (int kk = 0; kk < BK / 32; ++kk)  // K = 16 fp16 = 32 bytes per MMA, as for int8
+      for (int kk = 0; kk < BK / 32; ++kk) {  // K = 16 fp16 = 32 bytes per MMA, as for int8
+        if constexpr (kPair)
           mma_f16_pair(d, da + 2u * kk, db + 2u * kk, idesc_o, 1u);
-        any = true;
-        mma_commit_pair(&s.empty[stage], 0x3);
-        if (++stage == G::kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        else
+          mma_f16(d, da + 2u * kk, db + 2u * kk, idesc_o, 1u);
       }
-      mma_commit_pair(&s.ofull[pb], 0x3);
-      return true;
-    } else {
-      (void)pb;
-      (void)puse;
-      return false;
+      any = true;
+      if constexpr (kPair)
+        mma_commit_pair(&s.empty[stage], 0x3);
+      else
+        mma_commit(&s.empty[stage]);
+      if (++stage == G::kStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
     }
+    if constexpr (kPair)
+      mma_commit_pair(&s.ofull[pb], 0x3);
+    else
+      mma_commit(&s.ofull[pb]);
+    return true;
   };
   // (the stall test hook first waits on the drain barrier, which nothing has
   // arrived on yet: the wait runs out before any MMA is issued and the CTA
@@ -594,12 +598,14 @@ __device__ __forceinline__ void load_xo_fragment(const GemmArgs& p, int r0, int 
 }
 
 // This CTA's share of the operands of the tensor-core outlier product, by all
-// epilogue threads before the first tile: W^T [N, 128] (row j of column n is
+// epilogue threads before the first tile: W^T [N, 256] (row j of column n is
 // W[O[j], n], or the row recovered from Wq without an fp16 weight) and Xo
-// [M, 128], zero past n_o, in units of kOmUnit rows.  W rows are read along N
-// and transposed through shared memory so that both sides are coalesced.
-__device__ void gather_outlier_operands(const GemmArgs& p, const Shared& s, int et) {
+// [M, 256], zero from n_o up to the 64-column blocks the MMAs read (columns
+// past them are never read), in units of kOmUnit rows.  W rows are read along
+// N and transposed through shared memory so that both sides are coalesced.
+__device__ void gather_outlier_operands(const GemmArgs& p, const Shared& s, int et, int om) {
   const int n_o = *p.n_o;
+  const int ncol = 64 * om;  // columns written per row
   const int units_n = (p.N + kOmUnit - 1) / kOmUnit;
   const int units = units_n + (p.M + kOmUnit - 1) / kOmUnit;
   const __half* W = static_cast<const __half*>(p.W);
@@ -613,7 +619,7 @@ __device__ void gather_outlier_operands(const GemmArgs& p, const Shared& s, int 
       const int m0 = (u - units_n) * kOmUnit;
       for (int i = et; i < kOmUnit * kOmCols; i += kEpiThreads) {
         const int m = m0 + i / kOmCols, j = i % kOmCols;
-        if (m < p.M) xp[int64_t(m) * kOmCols + j] = j < n_o ? __half_as_ushort(Xo[int64_t(m) * p.ldo + j]) : 0;
+        if (m < p.M && j < ncol) xp[int64_t(m) * kOmCols + j] = j < n_o ? __half_as_ushort(Xo[int64_t(m) * p.ldo + j]) : 0;
       }
       continue;
     }
@@ -621,7 +627,7 @@ __device__ void gather_outlier_operands(const GemmArgs& p, const Shared& s, int 
     if (W == nullptr) {  // no fp16 weight kept: the rows recovered from Wq
       for (int i = et; i < kOmUnit * kOmCols; i += kEpiThreads) {
         const int n = n0 + i / kOmCols, j = i % kOmCols;
-        if (n < p.N)
+        if (n < p.N && j < ncol)
           wt[int64_t(n) * kOmCols + j] =
               j < n_o ? dequant_weight_bits(p.Wq[int64_t(n) * p.ldk + __ldg(p.O + j)], __ldg(p.cs + n)) : 0;
       }
@@ -630,6 +636,7 @@ __device__ void gather_outlier_operands(const GemmArgs& p, const Shared& s, int 
     // pieces of 8 columns of a W row into the transposing tile
     for (int pc = et; pc < kOmCols * (kOmUnit / 8); pc += kEpiThreads) {
       const int j = pc / (kOmUnit / 8), c = 8 * (pc % (kOmUnit / 8));
+      if (j >= ncol) continue;
       uint16_t v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       if (j < n_o) {
         const __half* wr = W + int64_t(__ldg(p.O + j)) * p.ldw + n0 + c;
@@ -653,7 +660,7 @@ __device__ void gather_outlier_operands(const GemmArgs& p, const Shared& s, int 
     named_bar_sync(1, kEpiThreads);
     for (int pc = et; pc < kOmUnit * (kOmCols / 8); pc += kEpiThreads) {
       const int r = pc / (kOmCols / 8), c = 8 * (pc % (kOmCols / 8));
-      if (n0 + r < p.N)
+      if (n0 + r < p.N && c < ncol)
         *reinterpret_cast<uint4*>(wt + int64_t(n0 + r) * kOmCols + c) =
             *reinterpret_cast<const uint4*>(tile + r * kOmStride + c);
     }
@@ -694,12 +701,12 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
   // this warp's Y staging tile (1024-byte aligned: the 128-byte swizzle repeats every 8 rows)
   const uint32_t ystage_off = static_cast<uint32_t>(warp - 2) * G::kYBytes;
   const uint32_t ystage = smem_u32(s.ystage) + ystage_off;
-  // the pair leader's dequantized-tile barriers (tensor-core outlier product)
+  // the dequantized-tile barriers (tensor-core outlier product; the pair leader's for CTA pairs)
   const uint32_t deq_leader = kPair ? mapa_shared(smem_u32(s.deq), 0) : smem_u32(s.deq);
   if (om > 0) {
     // this CTA's share of the gathered operands, then one release per CTA
     // (the producers wait for all of them before their first outlier block)
-    gather_outlier_operands(p, s, et);
+    gather_outlier_operands(p, s, et, om);
     fence_proxy_async_global();
     named_bar_sync(1, kEpiThreads);
     if (et == 0) red_add_release_gpu_u32(p.om_sync, 1u);
@@ -869,7 +876,10 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          if constexpr (kPair) mbar_arrive_cluster(deq_leader + b * 8u);
+          if constexpr (kPair)
+            mbar_arrive_cluster(deq_leader + b * 8u);
+          else
+            mbar_arrive(&s.deq[b]);
         }
         const bool done = wait_or_abort(&s.ofull[b], use, p.status, s.abort);
         if (!named_bar_and(2, kEpiThreads, done)) break;
@@ -1108,7 +1118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // library waits (griddepcontrol.wait) for this grid to complete before it
   // touches memory this grid reads or writes.
   griddep_launch_dependents();
-  const bool om_possible = kPair && !kRaw && p.om_ok;
+  const bool om_possible = !kRaw && p.om_ok;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -1226,7 +1236,7 @@ cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const
                            int num_sms, cudaStream_t stream, bool pdl) {
   const bool pair = gemm_uses_pair(a.M);
   GemmArgs b = a;
-  b.om_ok = a.om_ok && pair && !raw_i32 && a.xo_p != nullptr && a.wo_t != nullptr && a.om_sync != nullptr;
+  b.om_ok = a.om_ok && !raw_i32 && a.xo_p != nullptr && a.wo_t != nullptr && a.om_sync != nullptr;
   if (raw_i32) {
     return pair ? launch_variant<true, true>(tmA, tmB, tmY, tmXo, tmWo, b, num_sms, stream, pdl)
                 : launch_variant<true, false>(tmA, tmB, tmY, tmXo, tmWo, b, num_sms, stream, pdl);

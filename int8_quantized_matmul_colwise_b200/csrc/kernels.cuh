@@ -77,20 +77,21 @@ struct GemmArgs {
   uint32_t* status;
   bool y_tma;         // Y is written through the tmY tensor map (16-byte aligned rows)
   uint32_t stall;     // test hook: stall mask (ptx.cuh), 0 in normal use
-  // The outlier product on the tensor cores (CTA pairs, K/256 < n_o <=
-  // kOutlierMmaMax): the kernel gathers Xo and the outlier rows of W, zero
-  // padded to kOutlierMmaMax columns, into xo_p [M, 128] and wo_t [N, 128]
-  // (fp16, K-major, read back through the tmXo / tmWo tensor maps); om_sync
-  // holds two counters that are zero between calls.  om_ok false: never.
+  // The outlier product on the tensor cores (K/256 < n_o <= kOutlierMmaMax):
+  // the kernel gathers Xo and the outlier rows of W, zero padded to a
+  // multiple of 64 columns, into xo_p [M, kOutlierMmaMax] and wo_t
+  // [N, kOutlierMmaMax] (fp16, K-major, read back through the tmXo / tmWo
+  // tensor maps); om_sync holds two counters that are zero between calls.
+  // om_ok false: never.
   bool om_ok;
   void* xo_p;
   void* wo_t;
   uint32_t* om_sync;
 };
 
-// Outlier columns the tensor-core outlier product takes at most (two blocks of
-// 64 fp16 columns), and the workspace bytes it needs for M x N.
-constexpr int kOutlierMmaMax = 128;
+// Outlier columns the tensor-core outlier product takes at most (four blocks
+// of 64 fp16 columns), and the workspace bytes it needs for M x N.
+constexpr int kOutlierMmaMax = 256;
 inline size_t outlier_mma_bytes(int64_t M, int64_t N) {
   return size_t(M) * 2 * kOutlierMmaMax + size_t(N) * 2 * kOutlierMmaMax;
 }
@@ -103,9 +104,10 @@ bool gemm_uses_pair(int M);
 // int8 in boxes of gemm_b_box_rows(M) rows, 128 bytes along K, 128-byte
 // swizzle.  raw_i32 selects the accumulator-dump epilogue.
 // tmY: Y [M rows, N cols] fp16 in boxes of 16 rows x 64 columns, 128-byte
-// swizzle (used when a.y_tma).  tmXo / tmWo: a.xo_p [M rows, 128 cols] and
-// a.wo_t [N rows, 128 cols] fp16 in boxes of 128 rows x 64 columns, 128-byte
-// swizzle (used when a.om_ok).
+// swizzle (used when a.y_tma).  tmXo / tmWo: a.xo_p [M rows, kOutlierMmaMax
+// cols] and a.wo_t [N rows, kOutlierMmaMax cols] fp16 in boxes of 64 columns
+// and 128 (Xo) / gemm_b_box_rows(M) (W) rows, 128-byte swizzle (used when
+// a.om_ok).
 cudaError_t launch_gemm_i8(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY,
                            const CUtensorMap& tmXo, const CUtensorMap& tmWo, const GemmArgs& a, bool raw_i32,
                            int num_sms, cudaStream_t stream, bool pdl);

@@ -680,16 +680,17 @@ def test_bias_every_kernel(L, M, N, K, how):
     (200, 300, 8192, 24, 0),     # n_o <= K / 256: the product on the CUDA cores, one round
     (64, 257, 32768, 100, 8),    # on the CUDA cores, two rounds, padded ldy
     (100, 257, 1024, 12, 0),     # 16 or fewer outliers but n_o > K / 256: mma.sync in the one-pass epilogue
-    (300, 512, 1024, 129, 0),    # CTA pairs past the tensor-core product's 128 columns: mma.sync rounds
-    (129, 257, 1024, 250, 3),    # the same, three rounds, direct stores
+    (300, 512, 1024, 260, 0),    # past the tensor-core product's 256 columns: mma.sync rounds on every path
 ])
 def test_many_outliers_epilogue_rounds(L, M, N, K, n_out, ldy_pad):
     """The GEMM epilogue with more than 16 outlier columns: the tile's
     64-column chunks outermost, rounds of up to 96 outlier rows, the bias added
     in the last round, for the fp16 weight and the int8-only weight; the
-    16-bit product by mma.sync (n_o > K / 256) and on the CUDA cores.  (CTA
-    pairs with K / 256 < n_o <= 128 take the tensor-core product, tested
-    below.)"""
+    16-bit product by mma.sync (n_o > K / 256) and on the CUDA cores.  With
+    K / 256 < n_o <= 256 the whole path takes the tensor-core product (tested
+    below), so each case also runs the split GEMM entry point with a
+    256-byte workspace, which has no room for that product's operands and
+    leaves it to the epilogue."""
     rng = np.random.default_rng(M + N + K + n_out)
     X, W, _ = wl.random_small(rng, M, K, N, 0)
     cols = np.sort(rng.choice(K, size=n_out, replace=False))
@@ -706,6 +707,14 @@ def test_many_outliers_epilogue_rounds(L, M, N, K, n_out, ldy_pad):
         assert int(L.workspace_views(ws, M, N, K, K)["n_outlier"].item()) >= n_out
         r = oracle.mixed_matmul(X, W, 6.0, bias=b, int8_weight=not keep)
         y_close(host(Y), r["Y"])
+        # the epilogue's own product: the split entry point without room for the gathered operands
+        act = L.quantize_act_rowwise_outliers(dev(X), 6.0)
+        small = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        big2 = torch.zeros((M, N + ldy_pad), dtype=torch.float16, device="cuda")
+        Y2 = big2[:, :N]
+        L.mixed_gemm(act, Wq, cs, Wd if keep else None, Y=Y2, ws=small, bias=dev(b))
+        assert_status_ok(L, small)
+        y_close(host(Y2), r["Y"])
 
 
 OM_CASES = [
@@ -718,15 +727,21 @@ OM_CASES = [
     (2048, 4096, 1024, 40, 0),   # several tiles per CTA pair: each tile's blocks enter the next tile's main loop
     (1024, 8192, 256, 20, 0),    # main loops shorter than the lag: the blocks follow the next tile's main loop
     (129, 257, 1024, 12, 0),     # 16 or fewer outliers (one block, mostly zero padding)
+    (300, 512, 1024, 200, 0),    # four blocks
+    (300, 512, 1024, 256, 0),    # four full blocks (the most it takes)
+    (129, 257, 1024, 250, 3),    # four blocks, direct stores
+    (100, 600, 2048, 40, 3),     # single-CTA tiles (M <= 128), direct stores
+    (64, 1000, 1000, 20, 0),     # single-CTA tiles, ragged N and K
+    (128, 4096, 512, 70, 0),     # single-CTA tiles, several tiles per CTA, main loops shorter than the lag
 ]
 
 
 @pytest.mark.parametrize("M,N,K,n_out,ldy_pad", OM_CASES)
 def test_outlier_product_on_the_tensor_cores(L, M, N, K, n_out, ldy_pad):
-    """CTA-pair GEMMs with K / 256 < n_o <= 128: the epilogue dequantizes the
-    tile in TMEM and kind::f16 MMAs add the outlier product onto it from the
-    gathered Xo and W^T (fp16 weight, int8-only weight, the split entry point),
-    with the bias.  Y against the oracle; repeated calls on one workspace give
+    """Prefill GEMMs (CTA pairs and single CTAs) with K / 256 < n_o <= 256:
+    the epilogue dequantizes the tile in TMEM and kind::f16 MMAs add the
+    outlier product onto it from the gathered Xo and W^T (fp16 weight,
+    int8-only weight, the split entry point), with the bias.  Y against the oracle; repeated calls on one workspace give
     the same bits and leave the gather counters at zero."""
     rng = np.random.default_rng(7 * M + N + K + n_out)
     X, W, _ = wl.random_small(rng, M, K, N, 0)
