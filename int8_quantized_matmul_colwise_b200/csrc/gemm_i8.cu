@@ -68,9 +68,13 @@ constexpr int kWo2Stride = 72;  // halves per staged row of a chunk: 144 bytes, 
 // MMAs (fp16 operands, fp32 accumulation).  Each block of 64 outlier columns
 // is one ring stage with the int8 stage's geometry (the tile's rows of Xo and
 // of the gathered W^T, 128 bytes each), and a tile's blocks enter the ring
-// kOmLag blocks into the next tile's main loop, by which time the epilogue has
-// the tile dequantized.
-constexpr int kOmLag = 4;
+// om_insert() blocks into the next tile's main loop (kOmLag, or half of a
+// shorter one), by which time the epilogue has the tile dequantized and still
+// has half a main loop to finish it before its accumulator is needed again.
+constexpr int kOmLag = 8;
+__host__ __device__ constexpr int om_insert(int num_k) {
+  return (num_k + 1) / 2 < kOmLag ? (num_k + 1) / 2 : kOmLag;
+}
 constexpr int kOmCols = kOutlierMmaMax;   // fp16 columns (row stride) of the gathered operands
 constexpr int kOmUnit = 16;               // rows of W^T or Xo per gather unit
 constexpr int kOmStride = kOmCols + 8;    // halves per row of the transposing tile: 528 bytes
@@ -282,7 +286,7 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
   bool ok = true;
   bool prev = false;
   int pya = 0, pyb = 0;  // the previous tile's rows
-  const int ins = sc.num_k < kOmLag ? sc.num_k : kOmLag;
+  const int ins = om_insert(sc.num_k);
   for (int tile = sc.first; tile < sc.num_tiles && ok; tile += sc.stride) {
     int mb, nb;
     tile_coords(tile, sc, mb, nb);
@@ -360,7 +364,7 @@ __device__ void run_mma(const Shared& s, uint32_t tmem_base, const Sched& sc, co
   // arrived on yet: the wait runs out before any MMA is issued and the CTA
   // takes the abort path)
   if ((stall & kStallGemmOperands) && !wait_or_abort(s.drain, 0, status, s.abort)) ok = false;
-  const int ins = sc.num_k < kOmLag ? sc.num_k : kOmLag;
+  const int ins = om_insert(sc.num_k);
   for (int tile = sc.first; tile < sc.num_tiles && ok; tile += sc.stride, ++it) {
     const uint32_t b = it & 1u;
     const uint32_t use = (it >> 1) & 1u;

@@ -725,14 +725,15 @@ OM_CASES = [
     (300, 512, 1024, 128, 0),    # two full blocks (the most it takes)
     (513, 1000, 1000, 50, 3),    # direct stores (rows not 16-byte aligned), K not a multiple of 128
     (2048, 4096, 1024, 40, 0),   # several tiles per CTA pair: each tile's blocks enter the next tile's main loop
-    (1024, 8192, 256, 20, 0),    # main loops shorter than the lag: the blocks follow the next tile's main loop
+    (1024, 8192, 256, 20, 0),    # short main loops (two blocks): the outlier blocks after the next tile's first
+    (4096, 4096, 128, 5, 0),     # one-block main loops: the outlier blocks follow the next tile's whole main loop
     (129, 257, 1024, 12, 0),     # 16 or fewer outliers (one block, mostly zero padding)
     (300, 512, 1024, 200, 0),    # four blocks
     (300, 512, 1024, 256, 0),    # four full blocks (the most it takes)
     (129, 257, 1024, 250, 3),    # four blocks, direct stores
     (100, 600, 2048, 40, 3),     # single-CTA tiles (M <= 128), direct stores
     (64, 1000, 1000, 20, 0),     # single-CTA tiles, ragged N and K
-    (128, 4096, 512, 70, 0),     # single-CTA tiles, several tiles per CTA, main loops shorter than the lag
+    (128, 4096, 512, 70, 0),     # single-CTA tiles, several tiles per CTA, short main loops
 ]
 
 
