@@ -75,8 +75,9 @@ const char* llmint8_status_string(llmint8_status s);
  * first use (llmint8_workspace_init or any memset); the library leaves the
  * parts that must start at zero back at zero.  It holds the status word, the
  * column maxima, the outlier set, the row scales, Xq, the gathered outlier
- * columns of X and, for M <= 32, the split-K sums of the decode GEMM.
- * Returns 0 for invalid sizes. */
+ * columns of X and, for M <= 32, the split-K sums of the decode GEMM, or, for
+ * M > 32, the operands of the tensor-core outlier product (fp16 [M, 256] and
+ * [N, 256], 512 * (M + N) bytes).  Returns 0 for invalid sizes. */
 size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K, int64_t outlier_cap);
 
 /* Zero-fill `ws` (cudaMemsetAsync on `stream`). */
