@@ -78,6 +78,11 @@ def test_workspace_layout_and_size(lib):
     assert regions[-1][0] + regions[-1][1] <= L.total
     L2 = capi.llmint8_workspace_layout(3, 33, 24, 1)
     assert L2.ldq == 32 and L2.ldo == 8
+    # prefill calls (M > 32) end with the tensor-core outlier product's operands,
+    # fp16 [M, 256] and [N, 256], past Xo
+    assert L.total >= L.xo + 2 * M * L.ldo + 512 * (M + N)
+    L3 = capi.llmint8_workspace_layout(33, 1000, 1000, 1000)
+    assert L3.total >= L3.xo + 2 * 33 * L3.ldo + 512 * (33 + 1000)
 
 
 @pytest.mark.parametrize("M,N,K,cap", [(0, 1, 1, 1), (1, 0, 1, 1), (1, 1, 0, 1), (1, 1, 133144, 1),
