@@ -792,7 +792,12 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
             d[n][3] += b2.y;
           }
         }
-        if (last && p.y_tma) {
+        if (last) {
+          // fp16 Y through the warp's 16 x 64 staging tile (128-byte swizzle):
+          // a TMA store when Y's rows are 16-byte aligned; otherwise one row
+          // at a time, each store instruction covering 64 consecutive columns
+          // of a row (stores from the fragment layout would scatter over
+          // eight rows each)
           uint32_t lo[8], hi[8];
 #pragma unroll
           for (int n = 0; n < 8; ++n) {
@@ -802,7 +807,8 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
             lo[n] = *reinterpret_cast<const uint32_t*>(&a);
             hi[n] = *reinterpret_cast<const uint32_t*>(&bb);
           }
-          if (lane == 0) bulk_wait_read_all();  // the previous store has left the staging tile
+          // the previous store (TMA) or row reads (direct) have left the staging tile
+          if (p.y_tma && lane == 0) bulk_wait_read_all();
           __syncwarp();
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -811,29 +817,28 @@ __device__ void run_epilogue(const GemmArgs& p, const CUtensorMap& tmY, const Sh
             stmatrix_x4(ystage + rr * 128u + ((nn ^ (rr & 7)) << 4), lo[2 * i], hi[2 * i], lo[2 * i + 1],
                         hi[2 * i + 1]);
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmY, s.ystage + ystage_off, nb * BN + c * 64, r0);
-            bulk_commit();
-          }
-        } else if (last) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int r = r0 + g + 8 * h;
-            if (r < p.M) {
+          if (p.y_tma) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, s.ystage + ystage_off, nb * BN + c * 64, r0);
+              bulk_commit();
+            }
+          } else {
+            __syncwarp();
+            const int col = nb * BN + c * 64 + 2 * static_cast<int>(lane);  // this lane's two columns
+#pragma unroll 1
+            for (int rr = 0; rr < 16; ++rr) {
+              const int r = r0 + rr;
+              if (r >= p.M) break;
+              const uint32_t w = ld_shared_u32(ystage + static_cast<uint32_t>(rr) * 128u +
+                                               (((lane >> 2) ^ static_cast<uint32_t>(rr & 7)) << 4) + (lane & 3) * 4u);
               __half* yr = Y + static_cast<int64_t>(r) * p.ldy;
-#pragma unroll
-              for (int n = 0; n < 8; ++n) {
-                const int col = nb * BN + c * 64 + 8 * n + 2 * t4;
-                float y0 = d[n][2 * h], y1 = d[n][2 * h + 1];
-                if (overflow) y0 = y1 = __int_as_float(0x7fc00000);
-                if (y_pair && col + 1 < p.N) {
-                  *reinterpret_cast<__half2*>(yr + col) = __floats2half2_rn(y0, y1);
-                } else {
-                  if (col < p.N) yr[col] = __float2half_rn(y0);
-                  if (col + 1 < p.N) yr[col + 1] = __float2half_rn(y1);
-                }
+              if (y_pair && col + 1 < p.N) {
+                *reinterpret_cast<uint32_t*>(yr + col) = w;
+              } else {
+                if (col < p.N) yr[col] = __ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu));
+                if (col + 1 < p.N) yr[col + 1] = __ushort_as_half(static_cast<unsigned short>(w >> 16));
               }
             }
           }
