@@ -21,6 +21,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import threading
@@ -482,8 +483,15 @@ def measure_supplementary(L, torch, dev, peaks, clocks, leg_s, only=""):
 
 # ------------------------------------------------------------------ our arm
 def source_digest(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """First 16 hex digits of the sha256 of a C++ source with its comments
+    removed and its white space collapsed: the code the counters were taken
+    on, whatever its comments say."""
+    with open(path) as f:
+        src = f.read()
+    src = re.sub(r"//[^\n]*", "", src)
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"\s+", " ", src).strip()
+    return hashlib.sha256(src.encode()).hexdigest()[:16]
 
 
 def recorded_traffic(wl_name):
@@ -496,7 +504,7 @@ def recorded_traffic(wl_name):
         return None
     src = os.path.join(ROOT, "int8_quantized_matmul_colwise_b200", "csrc", "gemm_i8.cu")
     ent = d.get(wl_name)
-    if not ent or ent.get("gemm_source_sha256_16") != source_digest(src):
+    if not ent or ent.get("gemm_code_sha256_16") != source_digest(src):
         return None
     return ent.get("dram_bytes_per_launch")
 

@@ -28,11 +28,17 @@
 //   warps 2-9   epilogue, two warps per TMEM lane quarter, 16 rows each:
 //               tcgen05.ld in the mma.m16n8 fragment layout, dequantize with
 //               rs[i] * cs[j] / 127^2, add the 16-bit outlier product
-//               sum_t Xo[i,t] * W[O[t], j] with warp-level tensor-core MMAs
-//               (fp16 operands, fp32 accumulation) straight into that
-//               fragment, round once to fp16 and store.  The tile's W rows,
+//               sum_t Xo[i,t] * W[O[t], j] (fp16 operands, fp32 accumulation;
+//               see below for where it runs), round once to fp16 and store
+//               through a shared-memory staging tile.  The tile's W rows,
 //               column scales, row scales and Xo fragments are fetched before
 //               the accumulator wait.
+// The outlier product: n_o <= K/256 on the CUDA cores in the epilogue;
+// K/256 < n_o <= 256 on the tensor cores (the epilogue writes the dequantized
+// tile back to TMEM as fp32, the MMA thread accumulates kind::f16 MMAs onto it
+// from operands the epilogue warps gather into the workspace before their
+// first tile, and the epilogue rounds the sum); past that, or without room in
+// the workspace, warp-level mma.sync in the epilogue.
 // Every mbarrier wait is bounded; a wait that gives up sets the status word's
 // timeout bit, raises a CTA abort flag and the CTA drains and exits.
 #include <cuda_fp16.h>
